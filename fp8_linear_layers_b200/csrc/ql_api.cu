@@ -1,0 +1,290 @@
+// ql_api.cu -- the C ABI of libqlinear.so: argument checks, dispatch, status.
+//
+// Every entry point validates its arguments on the host and returns an error
+// before launching anything; none of them allocates, frees or synchronises
+// (except qlinear_get_device_status, whose job is to synchronise).
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "ql_common.cuh"
+#include "ql_internal.h"
+
+// One status word per device (a __device__ variable exists once per device
+// context); kernels get its address as an argument.
+__device__ ql::DevStatus g_ql_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int major = 0;
+  int minor = 0;
+  ql::DevStatus* status = nullptr;
+};
+
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_devices_mu;
+thread_local char g_last_cuda_error[256] = "";
+
+ql_status cuda_fail(cudaError_t e, const char* where) {
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s (%s)", where,
+                cudaGetErrorName(e), cudaGetErrorString(e));
+  return e == cudaErrorNotSupported ? QL_ERR_UNSUPPORTED_SHAPE : QL_ERR_CUDA;
+}
+
+// Properties of the current device, queried once per device.
+ql_status current_device(DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return QL_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_devices_mu);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.ready) {
+    if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    if ((e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    if ((e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_ql_status)) != cudaSuccess)
+      return cuda_fail(e, "cudaGetSymbolAddress");
+    d.status = static_cast<ql::DevStatus*>(p);
+    d.ready = true;
+  }
+  if (d.major != 10 || d.minor != 0) return QL_ERR_DEVICE;  // built for sm_100a only
+  *out = d;
+  return QL_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_scheme(ql_scheme s) {
+  return s == QL_W8A8_INT8_ROW || s == QL_FP8_E4M3_ROW || s == QL_FP8_E4M3_BLOCK128;
+}
+
+constexpr int64_t kIndexLimit = int64_t(1) << 31;
+
+// Shape rules shared by every entry point.
+ql_status check_k(ql_scheme s, int64_t K) {
+  if (K <= 0) return QL_ERR_INVALID_ARG;
+  if (K % 16) return QL_ERR_UNSUPPORTED_SHAPE;
+  if (s == QL_FP8_E4M3_BLOCK128 && K % 128) return QL_ERR_UNSUPPORTED_SHAPE;
+  if (s == QL_W8A8_INT8_ROW && K > 133144) return QL_ERR_UNSUPPORTED_SHAPE;  // K * 127^2 < 2^31
+  if (s != QL_W8A8_INT8_ROW && K >= 131072) return QL_ERR_UNSUPPORTED_SHAPE;
+  return QL_OK;
+}
+
+ql_status check_n(ql_scheme s, int64_t N, int64_t K) {
+  if (N <= 0) return QL_ERR_INVALID_ARG;
+  if (s == QL_FP8_E4M3_BLOCK128 && N % 128) return QL_ERR_UNSUPPORTED_SHAPE;
+  if (N * K >= kIndexLimit) return QL_ERR_UNSUPPORTED_SHAPE;
+  return QL_OK;
+}
+
+ql_status check_m(int64_t M, int64_t N, int64_t K) {
+  if (M < 0) return QL_ERR_INVALID_ARG;
+  if (M * K >= kIndexLimit || M * N >= kIndexLimit) return QL_ERR_UNSUPPORTED_SHAPE;
+  return QL_OK;
+}
+
+#define QL_TRY(expr)                   \
+  do {                                 \
+    ql_status _s = (expr);             \
+    if (_s != QL_OK) return _s;        \
+  } while (0)
+
+ql_status need(const void* p) {
+  if (!p) return QL_ERR_INVALID_ARG;
+  return aligned16(p) ? QL_OK : QL_ERR_MISALIGNED;
+}
+
+ql_status check_debug(const ql_debug* dbg) {
+  if (!dbg) return QL_OK;
+  const void* ps[4] = {dbg->qx, dbg->sx, dbg->acc_i32, dbg->acc_f32};
+  for (const void* p : ps)
+    if (p && !aligned16(p)) return QL_ERR_MISALIGNED;
+  return QL_OK;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+ql_status qlinear_quantize_weight(ql_scheme scheme, const uint16_t* w, int64_t N, int64_t K,
+                                  void* wq, float* sw, void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_n(scheme, N, K));
+  QL_TRY(need(w));
+  QL_TRY(need(wq));
+  QL_TRY(need(sw));
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  cudaError_t e = ql::launch_quantize_weight(scheme, w, N, K, static_cast<uint8_t*>(wq), sw,
+                                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_quantize_weight");
+}
+
+ql_status qlinear_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, int64_t K,
+                               void* qx, float* sx, void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_m(M, 1, K));
+  if (M == 0) return QL_OK;
+  QL_TRY(need(x));
+  QL_TRY(need(qx));
+  QL_TRY(need(sx));
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  cudaError_t e = ql::launch_quantize_act(scheme, x, M, K, static_cast<uint8_t*>(qx), sx,
+                                          static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_quantize_act");
+}
+
+ql_status qlinear_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
+                       int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg, void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_n(scheme, N, K));
+  if (K > ql::gemv_max_k()) return QL_ERR_UNSUPPORTED_SHAPE;
+  QL_TRY(need(x));
+  QL_TRY(need(wq));
+  QL_TRY(need(sw));
+  QL_TRY(need(y));
+  QL_TRY(check_debug(dbg));
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  cudaError_t e = ql::launch_gemv(scheme, x, wq, sw, N, K, y, dbg, d.sms, d.status,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemv");
+}
+
+ql_status qlinear_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
+                             int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
+                             size_t ws_bytes, const ql_debug* dbg, void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_n(scheme, N, K));
+  QL_TRY(check_m(M, N, K));
+  if (M == 0) return QL_OK;
+  if (M > 32) return QL_ERR_UNSUPPORTED_SHAPE;
+  QL_TRY(need(x));
+  QL_TRY(need(wq));
+  QL_TRY(need(sw));
+  QL_TRY(need(y));
+  QL_TRY(check_debug(dbg));
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  const size_t need_ws = ql::gemm_small_workspace_bytes(scheme, M, N, K, d.sms);
+  if (need_ws && (!workspace || ws_bytes < need_ws)) return QL_ERR_WORKSPACE;
+  if (need_ws && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return QL_ERR_MISALIGNED;
+  cudaError_t e = ql::launch_gemm_small(scheme, x, wq, sw, M, N, K, y, workspace, ws_bytes, dbg,
+                                        d.sms, d.status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm_small");
+}
+
+ql_status qlinear_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
+                       const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                       void* workspace, size_t ws_bytes, const ql_debug* dbg, void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_n(scheme, N, K));
+  QL_TRY(check_m(M, N, K));
+  if (M == 0) return QL_OK;
+  QL_TRY(need(qx));
+  QL_TRY(need(sx));
+  QL_TRY(need(wq));
+  QL_TRY(need(sw));
+  QL_TRY(need(y));
+  QL_TRY(check_debug(dbg));
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  const size_t need_ws = ql::gemm_workspace_bytes(scheme, M, N, K, d.sms);
+  if (need_ws && (!workspace || ws_bytes < need_ws)) return QL_ERR_WORKSPACE;
+  if (need_ws && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return QL_ERR_MISALIGNED;
+  cudaError_t e = ql::launch_gemm(scheme, qx, sx, wq, sw, M, N, K, y, workspace, ws_bytes, dbg,
+                                  d.sms, d.status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm");
+}
+
+size_t qlinear_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K) {
+  DeviceInfo d;
+  if (!valid_scheme(scheme) || M <= 0 || N <= 0 || K <= 0 || current_device(&d) != QL_OK) return 0;
+  if (M <= 32) return ql::gemm_small_workspace_bytes(scheme, M, N, K, d.sms);
+  return ql::gemm_workspace_bytes(scheme, M, N, K, d.sms);
+}
+
+static size_t forward_act_bytes(ql_scheme scheme, int64_t M, int64_t K) {
+  const size_t q = round_up((size_t)(M * K), 256);
+  const size_t s = round_up((size_t)M * (scheme == QL_FP8_E4M3_BLOCK128 ? K / 128 : 1) * 4, 256);
+  return q + s;
+}
+
+size_t qlinear_forward_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K) {
+  DeviceInfo d;
+  if (!valid_scheme(scheme) || M <= 0 || N <= 0 || K <= 0 || current_device(&d) != QL_OK) return 0;
+  if (M == 1 && K <= ql::gemv_max_k()) return 0;
+  if (M <= 32) return ql::gemm_small_workspace_bytes(scheme, M, N, K, d.sms);
+  return forward_act_bytes(scheme, M, K) + ql::gemm_workspace_bytes(scheme, M, N, K, d.sms);
+}
+
+ql_status qlinear_forward(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
+                          int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_m(M, N, K));
+  if (M == 0) return QL_OK;
+  if (M == 1 && K > 0 && K <= ql::gemv_max_k())
+    return qlinear_gemv(scheme, x, wq, sw, N, K, y, nullptr, stream);
+  if (M <= 32)
+    return qlinear_gemm_small(scheme, x, wq, sw, M, N, K, y, workspace, ws_bytes, nullptr, stream);
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_n(scheme, N, K));
+  const size_t act = forward_act_bytes(scheme, M, K);
+  if (!workspace || ws_bytes < act) return QL_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return QL_ERR_MISALIGNED;
+  uint8_t* qx = static_cast<uint8_t*>(workspace);
+  float* sx = reinterpret_cast<float*>(qx + round_up((size_t)(M * K), 256));
+  QL_TRY(qlinear_quantize_act(scheme, x, M, K, qx, sx, stream));
+  uint8_t* rest = static_cast<uint8_t*>(workspace) + act;
+  return qlinear_gemm(scheme, qx, sx, wq, sw, M, N, K, y, ws_bytes > act ? rest : nullptr,
+                      ws_bytes - act, nullptr, stream);
+}
+
+ql_status qlinear_get_device_status(void* stream, uint32_t* detail) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  ql::DevStatus h{0, 0}, zero{0, 0};
+  if ((e = cudaMemcpyFromSymbol(&h, g_ql_status, sizeof(h))) != cudaSuccess)
+    return cuda_fail(e, "cudaMemcpyFromSymbol");
+  if (h.code && (e = cudaMemcpyToSymbol(g_ql_status, &zero, sizeof(zero))) != cudaSuccess)
+    return cuda_fail(e, "cudaMemcpyToSymbol");
+  if (detail) *detail = h.detail;
+  return static_cast<ql_status>(h.code);
+}
+
+const char* qlinear_status_string(ql_status status) {
+  switch (status) {
+    case QL_OK: return "ok";
+    case QL_ERR_INVALID_ARG: return "invalid argument (null pointer, unknown scheme or negative size)";
+    case QL_ERR_UNSUPPORTED_SHAPE: return "shape not supported by this scheme or entry point";
+    case QL_ERR_MISALIGNED: return "device pointer not 16-byte aligned (workspace: 256-byte)";
+    case QL_ERR_CUDA: return "CUDA call failed (see qlinear_last_cuda_error)";
+    case QL_ERR_TIMEOUT: return "a kernel's bounded wait gave up";
+    case QL_ERR_DEVICE: return "no usable sm_100 device is current";
+    case QL_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+const char* qlinear_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

@@ -1,0 +1,59 @@
+// ql_internal.h -- host-side launchers shared between the qlinear translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <type_traits>
+
+#include "../../include/qlinear.h"
+
+namespace ql {
+
+struct DevStatus;
+
+// Raise a kernel's dynamic shared-memory limit once per device (and again only
+// if a larger size is asked for), so launches do not pay for the attribute call.
+template <typename Kernel>
+inline cudaError_t ensure_smem(Kernel kern, int bytes) {
+  static int done[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && __atomic_load_n(&done[dev], __ATOMIC_ACQUIRE) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) {
+    int cur = __atomic_load_n(&done[dev], __ATOMIC_ACQUIRE);
+    while (cur < bytes && !__atomic_compare_exchange_n(&done[dev], &cur, bytes, false,
+                                                        __ATOMIC_ACQ_REL, __ATOMIC_ACQUIRE)) {
+    }
+  }
+  return e;
+}
+
+cudaError_t launch_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, int64_t K,
+                                uint8_t* qx, float* sx, cudaStream_t st);
+cudaError_t launch_quantize_weight(ql_scheme scheme, const uint16_t* w, int64_t N, int64_t K,
+                                   uint8_t* wq, float* sw, cudaStream_t st);
+
+int gemv_max_k();
+cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
+                        int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg, int num_sms,
+                        DevStatus* status, cudaStream_t st);
+
+// Large-M tcgen05 GEMM on pre-quantized activations.
+size_t gemm_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
+                        const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                        void* workspace, size_t ws_bytes, const ql_debug* dbg, int num_sms,
+                        DevStatus* status, cudaStream_t st);
+
+// Small-M (1..32) tensor-core GEMM, K split across the SMs.
+size_t gemm_small_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq,
+                              const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                              void* workspace, size_t ws_bytes, const ql_debug* dbg, int num_sms,
+                              DevStatus* status, cudaStream_t st);
+
+}  // namespace ql

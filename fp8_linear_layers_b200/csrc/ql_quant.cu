@@ -1,0 +1,202 @@
+// ql_quant.cu -- activation and weight quantization kernels.
+//
+// Activations ("Llama 3.1 8B Instruct W8A8", intro and "Loading": inputs
+// rounded to int8 a token at a time; "Meta-Llama-3.1-8B-Instruct-FP8-dynamic"
+// recipe: per-token dynamic symmetric FP8; "Qwen3 8B FP8", "Loading": FP8 128
+// inputs at a time) and weights (the same pages' weight formats: one scale per
+// output row, or one per 128x128 block).
+//
+// Every kernel here is HBM-bound: it reads bf16 once and writes one byte per
+// element.  Absmax reductions are warp shuffles (plus one shared-memory step
+// for a whole row); the scale is one IEEE f32 division and each code one more.
+#include "ql_common.cuh"
+#include "ql_internal.h"
+
+namespace ql {
+
+// Row-wise quantization of [rows, K] bf16: one CTA per row, one scale per row.
+//   kInt8       int8 codes clamp(rne(x/s)) with s = a/127, else E4M3 with s = a/448
+//   kBf16Scale  the scale is rounded to bf16 before use (W8A8 weight scales)
+// Each thread keeps up to kCache 16-byte chunks of the row in registers so the
+// row is read from HBM once; longer rows re-read the remainder from L2.
+template <bool kInt8, bool kBf16Scale, int kThreads, int kCache>
+__global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __restrict__ x,
+                                                              int64_t K, uint8_t* __restrict__ q,
+                                                              float* __restrict__ s_out) {
+  const int64_t row = blockIdx.x;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
+  const int64_t nchunk = K / 8;  // 8 bf16 per 16-byte chunk
+  const int t = threadIdx.x;
+
+  uint4 cache[kCache];
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kCache; ++i) {
+    int64_t c = t + (int64_t)i * kThreads;
+    if (c < nchunk) {
+      cache[i] = __ldg(xr + c);
+      const uint32_t w[4] = {cache[i].x, cache[i].y, cache[i].z, cache[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+    }
+  }
+  for (int64_t c = t + (int64_t)kCache * kThreads; c < nchunk; c += kThreads) {
+    uint4 v = __ldg(xr + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+  }
+
+  __shared__ float red[kThreads / 32];
+  a = warp_max(a);
+  if ((t & 31) == 0) red[t >> 5] = a;
+  __syncthreads();
+  if (t < 32) {
+    float v = (t < kThreads / 32) ? red[t] : 0.0f;
+    v = warp_max(v);
+    if (t == 0) red[0] = v;
+  }
+  __syncthreads();
+  a = red[0];
+  float s = a / (kInt8 ? 127.0f : 448.0f);
+  if (kBf16Scale) s = __uint_as_float((uint32_t)f32_to_bf16_rn(s) << 16);
+  if (t == 0) s_out[row] = s;
+
+  uint2* qr = reinterpret_cast<uint2*>(q + row * K);
+  auto emit = [&](int64_t c, const uint4& v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float f0 = bf16_lo(w[2 * h]), f1 = bf16_hi(w[2 * h]);
+      const float f2 = bf16_lo(w[2 * h + 1]), f3 = bf16_hi(w[2 * h + 1]);
+      if (kInt8) {
+        o[h] = (uint32_t)(int8_code(f0, s) & 0xFF) | ((uint32_t)(int8_code(f1, s) & 0xFF) << 8) |
+               ((uint32_t)(int8_code(f2, s) & 0xFF) << 16) |
+               ((uint32_t)(int8_code(f3, s) & 0xFF) << 24);
+      } else {
+        o[h] = f32x2_to_e4m3x2(e4m3_quotient(f0, s), e4m3_quotient(f1, s)) |
+               (f32x2_to_e4m3x2(e4m3_quotient(f2, s), e4m3_quotient(f3, s)) << 16);
+      }
+    }
+    qr[c] = make_uint2(o[0], o[1]);
+  };
+#pragma unroll
+  for (int i = 0; i < kCache; ++i) {
+    int64_t c = t + (int64_t)i * kThreads;
+    if (c < nchunk) emit(c, cache[i]);
+  }
+  for (int64_t c = t + (int64_t)kCache * kThreads; c < nchunk; c += kThreads) emit(c, __ldg(xr + c));
+}
+
+// Per-(token, 128-group) E4M3 quantization: 16 lanes per group, each lane one
+// 16-byte chunk (8 bf16); the group absmax is a 16-lane shuffle reduction.
+__global__ void __launch_bounds__(256) quant_groups_kernel(const uint16_t* __restrict__ x,
+                                                           int64_t ngroups,
+                                                           uint8_t* __restrict__ q,
+                                                           float* __restrict__ s_out) {
+  const int64_t g = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4);
+  const int lane16 = threadIdx.x & 15;
+  const bool live = g < ngroups;
+  uint4 v = make_uint4(0, 0, 0, 0);
+  // group g covers elements [128 g, 128 g + 128) of the flattened [M, K]
+  // (K is a multiple of 128, so groups never straddle tokens)
+  if (live) v = __ldg(reinterpret_cast<const uint4*>(x + g * 128) + lane16);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float a = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if (!live) return;
+  const float s = a / 448.0f;
+  uint32_t o2[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+    o2[h] = f32x2_to_e4m3x2(e4m3_quotient(bf16_lo(w[2 * h]), s), e4m3_quotient(bf16_hi(w[2 * h]), s)) |
+            (f32x2_to_e4m3x2(e4m3_quotient(bf16_lo(w[2 * h + 1]), s),
+                             e4m3_quotient(bf16_hi(w[2 * h + 1]), s))
+             << 16);
+  reinterpret_cast<uint2*>(q + g * 128)[lane16] = make_uint2(o2[0], o2[1]);
+  if (lane16 == 0) s_out[g] = s;
+}
+
+// 128x128 weight blocks: one CTA per block, 256 threads x 8 chunks of 8 bf16.
+__global__ void __launch_bounds__(256) quant_wblock_kernel(const uint16_t* __restrict__ w,
+                                                           int64_t K, uint8_t* __restrict__ q,
+                                                           float* __restrict__ s_out) {
+  const int64_t KB = K / 128;
+  const int64_t nb = blockIdx.x / KB, kb = blockIdx.x % KB;
+  const int t = threadIdx.x;
+  uint4 v[8];
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = t + i * 256;  // 2048 chunks: 128 rows x 16 chunks
+    const int64_t r = nb * 128 + (c >> 4);
+    v[i] = __ldg(reinterpret_cast<const uint4*>(w + r * K + kb * 128) + (c & 15));
+    const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16_lo(u[j])), fabsf(bf16_hi(u[j]))));
+  }
+  __shared__ float red[8];
+  a = warp_max(a);
+  if ((t & 31) == 0) red[t >> 5] = a;
+  __syncthreads();
+  float m = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
+  const float s = m / 448.0f;
+  if (t == 0) s_out[nb * KB + kb] = s;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = t + i * 256;
+    const int64_t r = nb * 128 + (c >> 4);
+    const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    uint32_t o2[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      o2[h] = f32x2_to_e4m3x2(e4m3_quotient(bf16_lo(u[2 * h]), s), e4m3_quotient(bf16_hi(u[2 * h]), s)) |
+              (f32x2_to_e4m3x2(e4m3_quotient(bf16_lo(u[2 * h + 1]), s),
+                               e4m3_quotient(bf16_hi(u[2 * h + 1]), s))
+               << 16);
+    reinterpret_cast<uint2*>(q + r * K + kb * 128)[c & 15] = make_uint2(o2[0], o2[1]);
+  }
+}
+
+template <bool kInt8, bool kBf16Scale>
+static cudaError_t launch_rows(const uint16_t* x, int64_t rows, int64_t K, uint8_t* q, float* s,
+                               cudaStream_t st) {
+  if (K <= 8 * 8 * 256)
+    quant_rows_kernel<kInt8, kBf16Scale, 256, 8><<<(unsigned)rows, 256, 0, st>>>(x, K, q, s);
+  else
+    quant_rows_kernel<kInt8, kBf16Scale, 512, 8><<<(unsigned)rows, 512, 0, st>>>(x, K, q, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, int64_t K,
+                                uint8_t* qx, float* sx, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  switch (scheme) {
+    case QL_W8A8_INT8_ROW: return launch_rows<true, false>(x, M, K, qx, sx, st);
+    case QL_FP8_E4M3_ROW: return launch_rows<false, false>(x, M, K, qx, sx, st);
+    default: {
+      const int64_t ngroups = M * (K / 128);
+      quant_groups_kernel<<<(unsigned)((ngroups + 15) / 16), 256, 0, st>>>(x, ngroups, qx, sx);
+      return cudaGetLastError();
+    }
+  }
+}
+
+cudaError_t launch_quantize_weight(ql_scheme scheme, const uint16_t* w, int64_t N, int64_t K,
+                                   uint8_t* wq, float* sw, cudaStream_t st) {
+  switch (scheme) {
+    case QL_W8A8_INT8_ROW: return launch_rows<true, true>(w, N, K, wq, sw, st);
+    case QL_FP8_E4M3_ROW: return launch_rows<false, false>(w, N, K, wq, sw, st);
+    default:
+      quant_wblock_kernel<<<(unsigned)((N / 128) * (K / 128)), 256, 0, st>>>(w, K, wq, sw);
+      return cudaGetLastError();
+  }
+}
+
+}  // namespace ql

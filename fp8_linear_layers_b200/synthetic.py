@@ -94,3 +94,28 @@ def make_w(N: int, K: int, seed: int = 0, tag: str = "W", std: float = WEIGHT_ST
 def make_uniform_bits(n: int, seed: int = 0, tag: str = "bits") -> np.ndarray:
     """n uniformly random 32-bit patterns (for codec sweeps)."""
     return _rng(seed, tag).integers(0, 2**32, size=n, dtype=np.uint64).astype(np.uint32)
+
+
+def _torch_gen(seed: int, tag: str, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence([seed, zlib.crc32(tag.encode())]).generate_state(1)[0]))
+    return g
+
+
+def make_x_device(M: int, K: int, seed: int = 0, tag: str = "X", outliers: int = 0,
+                  device="cuda") -> torch.Tensor:
+    """Same recipe as ``make_x`` drawn by torch's generator on ``device`` (for
+    large benchmark inputs); returns a bf16 tensor."""
+    g = _torch_gen(seed, f"{tag}:{M}x{K}", device)
+    x = torch.randn((M, K), generator=g, device=device, dtype=torch.float32)
+    if outliers:
+        cols = torch.randperm(K, generator=g, device=device)[:outliers]
+        x[:, cols] *= OUTLIER_GAIN
+    return x.to(torch.bfloat16)
+
+
+def make_w_device(N: int, K: int, seed: int = 0, tag: str = "W", std: float = WEIGHT_STD,
+                  device="cuda") -> torch.Tensor:
+    """Same recipe as ``make_w`` drawn by torch's generator on ``device``."""
+    g = _torch_gen(seed, f"{tag}:{N}x{K}", device)
+    return (torch.randn((N, K), generator=g, device=device, dtype=torch.float32) * std).to(torch.bfloat16)

@@ -1,0 +1,196 @@
+/*
+ * qlinear.h -- C ABI of libqlinear.so: quantized decoder projections on B200
+ * (sm_100a), Y = (s_x (x) s_w) . (Q(X) . W_q^T).
+ *
+ * Three schemes, as the model pages define them:
+ *   QL_W8A8_INT8_ROW      "Llama 3.1 8B Instruct W8A8", intro and "Loading":
+ *                         int8 weights with one (bf16) scale per output row,
+ *                         inputs rounded to int8 a token at a time, int8
+ *                         products summed in int32.
+ *   QL_FP8_E4M3_ROW       "Meta-Llama-3.1-8B-Instruct-FP8-dynamic" README,
+ *                         "Model Optimizations" and the "Creation" recipe: E4M3
+ *                         weights per output channel (static, symmetric), E4M3
+ *                         activations per token (dynamic, symmetric).
+ *   QL_FP8_E4M3_BLOCK128  "Qwen3 8B FP8", intro and "Loading": E4M3 weights with
+ *                         one scale per 128x128 block (a multiplier), inputs
+ *                         rounded to E4M3 128 inputs at a time; widths must be
+ *                         multiples of 128.
+ *
+ * Numerics (identical in every entry point):
+ *   activation scale  s = absmax / 127 (int8) or absmax / 448 (E4M3), one IEEE
+ *                     f32 division over the token (row schemes) or over each
+ *                     128-wide group of the token (block scheme); an all-zero
+ *                     token or group gets s = 0 and codes 0.
+ *   activation code   q = clamp(rne(x / s), -127, 127) for int8, or the E4M3
+ *                     value nearest x / s (ties to even, saturating at +-448);
+ *                     x / s is an IEEE f32 division.
+ *   weight scale      int8: bf16(absmax_row / 127); E4M3 row: absmax_row / 448;
+ *                     E4M3 block: absmax_block / 448 (f32), block = 128 output
+ *                     rows x 128 input columns.
+ *   epilogue          row schemes: y = bf16_rne(((f32)acc * s_x[m]) * s_w[n]),
+ *                     acc the int32 (int8) or f32 (E4M3) sum over K; block
+ *                     scheme: y = bf16_rne(sum_kb P_kb * s_x[m,kb] * s_w[n/128,kb])
+ *                     with P_kb the f32 sum over the kb-th 128 inputs.
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" must be device (or managed) memory of the
+ *     current CUDA device; "host" pointers are ordinary host memory.  The
+ *     caller owns every buffer; the library never allocates, frees or keeps a
+ *     pointer after the call returns.
+ *   - bf16 tensors are passed as their 16-bit patterns (uint16_t).
+ *   - All matrices are row-major and dense: X / q_x [M,K], W / W_q [N,K]
+ *     (nn.Linear [out, in]), Y [M,N]; row scales s_x [M], s_w [N]; block
+ *     scales s_x [M, K/128], s_w [N/128, K/128].
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     are asynchronous: argument errors are returned before anything is
+ *     launched; launch errors come back as QL_ERR_CUDA; faults inside a kernel
+ *     surface at the caller's next synchronisation.  No entry point
+ *     synchronises except qlinear_get_device_status.
+ *   - Preconditions checked on the host: non-null pointers (unless said
+ *     optional), M >= 0 (M = 0 is a no-op), N > 0, K > 0, K % 16 == 0, every
+ *     device pointer 16-byte aligned, N % 128 == 0 and K % 128 == 0 for the
+ *     block scheme, K <= 133144 for int8 (int32 range of K * 127^2) and
+ *     K < 131072 for E4M3; M >= 1 with no upper limit except int32 indexing
+ *     (M * K and M * N below 2^31).
+ *   - Kernels that wait on a barrier wait a bounded time; if a wait gives up
+ *     the kernel records QL_ERR_TIMEOUT in a device status word and returns
+ *     without finishing its output.  qlinear_get_device_status reads it.
+ */
+#ifndef QLINEAR_H
+#define QLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ql_scheme {
+  QL_W8A8_INT8_ROW = 0,
+  QL_FP8_E4M3_ROW = 1,
+  QL_FP8_E4M3_BLOCK128 = 2
+} ql_scheme;
+
+typedef enum ql_status {
+  QL_OK = 0,
+  QL_ERR_INVALID_ARG = 1,       /* null pointer, bad scheme, negative size        */
+  QL_ERR_UNSUPPORTED_SHAPE = 2, /* a size the scheme or the entry point excludes  */
+  QL_ERR_MISALIGNED = 3,        /* a device pointer not 16-byte aligned           */
+  QL_ERR_CUDA = 4,              /* a CUDA runtime / driver call failed            */
+  QL_ERR_TIMEOUT = 5,           /* a kernel's bounded wait gave up                */
+  QL_ERR_DEVICE = 6,            /* no usable sm_100 device is current             */
+  QL_ERR_WORKSPACE = 7          /* workspace missing or smaller than required     */
+} ql_status;
+
+/* Optional capture of intermediate values for bit-exact checks; pass NULL in
+ * production.  Each member may be NULL.  All are device pointers, 16-byte
+ * aligned, owned by the caller. */
+typedef struct ql_debug {
+  void* qx;         /* [M,K] bytes: the activation codes the kernel multiplied */
+  float* sx;        /* [M] or [M,K/128]: the activation scales it used        */
+  int32_t* acc_i32; /* [M,N]: int32 accumulators before the epilogue (int8)   */
+  float* acc_f32;   /* [M,N]: f32 accumulators before the epilogue (E4M3 row) */
+} ql_debug;
+
+/* ---------------------------------------------------------------------- */
+
+/* Weight quantization (offline, checkpoint side), on the GPU.
+ * Pages: W8A8 intro (int8, one bf16 scale per output row); FP8-dynamic README
+ * "Model Optimizations" / recipe (E4M3, per channel, static, symmetric); Qwen3
+ * FP8 intro (E4M3, one multiplier per 128x128 block).
+ *   w    device, bf16 [N,K]
+ *   wq   device, out: [N,K] int8 or E4M3 bytes
+ *   sw   device, out: f32 [N] (row schemes; the int8 scale holds a bf16 value)
+ *        or [N/128, K/128] (block scheme)
+ * Errors: argument checks as above. */
+ql_status qlinear_quantize_weight(ql_scheme scheme, const uint16_t* w, int64_t N, int64_t K,
+                                  void* wq, float* sw, void* stream);
+
+/* Dynamic activation quantization (a per-token or per-128-group absmax by warp
+ * shuffles, the scale, the rounded codes).  Pages: W8A8 intro and "Loading"
+ * ("rounded to int8 a token at a time"); FP8-dynamic recipe (per token,
+ * dynamic, symmetric); Qwen3 FP8 "Loading" ("rounded to FP8 128 inputs at a
+ * time").
+ *   x    device, bf16 [M,K]
+ *   qx   device, out: [M,K] codes
+ *   sx   device, out: f32 [M] (row schemes) or [M, K/128] (block scheme) */
+ql_status qlinear_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, int64_t K,
+                               void* qx, float* sx, void* stream);
+
+/* M = 1 decode product, activation quantization fused: one kernel streams
+ * each weight byte once.  Pages: W8A8 "Loading" ("one row in a kernel that
+ * reads each byte once"); Qwen3 FP8 "Loading" (same, FP8).
+ *   x    device, bf16 [1,K]
+ *   wq   device, [N,K] codes from qlinear_quantize_weight (or a checkpoint)
+ *   sw   device, weight scales as produced by qlinear_quantize_weight
+ *   y    device, out: bf16 [1,N]
+ *   dbg  optional (NULL): captures q_x, s_x and, for int8, acc_i32 / for E4M3
+ *        row, acc_f32 ([1,N]) */
+ql_status qlinear_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
+                       int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg, void* stream);
+
+/* 2 <= M <= 32 product on the tensor cores (tcgen05, tokens on the MMA N side,
+ * weights on the 128-row side, K split across the SMs).  Pages: W8A8
+ * "Loading" ("up to 32 rows on tensor cores"); Qwen3 FP8 "Loading" (same).
+ * Activation quantization runs in the same call (a short quantize pass
+ * overlapped with the weight stream by programmatic dependent launch).
+ *   x          device, bf16 [M,K]
+ *   workspace  device, at least qlinear_workspace_bytes(scheme, M, N, K)
+ *              bytes, 256-byte aligned, ZERO-FILLED before its first use; a
+ *              call that completes leaves it zero-filled again (after a
+ *              QL_ERR_TIMEOUT, zero it again).  Two calls in flight at the
+ *              same time must not share a workspace.
+ *   dbg        optional (NULL): q_x, s_x, acc_i32 (int8) / acc_f32 (E4M3 row) */
+ql_status qlinear_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
+                             int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
+                             size_t ws_bytes, const ql_debug* dbg, void* stream);
+
+/* Large-M product on pre-quantized activations (tcgen05 kind::i8 into int32
+ * TMEM accumulators, or kind::f8f6f4 E4M3 into f32; TMA-fed shared-memory
+ * ring; the scale epilogue fused; for the block scheme each 128-wide K block
+ * is promoted into f32 registers with its two scales).  Pages: W8A8 "Loading"
+ * ("longer inputs rounded to int8 a row at a time and multiplied in int8 ...
+ * summing in int32"); Qwen3 FP8 "Loading" (block scales).
+ *   qx, sx     device, from qlinear_quantize_act
+ *   workspace  device, qlinear_workspace_bytes(...) bytes (may be 0 / NULL
+ *              when that returns 0), same rules as qlinear_gemm_small
+ *   dbg        optional (NULL): acc_i32 (int8) / acc_f32 (E4M3 row) [M,N] */
+ql_status qlinear_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
+                       const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                       void* workspace, size_t ws_bytes, const ql_debug* dbg, void* stream);
+
+/* The projection as a model calls it: bf16 X in, bf16 Y out, dispatching on
+ * the token count the way the pages' "Loading" sections describe: M = 1 ->
+ * qlinear_gemv, 2..32 -> qlinear_gemm_small, > 32 -> qlinear_quantize_act
+ * into the workspace, then qlinear_gemm.
+ *   workspace  device, qlinear_forward_workspace_bytes(scheme, M, N, K) bytes,
+ *              zero-filled before first use (as for qlinear_gemm_small). */
+ql_status qlinear_forward(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
+                          int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/* Workspace sizes (bytes) for the current device; 0 means none is needed.
+ * qlinear_workspace_bytes covers qlinear_gemm_small (2 <= M <= 32) and
+ * qlinear_gemm (M > 32); qlinear_forward_workspace_bytes adds the quantized
+ * activations qlinear_forward keeps there for M > 32. */
+size_t qlinear_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K);
+size_t qlinear_forward_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K);
+
+/* Synchronises `stream`, then reads and clears the device status word that
+ * kernels set when a bounded wait gives up.  Returns QL_OK, QL_ERR_TIMEOUT
+ * (with *detail, if non-NULL, naming the kernel and the wait site), or
+ * QL_ERR_CUDA if the synchronisation itself failed. */
+ql_status qlinear_get_device_status(void* stream, uint32_t* detail);
+
+/* Static description of a status code. */
+const char* qlinear_status_string(ql_status status);
+
+/* The CUDA error text behind the most recent QL_ERR_CUDA on this thread. */
+const char* qlinear_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLINEAR_H */

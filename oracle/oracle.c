@@ -148,9 +148,18 @@ int32_t oracle_int8_round(float t) {
 
 /* E4M3 code -> exact integer in units of 2^-9 (every finite E4M3 value is an
  * integer multiple of 2^-9 of magnitude at most 448 * 2^9 = 229376). */
+static int64_t e4m3_units_table[256];
+static int e4m3_units_ready = 0;
+
 static int64_t e4m3_units(uint8_t c) {
-  double v = oracle_e4m3_decode(c);
-  return (int64_t)ldexp(v, 9);
+  if (!e4m3_units_ready) { /* filled once from the decoder above */
+    for (int i = 0; i < 256; ++i) {
+      double v = oracle_e4m3_decode((uint8_t)i);
+      e4m3_units_table[i] = isnan(v) ? 0 : (int64_t)ldexp(v, 9);
+    }
+    e4m3_units_ready = 1;
+  }
+  return e4m3_units_table[c];
 }
 
 /* ------------------------------------------------------------------------ */

@@ -1,0 +1,82 @@
+"""The C ABI library: it loads without a GPU, exports every function the header
+declares, and rejects bad arguments on the host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp8_linear_layers_b200 as ql
+from fp8_linear_layers_b200 import build as qbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlinear.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    qbuild.build()
+    return ql.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlinear_\w+)\s*\(", text)))
+
+
+def test_header_declarations_match_binding():
+    assert _declared() == sorted(ql.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code in range(8):
+        assert L.qlinear_status_string(code)
+    assert L.qlinear_status_string(99) == b"unknown status"
+
+
+ALIGNED = 0x10000  # a fake, 16-byte aligned address: never dereferenced on these paths
+
+
+def test_host_validation_rejects_before_launch(L):
+    INV, SHAPE, MIS = 1, 2, 3
+    # unknown scheme, null pointers, misaligned pointers
+    assert L.qlinear_gemv(7, ALIGNED, ALIGNED, ALIGNED, 64, 64, ALIGNED, None, None) == INV
+    assert L.qlinear_gemv(0, None, ALIGNED, ALIGNED, 64, 64, ALIGNED, None, None) == INV
+    assert L.qlinear_gemv(0, ALIGNED + 2, ALIGNED, ALIGNED, 64, 64, ALIGNED, None, None) == MIS
+    # K must be a multiple of 16; block scheme needs multiples of 128
+    assert L.qlinear_gemv(0, ALIGNED, ALIGNED, ALIGNED, 64, 40, ALIGNED, None, None) == SHAPE
+    assert L.qlinear_gemv(2, ALIGNED, ALIGNED, ALIGNED, 64, 256, ALIGNED, None, None) == SHAPE
+    assert L.qlinear_gemv(2, ALIGNED, ALIGNED, ALIGNED, 128, 192, ALIGNED, None, None) == SHAPE
+    assert L.qlinear_quantize_act(2, ALIGNED, 4, 200, ALIGNED, ALIGNED, None) == SHAPE
+    assert L.qlinear_quantize_weight(2, ALIGNED, 100, 128, ALIGNED, ALIGNED, None) == SHAPE
+    # int8 accumulators are int32: K * 127^2 must stay below 2^31
+    assert L.qlinear_gemm(0, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 64, 64, 133152, ALIGNED, None, 0,
+                          None, None) == SHAPE
+    # negative sizes, and the small-M path's token limit
+    assert L.qlinear_quantize_act(0, ALIGNED, -1, 64, ALIGNED, ALIGNED, None) == INV
+    assert L.qlinear_gemm_small(0, ALIGNED, ALIGNED, ALIGNED, 33, 64, 64, ALIGNED, ALIGNED, 1 << 20,
+                                None, None) == SHAPE
+    # M = 0 is a no-op that succeeds without a device
+    assert L.qlinear_quantize_act(0, None, 0, 64, None, None, None) == 0
+    assert L.qlinear_forward(0, None, None, None, 0, 64, 64, None, None, 0, None) == 0
+
+
+def test_no_code_shared_between_oracle_and_product():
+    """The product never imports or links the oracle, and the oracle never
+    includes the product's headers."""
+    pkg = os.path.join(ROOT, "fp8_linear_layers_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", src, re.M), f
+                assert "oracle" not in src or f.endswith(".py") and "oracle" not in re.sub(
+                    r"(#.*|\"\"\"[\s\S]*?\"\"\")", "", src), f
+    osrc = open(os.path.join(ROOT, "oracle", "oracle.c")).read()
+    assert "#include \"" not in osrc and "qlinear" not in osrc.split("*/", 1)[1]
