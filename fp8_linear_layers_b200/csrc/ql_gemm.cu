@@ -1,12 +1,414 @@
-// ql_gemm.cu -- large-M tcgen05 GEMM (being written).
-#include "ql_common.cuh"
+// ql_gemm.cu -- large-M product on pre-quantized activations, tcgen05 + TMA.
+//
+// "Llama 3.1 8B Instruct W8A8", "Loading": longer inputs are rounded to int8 a
+// row at a time and multiplied in int8, summing in int32.  "Qwen3 8B FP8",
+// "Loading": longer inputs rounded to FP8 128 inputs at a time and multiplied
+// with block scales.  Here:
+//   acc[m,n] = sum_k q_x[m,k] q_w[n,k]       tcgen05.mma kind::i8  -> s32 TMEM
+//                                            tcgen05.mma kind::f8f6f4 (E4M3) -> f32 TMEM
+//   y[m,n]   = bf16(((f32)acc * s_x[m]) * s_w[n])                (row schemes)
+//   y[m,n]   = bf16(sum_kb P_kb[m,n] * s_x[m,kb] * s_w[n/128,kb])  (block scheme:
+//              each 128-deep partial P_kb gets its own TMEM buffer and is
+//              promoted into f32 registers by the epilogue warps)
+//
+// Persistent CTAs (one per SM), 128 x BN output tiles, warp roles:
+//   warp 0      TMA producer: A = q_x [128 x 128 B] and B = W_q [BN x 128 B]
+//               tiles into a 4..6-stage shared-memory ring (128-byte swizzle)
+//   warp 1      TMEM allocation and the single MMA-issuing thread: 4 MMAs of
+//               K = 32 per stage, tcgen05.commit releases the stage
+//   warps 2..9  epilogue: tcgen05.ld from TMEM, scales, bf16, global stores;
+//               two TMEM accumulators (or per-K-block buffers) let the
+//               epilogue of one tile overlap the MMAs of the next
+// Every mbarrier wait is bounded; on a timeout the kernel records it, drains
+// its own copies and MMAs, frees TMEM and returns.
+#include "ql_tc.cuh"
 #include "ql_internal.h"
 
 namespace ql {
-size_t gemm_workspace_bytes(ql_scheme, int64_t, int64_t, int64_t, int) { return 0; }
-cudaError_t launch_gemm(ql_scheme, const void*, const float*, const void*, const float*, int64_t,
-                        int64_t, int64_t, uint16_t*, void*, size_t, const ql_debug*, int,
-                        DevStatus*, cudaStream_t) {
-  return cudaErrorNotSupported;
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 128;  // bytes of K per stage: one 128-byte swizzle row
+constexpr int kGemmEpiWarps = 8;
+constexpr int kGemmThreads = 64 + kGemmEpiWarps * 32;
+constexpr int kTmemCols = 512;
+constexpr int kGemmSmemBudget = 200 * 1024;
+
+struct GemmParams {
+  const float* sx;
+  const float* sw;
+  uint16_t* y;
+  int M, N, K;
+  int mt, nt, nkb;  // tiles along M and N, K blocks of 128
+  int32_t* acc_i32;
+  float* acc_f32;
+  DevStatus* status;
+};
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStageA = kGemmBM * kGemmBK;
+  static constexpr int kStageB = BN * kGemmBK;
+  static constexpr int kStage = kStageA + kStageB;
+  static constexpr int kStages = (kGemmSmemBudget / kStage) > 8 ? 8 : (kGemmSmemBudget / kStage);
+  static constexpr int kRing = kStages * kStage;
+  static constexpr int kBufCols = BN <= 128 ? 128 : 256;  // TMEM columns per accumulator
+  static constexpr int kBufs = kTmemCols / kBufCols;
+  static constexpr int kHalf = BN / 2;                    // columns per epilogue warp
+  static constexpr int kSmem = kRing + 1024 + 256;
+  static_assert(BN % 64 == 0 && BN <= 256, "tile N");
+  static_assert(kStage % 1024 == 0, "stages must stay 1024-byte aligned");
+};
+
+QL_DEVINL uint8_t* align1024(uint8_t* p) {
+  const uint32_t a = smem_u32(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
 }
+
+// Store 32 consecutive bf16 outputs of row m starting at column n.
+QL_DEVINL void store_row32(uint16_t* __restrict__ y, int64_t m, int n, int N, const float* v) {
+  uint16_t* dst = y + m * (int64_t)N + n;
+  if (n + 32 <= N && (N & 7) == 0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        w[j] = (uint32_t)f32_to_bf16_rn(v[8 * q + 2 * j]) |
+               ((uint32_t)f32_to_bf16_rn(v[8 * q + 2 * j + 1]) << 16);
+      reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (n + j < N) dst[j] = f32_to_bf16_rn(v[j]);
+  }
+}
+
+template <ql_scheme S, int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmParams p) {
+  using Cfg = GemmCfg<BN>;
+  constexpr bool kInt8 = S == QL_W8A8_INT8_ROW;
+  constexpr bool kBlock = S == QL_FP8_E4M3_BLOCK128;
+  constexpr uint32_t kIdesc = tc::idesc(kInt8, kGemmBM, BN);
+  constexpr int kStages = Cfg::kStages;
+  constexpr int kBufs = Cfg::kBufs;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + Cfg::kRing);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + kBufs;
+  uint64_t* mma_done = tempty + kBufs;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = p.mt * p.nt;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < kBufs; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kGemmEpiWarps);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tc::prefetch_tmap(&tmA);
+    tc::prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_holder, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_a = l2_policy_evict_last();   // q_x: re-read by every N tile
+      const uint64_t pol_b = l2_policy_evict_first();  // W_q: read by the few M tiles at once
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const int m0 = (t % p.mt) * kGemmBM, n0 = (t / p.mt) * BN;
+        for (int kb = 0; kb < p.nkb; ++kb, ++it) {
+          const int s = it % kStages;
+          if (it >= (uint32_t)kStages &&
+              !mbar_wait_bounded(&empty[s], ((it / kStages) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = ring + s * Cfg::kStage;
+          mbar_arrive_expect_tx(&full[s], Cfg::kStage);
+          tc::tma_load_2d(st, &tmA, kb * kGemmBK, m0, &full[s], pol_a);
+          tc::tma_load_2d(st + Cfg::kStageA, &tmB, kb * kGemmBK, n0, &full[s], pol_b);
+        }
+      }
+      if (!ok) {
+        if (!*abort_flag) record_timeout(p.status, KID_GEMM, 1);
+        *abort_flag = 1;
+      }
+      // no copy may still be landing in shared memory when the CTA exits
+      for (uint32_t j = it > (uint32_t)kStages ? it - kStages : 0; j < it; ++j)
+        mbar_wait_bounded(&full[j % kStages], (j / kStages) & 1, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, jt = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        uint32_t d = 0;
+        if (!kBlock) {
+          const uint32_t buf = jt % kBufs;
+          if (jt >= (uint32_t)kBufs &&
+              !mbar_wait_bounded(&tempty[buf], ((jt / kBufs) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after();
+          d = tmem + buf * Cfg::kBufCols;
+        }
+        for (int kb = 0; kb < p.nkb; ++kb, ++it) {
+          if (kBlock) {
+            const uint32_t buf = jt % kBufs;
+            if (jt >= (uint32_t)kBufs &&
+                !mbar_wait_bounded(&tempty[buf], ((jt / kBufs) - 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc::fence_after();
+            d = tmem + buf * Cfg::kBufCols;
+          }
+          const int s = it % kStages;
+          if (!mbar_wait_bounded(&full[s], (it / kStages) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after();
+          const uint32_t a_addr = smem_u32(ring + s * Cfg::kStage);
+          const uint64_t adesc = tc::sw128_desc(a_addr);
+          const uint64_t bdesc = tc::sw128_desc(a_addr + Cfg::kStageA);
+#pragma unroll
+          for (int k = 0; k < kGemmBK / 32; ++k)
+            tc::mma<kInt8>(d, adesc + 2 * k, bdesc + 2 * k, kIdesc,
+                           kBlock ? (k != 0) : ((kb | k) != 0));
+          tc::commit(&empty[s]);  // the stage is free once these MMAs have read it
+          if (kBlock) {
+            tc::commit(&tfull[jt % kBufs]);
+            ++jt;
+          }
+        }
+        if (!ok) break;
+        if (!kBlock) {
+          tc::commit(&tfull[jt % kBufs]);
+          ++jt;
+        }
+      }
+      if (!ok) {
+        if (!*abort_flag) record_timeout(p.status, KID_GEMM, 2);
+        *abort_flag = 1;
+      }
+      tc::commit(mma_done);  // every MMA of this CTA has finished when this completes
+      mbar_wait_bounded(mma_done, 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int q = warp & 3;   // TMEM lane quarter this warp may access
+    const int h = ew >> 2;    // which half of the tile's columns
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const int KB = p.K / 128;
+    uint32_t jt = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      const int m0 = (t % p.mt) * kGemmBM, n0 = (t / p.mt) * BN;
+      const int m = m0 + q * 32 + lane;
+      const bool live_m = m < p.M;
+      const int c0 = h * Cfg::kHalf;  // first column of this warp inside the tile
+      if constexpr (!kBlock) {
+        const uint32_t buf = jt % kBufs;
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kBufs) & 1, abort_flag));
+        if (!ok) break;
+        tc::fence_after();
+        const float sxm = live_m ? __ldg(p.sx + m) : 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < Cfg::kHalf / 32; ++c) {
+          const int col = c0 + c * 32;
+          uint32_t r[32];
+          tc::ld32(tmem + lane_base + buf * Cfg::kBufCols + col, r);
+          tc::ld_wait();
+          const int n = n0 + col;
+          if (live_m && n < p.N) {
+            float v[32];
+            if (n + 32 <= p.N) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 4) {
+                const float4 s4 = __ldg(reinterpret_cast<const float4*>(p.sw + n + j));
+                const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const float a = kInt8 ? __int2float_rn((int)r[j + u]) : __uint_as_float(r[j + u]);
+                  v[j + u] = __fmul_rn(__fmul_rn(a, sxm), sv[u]);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const float a = kInt8 ? __int2float_rn((int)r[j]) : __uint_as_float(r[j]);
+                v[j] = (n + j < p.N) ? __fmul_rn(__fmul_rn(a, sxm), __ldg(p.sw + n + j)) : 0.0f;
+              }
+            }
+            if (p.acc_i32 || p.acc_f32) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (n + j < p.N) {
+                  if (kInt8 && p.acc_i32) p.acc_i32[(int64_t)m * p.N + n + j] = (int)r[j];
+                  if (!kInt8 && p.acc_f32) p.acc_f32[(int64_t)m * p.N + n + j] = __uint_as_float(r[j]);
+                }
+              }
+            }
+            store_row32(p.y, m, n, p.N, v);
+          }
+        }
+        tc::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+        ++jt;
+      } else {
+        // block scheme: promote each 128-deep partial into f32 registers
+        const int ncol = n0 + c0;
+        const bool live_n = ncol < p.N;
+        const int nbw = ncol >> 7;  // this warp's columns lie in one 128-row weight block
+        float acc[Cfg::kHalf];
+#pragma unroll
+        for (int j = 0; j < Cfg::kHalf; ++j) acc[j] = 0.0f;
+        for (int kb = 0; kb < p.nkb; ++kb) {
+          const uint32_t buf = jt % kBufs;
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kBufs) & 1, abort_flag));
+          if (!ok) break;
+          tc::fence_after();
+          const float scale = (live_m && live_n)
+                                  ? __ldg(p.sx + (int64_t)m * KB + kb) * __ldg(p.sw + (int64_t)nbw * KB + kb)
+                                  : 0.0f;
+#pragma unroll
+          for (int c = 0; c < Cfg::kHalf / 32; ++c) {
+            uint32_t r[32];
+            tc::ld32(tmem + lane_base + buf * Cfg::kBufCols + c0 + c * 32, r);
+            tc::ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(__uint_as_float(r[j]), scale, acc[c * 32 + j]);
+          }
+          tc::fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+          ++jt;
+        }
+        if (!ok) break;
+        if (live_m && live_n) {
+#pragma unroll
+          for (int c = 0; c < Cfg::kHalf / 32; ++c) store_row32(p.y, m, ncol + c * 32, p.N, &acc[c * 32]);
+        }
+      }
+    }
+    if (!ok) {
+      if (lane == 0 && !*abort_flag) record_timeout(p.status, KID_GEMM, 3);
+      *abort_flag = 1;
+    }
+  }
+
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+size_t gemm_workspace_bytes(ql_scheme, int64_t, int64_t, int64_t, int) { return 0; }
+
+// Tile width for this shape: fill the SMs' waves best, 128-wide tiles taxed
+// for their higher shared-memory read rate per MMA.
+static int pick_bn(ql_scheme s, int64_t M, int64_t N, int sms) {
+  const int cands_row[3] = {256, 192, 128};
+  const int cands_blk[2] = {256, 128};
+  const int* c = s == QL_FP8_E4M3_BLOCK128 ? cands_blk : cands_row;
+  const int nc = s == QL_FP8_E4M3_BLOCK128 ? 2 : 3;
+  const int64_t mt = (M + kGemmBM - 1) / kGemmBM;
+  int best = c[0];
+  double best_eff = -1.0;
+  for (int i = 0; i < nc; ++i) {
+    const int64_t tiles = mt * ((N + c[i] - 1) / c[i]);
+    const int64_t waves = (tiles + sms - 1) / sms;
+    double eff = (double)(mt * N) / (double)(waves * sms * (int64_t)kGemmBM * c[i] / kGemmBM);
+    if (c[i] == 128) eff *= 0.85;
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = c[i];
+    }
+  }
+  return best;
+}
+
+template <ql_scheme S, int BN>
+static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
+                                 int sms, cudaStream_t st) {
+  using Cfg = GemmCfg<BN>;
+  cudaError_t e = ensure_smem<gemm_kernel<S, BN>>(Cfg::kSmem);
+  if (e != cudaSuccess) return e;
+  const int grid = (int)std::min<int64_t>((int64_t)p.mt * p.nt, sms);
+  gemm_kernel<S, BN><<<grid, kGemmThreads, Cfg::kSmem, st>>>(a, b, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
+                        const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y, void*,
+                        size_t, const ql_debug* dbg, int num_sms, DevStatus* status,
+                        cudaStream_t st) {
+  const int BN = pick_bn(scheme, M, N, num_sms);
+  GemmParams p;
+  p.sx = sx;
+  p.sw = sw;
+  p.y = y;
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.mt = (int)((M + kGemmBM - 1) / kGemmBM);
+  p.nt = (int)((N + BN - 1) / BN);
+  p.nkb = (int)((K + kGemmBK - 1) / kGemmBK);
+  p.acc_i32 = dbg ? dbg->acc_i32 : nullptr;
+  p.acc_f32 = dbg ? dbg->acc_f32 : nullptr;
+  p.status = status;
+  CUtensorMap ta, tb;
+  cudaError_t e = make_tmap_u8_sw128(&ta, qx, (uint64_t)K, (uint64_t)M, (uint64_t)K, kGemmBK, kGemmBM);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_u8_sw128(&tb, wq, (uint64_t)K, (uint64_t)N, (uint64_t)K, kGemmBK, (uint32_t)BN);
+  if (e != cudaSuccess) return e;
+  switch (scheme) {
+    case QL_W8A8_INT8_ROW:
+      if (BN == 256) return launch_gemm_t<QL_W8A8_INT8_ROW, 256>(p, ta, tb, num_sms, st);
+      if (BN == 192) return launch_gemm_t<QL_W8A8_INT8_ROW, 192>(p, ta, tb, num_sms, st);
+      return launch_gemm_t<QL_W8A8_INT8_ROW, 128>(p, ta, tb, num_sms, st);
+    case QL_FP8_E4M3_ROW:
+      if (BN == 256) return launch_gemm_t<QL_FP8_E4M3_ROW, 256>(p, ta, tb, num_sms, st);
+      if (BN == 192) return launch_gemm_t<QL_FP8_E4M3_ROW, 192>(p, ta, tb, num_sms, st);
+      return launch_gemm_t<QL_FP8_E4M3_ROW, 128>(p, ta, tb, num_sms, st);
+    default:
+      if (BN == 256) return launch_gemm_t<QL_FP8_E4M3_BLOCK128, 256>(p, ta, tb, num_sms, st);
+      return launch_gemm_t<QL_FP8_E4M3_BLOCK128, 128>(p, ta, tb, num_sms, st);
+  }
+}
+
 }  // namespace ql

@@ -1,12 +1,464 @@
-// ql_gemm_small.cu -- small-M tcgen05 GEMM (being written).
-#include "ql_common.cuh"
+// ql_gemm_small.cu -- 1 <= M <= 32 tokens on the tensor cores (tcgen05).
+//
+// "Llama 3.1 8B Instruct W8A8", "Loading": "up to 32 rows on tensor cores";
+// "Qwen3 8B FP8", "Loading": the same for the FP8 block scheme.  With at most
+// 32 tokens the product is still bound by the weight stream (<= 64 ops per
+// weight byte), so the design spreads W_q evenly over every SM:
+//
+//  * swap-AB: the MMA's 128-row A side is a 128-row tile of W_q, the tokens
+//    are its N side (16 or 32 columns); one MMA is 128 x NTOK x 32.
+//  * the W_q stream is cut into units of (128 weight rows x 128 bytes of K);
+//    CTA c owns the contiguous units [c U / G, (c+1) U / G), so every SM
+//    streams the same number of bytes.  A run of units inside one 128-row
+//    tile accumulates in TMEM; a tile that was split between CTAs is summed
+//    by the CTA that finishes last (an atomic arrival counter, no waiting),
+//    in a fixed contributor order, from per-CTA partial slots.
+//  * activation quantization runs first as its own short kernel writing q_x
+//    and s_x into the workspace; this kernel is launched with programmatic
+//    dependent launch, starts its weight loads at once and waits for the
+//    quantized tokens only before loading them.
+//
+// Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2..5
+// epilogue (one TMEM lane = one weight row per thread).  Every mbarrier wait is
+// bounded.
+#include "ql_tc.cuh"
 #include "ql_internal.h"
 
 namespace ql {
-size_t gemm_small_workspace_bytes(ql_scheme, int64_t, int64_t, int64_t, int) { return 0; }
-cudaError_t launch_gemm_small(ql_scheme, const uint16_t*, const void*, const float*, int64_t,
-                              int64_t, int64_t, uint16_t*, void*, size_t, const ql_debug*, int,
-                              DevStatus*, cudaStream_t) {
-  return cudaErrorNotSupported;
+
+constexpr int kSmallEpiWarps = 4;
+constexpr int kSmallThreads = 64 + kSmallEpiWarps * 32;
+constexpr int kSmallTmemCols = 128;
+constexpr int kSmallBufs = 4;  // TMEM accumulators of 32 columns
+constexpr int kSmallBufCols = 32;
+constexpr uint32_t kSmallEpiBar = 1;
+
+template <int NTOK>
+struct SmallCfg {
+  static constexpr int kStageA = 128 * 128;
+  static constexpr int kStageB = NTOK * 128;
+  static constexpr int kStage = kStageA + kStageB;
+  static constexpr int kStages = (200 * 1024 / kStage) > 12 ? 12 : (200 * 1024 / kStage);
+  static constexpr int kRing = kStages * kStage;
+  static constexpr int kSmem = kRing + 1024 + 512;
+  static_assert(kStage % 1024 == 0, "stage alignment");
+};
+
+struct SmallParams {
+  const float* sx;  // workspace: [M] or [M, K/128]
+  const float* sw;
+  uint16_t* y;
+  int M, N, K;
+  int ntn;          // 128-row tiles of W_q
+  int nkb;          // 128-byte K blocks
+  int units;        // ntn * nkb
+  float* partials;  // [G][2][NTOK][128] 32-bit partial sums
+  unsigned* counters;  // [ntn], zero between calls
+  int32_t* acc_i32;
+  float* acc_f32;
+  DevStatus* status;
+};
+
+// OR vote over the epilogue warps that doubles as their barrier.
+QL_DEVINL bool epi_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(kSmallEpiBar), "r"(kSmallEpiWarps * 32)
+      : "memory");
+  return r != 0;
 }
+
+// First unit of CTA c, and the CTA that owns unit u, under the even split.
+QL_DEVINL int unit_begin(int c, int U, int G) { return (int)(((int64_t)c * U) / G); }
+QL_DEVINL int unit_owner(int u, int U, int G) { return (int)((((int64_t)u + 1) * G - 1) / U); }
+
+template <ql_scheme S, int NTOK>
+__global__ void __launch_bounds__(kSmallThreads, 1)
+    gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                      const SmallParams p) {
+  using Cfg = SmallCfg<NTOK>;
+  constexpr bool kInt8 = S == QL_W8A8_INT8_ROW;
+  constexpr bool kBlock = S == QL_FP8_E4M3_BLOCK128;
+  constexpr uint32_t kIdesc = tc::idesc(kInt8, 128, NTOK);
+  constexpr int kStages = Cfg::kStages;
+  using Acc = typename std::conditional<kInt8, int, float>::type;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + Cfg::kRing);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + kSmallBufs;
+  uint64_t* mma_done = tempty + kSmallBufs;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* last_flag = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int u0 = unit_begin(c, p.units, G), u1 = unit_begin(c + 1, p.units, G);
+  const int nkb = p.nkb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < kSmallBufs; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kSmallEpiWarps);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tc::prefetch_tmap(&tmW);
+    tc::prefetch_tmap(&tmX);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_holder, kSmallTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_last();
+      const int n = u1 - u0;
+      const int pre = n < kStages ? n : kStages;
+      // weights first: they do not depend on the quantization kernel
+      for (int j = 0; j < pre; ++j) {
+        const int u = u0 + j;
+        mbar_arrive_expect_tx(&full[j], Cfg::kStage);
+        tc::tma_load_2d(ring + j * Cfg::kStage, &tmW, (u % nkb) * 128, (u / nkb) * 128, &full[j], pol_w);
+      }
+      tc::grid_dependency_wait();  // q_x is written by the preceding kernel
+      for (int j = 0; j < pre; ++j) {
+        const int u = u0 + j;
+        tc::tma_load_2d(ring + j * Cfg::kStage + Cfg::kStageA, &tmX, (u % nkb) * 128, 0, &full[j], pol_x);
+      }
+      int issued = pre;
+      for (int j = pre; j < n; ++j) {
+        const int s = j % kStages;
+        if (!mbar_wait_bounded(&empty[s], ((j / kStages) - 1) & 1, abort_flag)) {
+          if (!*abort_flag) record_timeout(p.status, KID_GEMM_SMALL, 1);
+          *abort_flag = 1;
+          break;
+        }
+        const int u = u0 + j;
+        uint8_t* st = ring + s * Cfg::kStage;
+        mbar_arrive_expect_tx(&full[s], Cfg::kStage);
+        tc::tma_load_2d(st, &tmW, (u % nkb) * 128, (u / nkb) * 128, &full[s], pol_w);
+        tc::tma_load_2d(st + Cfg::kStageA, &tmX, (u % nkb) * 128, 0, &full[s], pol_x);
+        issued = j + 1;
+      }
+      for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
+        mbar_wait_bounded(&full[j % kStages], (j / kStages) & 1, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t jt = 0;
+      bool ok = true;
+      int j = 0;  // unit index inside this CTA's range
+      for (int u = u0; u < u1 && ok;) {
+        const int t = u / nkb;
+        const int seg_end = min(u1, (t + 1) * nkb);
+        uint32_t d = 0;
+        for (int v = u; v < seg_end; ++v, ++j) {
+          const bool first_of_seg = v == u;
+          if (kBlock || first_of_seg) {
+            const uint32_t buf = jt % kSmallBufs;
+            if (jt >= (uint32_t)kSmallBufs &&
+                !mbar_wait_bounded(&tempty[buf], ((jt / kSmallBufs) - 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc::fence_after();
+            d = tmem + buf * kSmallBufCols;
+          }
+          const int s = j % kStages;
+          if (!mbar_wait_bounded(&full[s], (j / kStages) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after();
+          const uint32_t a_addr = smem_u32(ring + s * Cfg::kStage);
+          const uint64_t adesc = tc::sw128_desc(a_addr);
+          const uint64_t bdesc = tc::sw128_desc(a_addr + Cfg::kStageA);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc::mma<kInt8>(d, adesc + 2 * k, bdesc + 2 * k, kIdesc,
+                           kBlock ? (k != 0) : (!first_of_seg || k != 0));
+          tc::commit(&empty[s]);
+          if (kBlock) {
+            tc::commit(&tfull[jt % kSmallBufs]);
+            ++jt;
+          }
+        }
+        if (!ok) break;
+        if (!kBlock) {
+          tc::commit(&tfull[jt % kSmallBufs]);
+          ++jt;
+        }
+        u = seg_end;
+      }
+      if (!ok) {
+        if (!*abort_flag) record_timeout(p.status, KID_GEMM_SMALL, 2);
+        *abort_flag = 1;
+      }
+      tc::commit(mma_done);
+      mbar_wait_bounded(mma_done, 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int et = threadIdx.x - 64;  // 0..127 = TMEM lane = weight row in the tile
+    const int q = warp & 3;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    const int KB = p.K / 128;
+    tc::grid_dependency_wait();  // s_x comes from the quantization kernel
+    uint32_t jt = 0;
+    bool ok = true;
+    for (int u = u0; u < u1 && ok;) {
+      const int t = u / nkb;
+      const int seg_end = min(u1, (t + 1) * nkb);
+      const bool whole = (u == t * nkb) && (seg_end == (t + 1) * nkb);
+      const int n = t * 128 + q * 32 + lane;
+      Acc acc[NTOK];
+#pragma unroll
+      for (int m = 0; m < NTOK; ++m) acc[m] = 0;
+      if constexpr (!kBlock) {
+        const uint32_t buf = jt % kSmallBufs;
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kSmallBufs) & 1, abort_flag));
+      }
+      if (!kBlock && ok) {
+        const uint32_t buf = jt % kSmallBufs;
+        tc::fence_after();
+        uint32_t r[32];
+        tc::ld32(tmem + lane_addr + buf * kSmallBufCols, r);
+        tc::ld_wait();
+#pragma unroll
+        for (int m = 0; m < NTOK; ++m) acc[m] = kInt8 ? (Acc)(int)r[m] : (Acc)__uint_as_float(r[m]);
+        tc::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+        ++jt;
+      } else if (kBlock) {
+        const float* swt = p.sw + (int64_t)t * KB;
+        for (int v = u; v < seg_end; ++v) {
+          const int kb = v - t * nkb;
+          const uint32_t buf = jt % kSmallBufs;
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kSmallBufs) & 1, abort_flag));
+          if (!ok) break;
+          tc::fence_after();
+          uint32_t r[32];
+          tc::ld32(tmem + lane_addr + buf * kSmallBufCols, r);
+          tc::ld_wait();
+          tc::fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+          ++jt;
+          const float swv = __ldg(swt + kb);
+#pragma unroll
+          for (int m = 0; m < NTOK; ++m) {
+            const float sxm = m < p.M ? __ldg(p.sx + (int64_t)m * KB + kb) : 0.0f;
+            acc[m] = fmaf(__uint_as_float(r[m]), sxm * swv, acc[m]);
+          }
+        }
+      }
+      // every epilogue warp leaves together if any of them gave up a wait
+      if (epi_any(!ok)) {
+        ok = false;
+        break;
+      }
+
+      bool do_epilogue = whole;
+      if (!whole) {
+        // park this segment's partial, then let the last contributor finish the tile
+        const int c_first = unit_owner(t * nkb, p.units, G);
+        const int c_last = unit_owner((t + 1) * nkb - 1, p.units, G);
+        const int my_slot = 2 * c + ((unit_begin(c, p.units, G) / nkb) == t ? 0 : 1);
+        float* slot = p.partials + (int64_t)my_slot * NTOK * 128;
+#pragma unroll
+        for (int m = 0; m < NTOK; ++m) {
+          if constexpr (kInt8)
+            reinterpret_cast<int*>(slot)[m * 128 + et] = acc[m];
+          else
+            slot[m * 128 + et] = acc[m];
+        }
+        __threadfence();
+        named_bar_sync(kSmallEpiBar, kSmallEpiWarps * 32);
+        if (et == 0) {
+          const unsigned old = atomicAdd(p.counters + t, 1u);
+          *last_flag = (old == (unsigned)(c_last - c_first));
+        }
+        named_bar_sync(kSmallEpiBar, kSmallEpiWarps * 32);
+        do_epilogue = *last_flag != 0;
+        if (do_epilogue) {
+          __threadfence();
+#pragma unroll
+          for (int m = 0; m < NTOK; ++m) acc[m] = 0;
+          for (int cc = c_first; cc <= c_last; ++cc) {
+            const int sl = 2 * cc + ((unit_begin(cc, p.units, G) / nkb) == t ? 0 : 1);
+            const float* src = p.partials + (int64_t)sl * NTOK * 128;
+#pragma unroll
+            for (int m = 0; m < NTOK; ++m) {
+              if constexpr (kInt8)
+                acc[m] += __ldcg(reinterpret_cast<const int*>(src) + m * 128 + et);
+              else
+                acc[m] += __ldcg(src + m * 128 + et);
+            }
+          }
+          if (et == 0) p.counters[t] = 0u;  // every contributor has arrived: reset for the next call
+        }
+      }
+      if (do_epilogue && n < p.N) {
+        const float swn = kBlock ? 1.0f : __ldg(p.sw + n);
+#pragma unroll
+        for (int m = 0; m < NTOK; ++m) {
+          if (m < p.M) {
+            float yv;
+            if constexpr (kInt8) {
+              if (p.acc_i32) p.acc_i32[(int64_t)m * p.N + n] = acc[m];
+              yv = __fmul_rn(__fmul_rn(__int2float_rn(acc[m]), __ldg(p.sx + m)), swn);
+            } else if constexpr (kBlock) {
+              yv = acc[m];
+            } else {
+              if (p.acc_f32) p.acc_f32[(int64_t)m * p.N + n] = acc[m];
+              yv = __fmul_rn(__fmul_rn(acc[m], __ldg(p.sx + m)), swn);
+            }
+            p.y[(int64_t)m * p.N + n] = f32_to_bf16_rn(yv);
+          }
+        }
+      }
+      u = seg_end;
+    }
+    if (!ok) {
+      if (lane == 0 && !*abort_flag) record_timeout(p.status, KID_GEMM_SMALL, 3);
+      *abort_flag = 1;
+    }
+  }
+
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after();
+    tc::tmem_dealloc(tmem, kSmallTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+namespace {
+struct SmallLayout {
+  size_t qx, sx, partials, counters, total;
+};
+
+SmallLayout small_layout(ql_scheme s, int64_t M, int64_t N, int64_t K, int sms) {
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  const int ntok = M <= 16 ? 16 : 32;
+  const int64_t units = ((N + 127) / 128) * ((K + 127) / 128);
+  const int64_t G = std::min<int64_t>(units, sms);
+  SmallLayout L;
+  L.qx = 0;
+  L.sx = up((size_t)(M * K));
+  L.partials = L.sx + up((size_t)M * (s == QL_FP8_E4M3_BLOCK128 ? K / 128 : 1) * 4);
+  L.counters = L.partials + up((size_t)G * 2 * ntok * 128 * 4);
+  L.total = L.counters + up((size_t)((N + 127) / 128) * 4);
+  return L;
+}
+}  // namespace
+
+size_t gemm_small_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms) {
+  return small_layout(scheme, M, N, K, num_sms).total;
+}
+
+template <ql_scheme S, int NTOK>
+static cudaError_t launch_small_t(const SmallParams& p, const CUtensorMap& tw, const CUtensorMap& tx,
+                                  int grid, cudaStream_t st) {
+  using Cfg = SmallCfg<NTOK>;
+  cudaError_t e = ensure_smem<gemm_small_kernel<S, NTOK>>(Cfg::kSmem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kSmallThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_small_kernel<S, NTOK>, tw, tx, p);
+}
+
+cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq,
+                              const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                              void* workspace, size_t ws_bytes, const ql_debug* dbg, int num_sms,
+                              DevStatus* status, cudaStream_t st) {
+  const SmallLayout L = small_layout(scheme, M, N, K, num_sms);
+  if (ws_bytes < L.total) return cudaErrorInvalidValue;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* qx = ws + L.qx;
+  float* sx = reinterpret_cast<float*>(ws + L.sx);
+  cudaError_t e = launch_quantize_act(scheme, x, M, K, qx, sx, st);
+  if (e != cudaSuccess) return e;
+
+  SmallParams p;
+  p.sx = sx;
+  p.sw = sw;
+  p.y = y;
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.ntn = (int)((N + 127) / 128);
+  p.nkb = (int)((K + 127) / 128);
+  p.units = p.ntn * p.nkb;
+  p.partials = reinterpret_cast<float*>(ws + L.partials);
+  p.counters = reinterpret_cast<unsigned*>(ws + L.counters);
+  p.acc_i32 = dbg ? dbg->acc_i32 : nullptr;
+  p.acc_f32 = dbg ? dbg->acc_f32 : nullptr;
+  p.status = status;
+  const int ntok = M <= 16 ? 16 : 32;
+  CUtensorMap tw, tx;
+  if ((e = make_tmap_u8_sw128(&tw, wq, (uint64_t)K, (uint64_t)N, (uint64_t)K, 128, 128)) != cudaSuccess)
+    return e;
+  if ((e = make_tmap_u8_sw128(&tx, qx, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)ntok)) !=
+      cudaSuccess)
+    return e;
+  const int grid = (int)std::min<int64_t>(p.units, num_sms);
+  switch (scheme) {
+    case QL_W8A8_INT8_ROW:
+      e = ntok == 16 ? launch_small_t<QL_W8A8_INT8_ROW, 16>(p, tw, tx, grid, st)
+                     : launch_small_t<QL_W8A8_INT8_ROW, 32>(p, tw, tx, grid, st);
+      break;
+    case QL_FP8_E4M3_ROW:
+      e = ntok == 16 ? launch_small_t<QL_FP8_E4M3_ROW, 16>(p, tw, tx, grid, st)
+                     : launch_small_t<QL_FP8_E4M3_ROW, 32>(p, tw, tx, grid, st);
+      break;
+    default:
+      e = ntok == 16 ? launch_small_t<QL_FP8_E4M3_BLOCK128, 16>(p, tw, tx, grid, st)
+                     : launch_small_t<QL_FP8_E4M3_BLOCK128, 32>(p, tw, tx, grid, st);
+  }
+  if (e != cudaSuccess) return e;
+  if (dbg && (dbg->qx || dbg->sx)) {
+    // debug capture of the quantized tokens (stream-ordered device copies)
+    if (dbg->qx && (e = cudaMemcpyAsync(dbg->qx, qx, (size_t)(M * K), cudaMemcpyDeviceToDevice, st)) != cudaSuccess)
+      return e;
+    const size_t sx_bytes = (size_t)M * (scheme == QL_FP8_E4M3_BLOCK128 ? K / 128 : 1) * 4;
+    if (dbg->sx && (e = cudaMemcpyAsync(dbg->sx, sx, sx_bytes, cudaMemcpyDeviceToDevice, st)) != cudaSuccess)
+      return e;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace ql

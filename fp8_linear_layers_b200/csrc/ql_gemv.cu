@@ -8,28 +8,38 @@
 // Design (B200, one persistent CTA per SM):
 //  * CTA b owns the contiguous output rows [b N / G, (b+1) N / G).  Those rows
 //    are one contiguous byte range of W_q, which a producer warp streams into
-//    a 4-stage shared-memory ring with bulk copies (the TMA engine), each stage
-//    holding whole rows (<= 32 KB), completion tracked by mbarriers.
-//  * 16 consumer warps first quantize x (fused per-token or per-128-group
-//    absmax, IEEE-divided scale, rounded codes) into shared memory and pull
-//    their fixed slice of the codes into registers, while the first stages
-//    are already in flight.
+//    a shared-memory ring (as many stages as fit, each holding whole rows)
+//    with bulk copies on the TMA engine, completion tracked by mbarriers.
+//  * The kernel is launched with programmatic dependent launch: it lets the
+//    next kernel on the stream start as soon as SMs free up, and streams its
+//    own weights before the previous kernel has finished; x (which a previous
+//    kernel may produce) is read, and y written, only after the grid
+//    dependency wait.  Weights must therefore not be written by work still in
+//    flight on the stream.
+//  * 16 consumer warps quantize x (fused per-token or per-128-group absmax,
+//    IEEE-divided scale, rounded codes) into shared memory and keep their
+//    fixed slice of the codes in registers.
 //  * Each consumer thread owns fixed 16-byte k-chunks of a row group; per
 //    chunk it runs 4 dp4a (int8, exact int32) or unpacks 16 E4M3 weights to
-//    f32 and does 16 FMAs (E4M3 x E4M3 products are exact in f32).  Partial
-//    sums are reduced with warp shuffles and one shared-memory step; the scale
-//    epilogue writes bf16.
-//  * Every wait is bounded; a consumer-wide vote makes all consumer threads
-//    leave together if any of them gave up, so no thread is left at a barrier.
+//    f32 and does 16 FMAs (E4M3 x E4M3 products are exact in f32).
+//  * No CTA-wide barrier per stage: each warp reduces its partial sums with
+//    shuffles into a per-stage slot and counts itself in; the last warp to
+//    finish a stage adds the slots in a fixed order, writes y and releases the
+//    ring stage.  Warps drift freely between stages.
+//  * Every wait is bounded; a warp that gives up raises a CTA abort flag that
+//    every other wait checks, so all roles leave without further barriers.
 #include "ql_common.cuh"
 #include "ql_internal.h"
+#include "ql_tc.cuh"
 
 namespace ql {
 
 constexpr int kGemvConsumers = 512;  // 16 warps
+constexpr int kGemvWarps = kGemvConsumers / 32;
 constexpr int kGemvThreads = kGemvConsumers + 32;
-constexpr int kGemvStages = 4;
-constexpr int kGemvStageBytes = 32768;
+constexpr int kGemvMaxStages = 8;
+constexpr int kGemvStageTarget = 32768;
+constexpr int kGemvSmemBudget = 200 * 1024;
 constexpr int kGemvMaxK = 32768;
 constexpr int kGemvMaxAcc = 4;
 constexpr uint32_t kBarConsumers = 1;  // named barrier id used by the consumer warps
@@ -43,30 +53,31 @@ struct GemvParams {
   int rows_per_stage;  // R_s: whole rows per ring stage
   int tg;              // threads per row group (power of two, 32..512)
   int stage_bytes;     // R_s * K rounded up to 128
+  int stages;          // ring depth
   ql_debug dbg;
   DevStatus* status;
 };
 
 struct GemvSmemLayout {
-  int ring, qx, sx, red, bars, flags, total;
+  int ring, qx, sx, part, bars, flags, total;
 };
 
-__host__ __device__ inline GemvSmemLayout gemv_layout(int64_t K, int stage_bytes) {
+__host__ __device__ inline GemvSmemLayout gemv_layout(int64_t K, int stage_bytes, int stages) {
   GemvSmemLayout L;
   int off = 0;
   L.ring = off;
-  off += kGemvStages * stage_bytes;
+  off += stages * stage_bytes;
   L.qx = off;
   off += (int)((K + 127) / 128) * 128;
   L.sx = off;
   off += (int)((K / 128 + 1 + 31) / 32) * 128;
-  L.red = off;
-  off += 2 * 16 * kGemvMaxAcc * 4;
-  L.bars = off;
-  off += 2 * kGemvStages * 8;
-  L.flags = off;
-  off += 16 * 4 + 16;
-  L.total = off;
+  L.part = off;  // [stages][16 warps][kGemvMaxAcc] partial sums
+  off += kGemvMaxStages * kGemvWarps * kGemvMaxAcc * 4;
+  L.bars = off;  // full[stages], empty[stages]
+  off += 2 * kGemvMaxStages * 8;
+  L.flags = off;  // abort flag, per-stage arrival counters, block reduction scratch
+  off += 16 + kGemvMaxStages * 4 + kGemvWarps * 4;
+  L.total = (off + 127) / 128 * 128;
   return L;
 }
 
@@ -76,20 +87,6 @@ QL_DEVINL uint4 lds128(uint32_t addr) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(addr));
   return v;
-}
-
-// Consumer-wide OR vote that doubles as the consumers' barrier.
-QL_DEVINL bool consumers_any(bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(kBarConsumers), "r"(kGemvConsumers)
-      : "memory");
-  return r != 0;
 }
 
 // 16 E4M3 codes (one 16-byte chunk) -> 16 f32 values.
@@ -122,6 +119,15 @@ QL_DEVINL float e4m3_chunk_dot(const uint4& wv, const float* xf) {
   return p0 + p1;
 }
 
+template <bool kInt8>
+QL_DEVINL uint32_t quant4(float f0, float f1, float f2, float f3, float s) {
+  if (kInt8)
+    return (uint32_t)(int8_code(f0, s) & 0xFF) | ((uint32_t)(int8_code(f1, s) & 0xFF) << 8) |
+           ((uint32_t)(int8_code(f2, s) & 0xFF) << 16) | ((uint32_t)(int8_code(f3, s) & 0xFF) << 24);
+  return f32x2_to_e4m3x2(e4m3_quotient(f0, s), e4m3_quotient(f1, s)) |
+         (f32x2_to_e4m3x2(e4m3_quotient(f2, s), e4m3_quotient(f3, s)) << 16);
+}
+
 template <ql_scheme kScheme, int kXC>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams p) {
   constexpr bool kInt8 = kScheme == QL_W8A8_INT8_ROW;
@@ -129,15 +135,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   using Acc = typename std::conditional<kInt8, int, float>::type;
 
   extern __shared__ __align__(1024) uint8_t smem[];
-  const GemvSmemLayout L = gemv_layout(p.K, p.stage_bytes);
+  const int nst = p.stages;
+  const GemvSmemLayout L = gemv_layout(p.K, p.stage_bytes, nst);
   uint8_t* ring = smem + L.ring;
   uint8_t* qx_s = smem + L.qx;
   float* sx_s = reinterpret_cast<float*>(smem + L.sx);
-  Acc* red = reinterpret_cast<Acc*>(smem + L.red);  // [2][16 warps][kGemvMaxAcc]
+  Acc* part = reinterpret_cast<Acc*>(smem + L.part);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* empty = full + kGemvStages;
+  uint64_t* empty = full + kGemvMaxStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.flags);
-  float* blockred = reinterpret_cast<float*>(smem + L.flags + 16);
+  int* arrivals = reinterpret_cast<int*>(smem + L.flags + 16);
+  float* blockred = reinterpret_cast<float*>(smem + L.flags + 16 + kGemvMaxStages * 4);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -149,24 +157,25 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   const int nstages = (int)((row_end - row_begin + Rs - 1) / Rs);
 
   if (tid == 0) {
-    for (int s = 0; s < kGemvStages; ++s) {
+    tc::launch_dependents();  // the next kernel may start as SMs free up
+    for (int s = 0; s < nst; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kGemvConsumers / 32);
+      mbar_init(&empty[s], 1);  // released by the warp that finishes the stage last
+      arrivals[s] = 0;
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
 
-  if (warp == kGemvConsumers / 32) {
+  if (warp == kGemvWarps) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t policy = l2_policy_evict_first();
       int issued = 0;
       for (int i = 0; i < nstages; ++i) {
-        const int slot = i % kGemvStages;
-        if (i >= kGemvStages &&
-            !mbar_wait_bounded(&empty[slot], ((i / kGemvStages) - 1) & 1, abort_flag)) {
+        const int slot = i % nst;
+        if (i >= nst && !mbar_wait_bounded(&empty[slot], ((i / nst) - 1) & 1, abort_flag)) {
           if (!*abort_flag) record_timeout(p.status, KID_GEMV, 1);
           *abort_flag = 1;
           break;
@@ -181,13 +190,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       // Drain: no copy may still be writing this CTA's shared memory when it
       // exits.  Only this thread arms the full barriers, so after its last
       // arm the parity test below cannot alias a later phase.
-      for (int i = max(0, issued - kGemvStages); i < issued; ++i)
-        mbar_wait_bounded(&full[i % kGemvStages], (i / kGemvStages) & 1, nullptr);
+      for (int i = max(0, issued - nst); i < issued; ++i)
+        mbar_wait_bounded(&full[i % nst], (i / nst) & 1, nullptr);
     }
     return;
   }
 
   // -------------------------------------------------------------- consumers
+  tc::grid_dependency_wait();  // x may be produced by the previous kernel
   // 1. Fused activation quantization of x [1, K] into shared memory.
   {
     const int64_t nchunk8 = K / 8;  // 16-byte chunks of 8 bf16
@@ -210,15 +220,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         const float s = a / 448.0f;
         if (c < nchunk8) {
           if ((lane & 15) == 0) sx_s[c >> 4] = s;
-          uint32_t o2[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            o2[h] = f32x2_to_e4m3x2(e4m3_quotient(bf16_lo(w[2 * h]), s),
-                                    e4m3_quotient(bf16_hi(w[2 * h]), s)) |
-                    (f32x2_to_e4m3x2(e4m3_quotient(bf16_lo(w[2 * h + 1]), s),
-                                     e4m3_quotient(bf16_hi(w[2 * h + 1]), s))
-                     << 16);
-          reinterpret_cast<uint2*>(qx_s)[c] = make_uint2(o2[0], o2[1]);
+          reinterpret_cast<uint2*>(qx_s)[c] =
+              make_uint2(quant4<false>(bf16_lo(w[0]), bf16_hi(w[0]), bf16_lo(w[1]), bf16_hi(w[1]), s),
+                         quant4<false>(bf16_lo(w[2]), bf16_hi(w[2]), bf16_lo(w[3]), bf16_hi(w[3]), s));
         }
       } else {
         a_tok = fmaxf(a_tok, a);
@@ -230,7 +234,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       named_bar_sync(kBarConsumers, kGemvConsumers);
       float a = blockred[0];
 #pragma unroll
-      for (int w = 1; w < 16; ++w) a = fmaxf(a, blockred[w]);
+      for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, blockred[w]);
       const float s = a / (kInt8 ? 127.0f : 448.0f);
       if (tid == 0) sx_s[0] = s;
 #pragma unroll
@@ -238,20 +242,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         const int64_t c = tid + (int64_t)i * kGemvConsumers;
         if (c < nchunk8) {
           const uint32_t w[4] = {xc[i].x, xc[i].y, xc[i].z, xc[i].w};
-          uint32_t o2[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const float f0 = bf16_lo(w[2 * h]), f1 = bf16_hi(w[2 * h]);
-            const float f2 = bf16_lo(w[2 * h + 1]), f3 = bf16_hi(w[2 * h + 1]);
-            if (kInt8)
-              o2[h] = (uint32_t)(int8_code(f0, s) & 0xFF) | ((uint32_t)(int8_code(f1, s) & 0xFF) << 8) |
-                      ((uint32_t)(int8_code(f2, s) & 0xFF) << 16) |
-                      ((uint32_t)(int8_code(f3, s) & 0xFF) << 24);
-            else
-              o2[h] = f32x2_to_e4m3x2(e4m3_quotient(f0, s), e4m3_quotient(f1, s)) |
-                      (f32x2_to_e4m3x2(e4m3_quotient(f2, s), e4m3_quotient(f3, s)) << 16);
-          }
-          reinterpret_cast<uint2*>(qx_s)[c] = make_uint2(o2[0], o2[1]);
+          reinterpret_cast<uint2*>(qx_s)[c] =
+              make_uint2(quant4<kInt8>(bf16_lo(w[0]), bf16_hi(w[0]), bf16_lo(w[1]), bf16_hi(w[1]), s),
+                         quant4<kInt8>(bf16_lo(w[2]), bf16_hi(w[2]), bf16_lo(w[3]), bf16_hi(w[3]), s));
         }
       }
     }
@@ -268,6 +261,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   // 2. This thread's fixed k-chunks of a row: kk = u + j * TG (16 bytes each).
   const int TG = p.tg;
   const int RP = kGemvConsumers / TG;  // row groups working side by side
+  const int wpg = TG / 32;             // warps per row group
   const int grp = tid / TG, u = tid % TG;
   const int64_t CR = K / 16;
   uint4 xq[kXC];
@@ -288,81 +282,90 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   // 3. Stream the ring.
   const uint32_t ring_a = smem_u32(ring);
   for (int i = 0; i < nstages; ++i) {
-    const int slot = i % kGemvStages;
+    const int slot = i % nst;
     const int64_t r0 = row_begin + (int64_t)i * Rs;
     const int nr = (int)min((int64_t)Rs, row_end - r0);
-    const bool ok = mbar_wait_bounded(&full[slot], (i / kGemvStages) & 1, abort_flag);
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], (i / nst) & 1, abort_flag))) {
+      if (lane == 0 && !*abort_flag) record_timeout(p.status, KID_GEMV, 2);
+      *abort_flag = 1;
+      break;
+    }
     Acc acc[kGemvMaxAcc];
 #pragma unroll
     for (int a = 0; a < kGemvMaxAcc; ++a) acc[a] = 0;
-    if (ok) {
-      const uint32_t stage_a = ring_a + slot * p.stage_bytes;
+    const uint32_t stage_a = ring_a + slot * p.stage_bytes;
 #pragma unroll
-      for (int a = 0; a < kGemvMaxAcc; ++a) {
-        const int r = grp + a * RP;
-        if (r < nr) {
-          const uint32_t row_a = stage_a + (uint32_t)(r * K);
-          float sw_blk[kBlock ? kXC : 1];
-          if (kBlock) {
-            const float* swr = p.sw + ((r0 + r) >> 7) * KB;
+    for (int a = 0; a < kGemvMaxAcc; ++a) {
+      const int r = grp + a * RP;
+      if (r < nr) {
+        const uint32_t row_a = stage_a + (uint32_t)(r * K);
+        float sw_blk[kBlock ? kXC : 1];
+        if (kBlock) {
+          const float* swr = p.sw + ((r0 + r) >> 7) * KB;
 #pragma unroll
-            for (int j = 0; j < kXC; ++j) sw_blk[j] = have[j] ? __ldg(swr + ((u + j * TG) >> 3)) : 0.0f;
-          }
+          for (int j = 0; j < kXC; ++j) sw_blk[j] = have[j] ? __ldg(swr + ((u + j * TG) >> 3)) : 0.0f;
+        }
 #pragma unroll
-          for (int j = 0; j < kXC; ++j) {
-            if (have[j]) {
-              const uint4 wv = lds128(row_a + (uint32_t)((u + j * TG) * 16));
-              if constexpr (kInt8) {
-                int s = acc[a];
-                s = __dp4a((int)wv.x, (int)xq[j].x, s);
-                s = __dp4a((int)wv.y, (int)xq[j].y, s);
-                s = __dp4a((int)wv.z, (int)xq[j].z, s);
-                s = __dp4a((int)wv.w, (int)xq[j].w, s);
-                acc[a] = s;
-              } else if constexpr (kBlock) {
-                acc[a] = fmaf(e4m3_chunk_dot(wv, &xf[16 * j]), xs[j] * sw_blk[j], acc[a]);
-              } else {
-                acc[a] += e4m3_chunk_dot(wv, &xf[16 * j]);
-              }
+        for (int j = 0; j < kXC; ++j) {
+          if (have[j]) {
+            const uint4 wv = lds128(row_a + (uint32_t)((u + j * TG) * 16));
+            if constexpr (kInt8) {
+              int s = acc[a];
+              s = __dp4a((int)wv.x, (int)xq[j].x, s);
+              s = __dp4a((int)wv.y, (int)xq[j].y, s);
+              s = __dp4a((int)wv.z, (int)xq[j].z, s);
+              s = __dp4a((int)wv.w, (int)xq[j].w, s);
+              acc[a] = s;
+            } else if constexpr (kBlock) {
+              acc[a] = fmaf(e4m3_chunk_dot(wv, &xf[16 * j]), xs[j] * sw_blk[j], acc[a]);
+            } else {
+              acc[a] += e4m3_chunk_dot(wv, &xf[16 * j]);
             }
           }
         }
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
-
-    // Reduce over the warp, then over the row group's warps.
-    Acc* rb = red + (i & 1) * 16 * kGemvMaxAcc;
+    // Reduce over the warp into this stage's partial slot, then count in.
+    Acc* ps = part + slot * kGemvWarps * kGemvMaxAcc;
 #pragma unroll
     for (int a = 0; a < kGemvMaxAcc; ++a) {
       Acc v = acc[a];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) rb[warp * kGemvMaxAcc + a] = v;
+      if (lane == 0) ps[warp * kGemvMaxAcc + a] = v;
     }
-    if (consumers_any(!ok)) {
-      if (tid == 0 && !*abort_flag) record_timeout(p.status, KID_GEMV, 2);
-      *abort_flag = 1;
-      break;
+    __syncwarp();
+    int before = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      before = atomicAdd(&arrivals[slot], 1);
     }
-    if (tid < nr) {
-      const int r = tid, g = r % RP, a = r / RP;
-      const int wpg = TG / 32;  // warps per row group
-      Acc v = rb[(g * wpg) * kGemvMaxAcc + a];
-      for (int w = 1; w < wpg; ++w) v += rb[(g * wpg + w) * kGemvMaxAcc + a];
-      const int64_t n = r0 + r;
-      float yv;
-      if constexpr (kInt8) {
-        if (p.dbg.acc_i32) p.dbg.acc_i32[n] = v;
-        yv = __fmul_rn(__fmul_rn(__int2float_rn(v), sx_tok), __ldg(p.sw + n));
-      } else if constexpr (kBlock) {
-        yv = v;
-      } else {
-        if (p.dbg.acc_f32) p.dbg.acc_f32[n] = v;
-        yv = __fmul_rn(__fmul_rn(v, sx_tok), __ldg(p.sw + n));
+    before = __shfl_sync(0xffffffffu, before, 0);
+    if (before == kGemvWarps - 1) {
+      // last warp of this stage: every warp has read the stage and written its slot
+      __threadfence_block();
+      if (lane < nr) {
+        const int r = lane, g = r % RP, a = r / RP;
+        Acc v = ps[(g * wpg) * kGemvMaxAcc + a];
+        for (int w = 1; w < wpg; ++w) v += ps[(g * wpg + w) * kGemvMaxAcc + a];
+        const int64_t n = r0 + r;
+        float yv;
+        if constexpr (kInt8) {
+          if (p.dbg.acc_i32) p.dbg.acc_i32[n] = v;
+          yv = __fmul_rn(__fmul_rn(__int2float_rn(v), sx_tok), __ldg(p.sw + n));
+        } else if constexpr (kBlock) {
+          yv = v;
+        } else {
+          if (p.dbg.acc_f32) p.dbg.acc_f32[n] = v;
+          yv = __fmul_rn(__fmul_rn(v, sx_tok), __ldg(p.sw + n));
+        }
+        p.y[n] = f32_to_bf16_rn(yv);
       }
-      p.y[n] = f32_to_bf16_rn(yv);
+      __syncwarp();
+      if (lane == 0) {
+        arrivals[slot] = 0;
+        mbar_arrive(&empty[slot]);
+      }
     }
   }
 }
@@ -375,26 +378,31 @@ static int pow2_floor(int64_t v) {
 
 int gemv_max_k() { return kGemvMaxK; }
 
+template <ql_scheme S, int XC>
+static cudaError_t launch_gemv_x(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
+  cudaError_t e = ensure_smem<gemv_kernel<S, XC>>((int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<S, XC>, p);
+}
+
 template <ql_scheme S>
-static cudaError_t launch_gemv_t(const GemvParams& p, int xc, int grid, size_t smem,
-                                 cudaStream_t st) {
-  cudaError_t e = cudaSuccess;
-#define QL_GEMV_CASE(XC)                                                                       \
-  case XC: {                                                                                   \
-    auto kern = gemv_kernel<S, XC>;                                                            \
-    e = ensure_smem(kern, (int)smem);                                                          \
-    if (e != cudaSuccess) return e;                                                            \
-    kern<<<grid, kGemvThreads, smem, st>>>(p);                                                 \
-    return cudaGetLastError();                                                                 \
-  }
+static cudaError_t launch_gemv_t(const GemvParams& p, int xc, int grid, size_t smem, cudaStream_t st) {
   switch (xc) {
-    QL_GEMV_CASE(1)
-    QL_GEMV_CASE(2)
-    QL_GEMV_CASE(4)
+    case 1: return launch_gemv_x<S, 1>(p, grid, smem, st);
+    case 2: return launch_gemv_x<S, 2>(p, grid, smem, st);
+    case 4: return launch_gemv_x<S, 4>(p, grid, smem, st);
     default: return cudaErrorInvalidValue;
   }
-#undef QL_GEMV_CASE
-  return e;
 }
 
 cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
@@ -407,21 +415,22 @@ cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, con
   p.y = y;
   p.N = N;
   p.K = K;
-  p.rows_per_stage = (int)std::max<int64_t>(1, std::min<int64_t>(32, kGemvStageBytes / K));
+  p.rows_per_stage = (int)std::max<int64_t>(1, std::min<int64_t>(32, kGemvStageTarget / K));
   const int64_t CR = K / 16;
   p.tg = (int)std::max<int64_t>(32, std::min<int64_t>(kGemvConsumers, pow2_floor(CR)));
   p.stage_bytes = (int)(((int64_t)p.rows_per_stage * K + 127) / 128 * 128);
+  const int fixed = gemv_layout(K, p.stage_bytes, 0).total;
+  p.stages = (int)std::min<int64_t>(kGemvMaxStages, (kGemvSmemBudget - fixed) / p.stage_bytes);
+  if (p.stages < 2) return cudaErrorInvalidConfiguration;
   p.dbg = dbg ? *dbg : ql_debug{nullptr, nullptr, nullptr, nullptr};
   p.status = status;
   const int64_t xc_needed = (CR + p.tg - 1) / p.tg;
   const int xc = xc_needed <= 1 ? 1 : (xc_needed <= 2 ? 2 : 4);
-  // rows in the ring at once are at most R_s per stage; each thread carries
-  // ceil(R_s / RP) accumulators
   const int RP = kGemvConsumers / p.tg;
   if ((p.rows_per_stage + RP - 1) / RP > kGemvMaxAcc) return cudaErrorInvalidConfiguration;
   const int64_t stage_rows_total = (N + p.rows_per_stage - 1) / p.rows_per_stage;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms, stage_rows_total));
-  const size_t smem = gemv_layout(K, p.stage_bytes).total;
+  const size_t smem = gemv_layout(K, p.stage_bytes, p.stages).total;
   switch (scheme) {
     case QL_W8A8_INT8_ROW: return launch_gemv_t<QL_W8A8_INT8_ROW>(p, xc, grid, smem, st);
     case QL_FP8_E4M3_ROW: return launch_gemv_t<QL_FP8_E4M3_ROW>(p, xc, grid, smem, st);

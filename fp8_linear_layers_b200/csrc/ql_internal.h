@@ -1,6 +1,7 @@
 // ql_internal.h -- host-side launchers shared between the qlinear translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -13,16 +14,16 @@ namespace ql {
 
 struct DevStatus;
 
-// Raise a kernel's dynamic shared-memory limit once per device (and again only
-// if a larger size is asked for), so launches do not pay for the attribute call.
-template <typename Kernel>
-inline cudaError_t ensure_smem(Kernel kern, int bytes) {
-  static int done[64] = {0};
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device), and
+// again only if a larger size is asked for, so launches skip the attribute call.
+template <auto kKernel>
+inline cudaError_t ensure_smem(int bytes) {
+  static int done[64] = {0};  // one table per kernel instantiation
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < 64 && __atomic_load_n(&done[dev], __ATOMIC_ACQUIRE) >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = cudaFuncSetAttribute(kKernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess && dev >= 0 && dev < 64) {
     int cur = __atomic_load_n(&done[dev], __ATOMIC_ACQUIRE);
     while (cur < bytes && !__atomic_compare_exchange_n(&done[dev], &cur, bytes, false,
@@ -31,6 +32,10 @@ inline cudaError_t ensure_smem(Kernel kern, int bytes) {
   }
   return e;
 }
+
+// 2-D TMA map over a row-major byte matrix, 128-byte swizzle, zero fill.
+cudaError_t make_tmap_u8_sw128(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                               uint64_t stride, uint32_t box_inner, uint32_t box_rows);
 
 cudaError_t launch_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, int64_t K,
                                 uint8_t* qx, float* sx, cudaStream_t st);

@@ -11,6 +11,7 @@
 // for a whole row); the scale is one IEEE f32 division and each code one more.
 #include "ql_common.cuh"
 #include "ql_internal.h"
+#include "ql_tc.cuh"
 
 namespace ql {
 
@@ -19,10 +20,14 @@ namespace ql {
 //   kBf16Scale  the scale is rounded to bf16 before use (W8A8 weight scales)
 // Each thread keeps up to kCache 16-byte chunks of the row in registers so the
 // row is read from HBM once; longer rows re-read the remainder from L2.
-template <bool kInt8, bool kBf16Scale, int kThreads, int kCache>
+//   kTrigger    let a dependent kernel launched with programmatic dependent
+//               launch start early (activations only: the dependents stream
+//               their weights before waiting, so weight writers never trigger)
+template <bool kInt8, bool kBf16Scale, bool kTrigger, int kThreads, int kCache>
 __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __restrict__ x,
                                                               int64_t K, uint8_t* __restrict__ q,
                                                               float* __restrict__ s_out) {
+  if (kTrigger && threadIdx.x == 0) tc::launch_dependents();
   const int64_t row = blockIdx.x;
   const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
   const int64_t nchunk = K / 8;  // 8 bf16 per 16-byte chunk
@@ -95,6 +100,7 @@ __global__ void __launch_bounds__(256) quant_groups_kernel(const uint16_t* __res
                                                            int64_t ngroups,
                                                            uint8_t* __restrict__ q,
                                                            float* __restrict__ s_out) {
+  if (threadIdx.x == 0) tc::launch_dependents();  // activations: dependents may start early
   const int64_t g = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4);
   const int lane16 = threadIdx.x & 15;
   const bool live = g < ngroups;
@@ -164,22 +170,28 @@ __global__ void __launch_bounds__(256) quant_wblock_kernel(const uint16_t* __res
   }
 }
 
-template <bool kInt8, bool kBf16Scale>
+template <bool kInt8, bool kBf16Scale, bool kTrigger>
 static cudaError_t launch_rows(const uint16_t* x, int64_t rows, int64_t K, uint8_t* q, float* s,
                                cudaStream_t st) {
   if (K <= 8 * 8 * 256)
-    quant_rows_kernel<kInt8, kBf16Scale, 256, 8><<<(unsigned)rows, 256, 0, st>>>(x, K, q, s);
+    quant_rows_kernel<kInt8, kBf16Scale, kTrigger, 256, 8><<<(unsigned)rows, 256, 0, st>>>(x, K, q, s);
   else
-    quant_rows_kernel<kInt8, kBf16Scale, 512, 8><<<(unsigned)rows, 512, 0, st>>>(x, K, q, s);
+    quant_rows_kernel<kInt8, kBf16Scale, kTrigger, 512, 8><<<(unsigned)rows, 512, 0, st>>>(x, K, q, s);
   return cudaGetLastError();
 }
+
+// An empty kernel launched normally after the weight quantizer: a following
+// kernel launched with programmatic dependent launch may start as soon as
+// this one exits, and this one starts only once the weights are complete and
+// visible, so weights are never streamed before they are written.
+__global__ void stream_order_kernel() {}
 
 cudaError_t launch_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, int64_t K,
                                 uint8_t* qx, float* sx, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   switch (scheme) {
-    case QL_W8A8_INT8_ROW: return launch_rows<true, false>(x, M, K, qx, sx, st);
-    case QL_FP8_E4M3_ROW: return launch_rows<false, false>(x, M, K, qx, sx, st);
+    case QL_W8A8_INT8_ROW: return launch_rows<true, false, true>(x, M, K, qx, sx, st);
+    case QL_FP8_E4M3_ROW: return launch_rows<false, false, true>(x, M, K, qx, sx, st);
     default: {
       const int64_t ngroups = M * (K / 128);
       quant_groups_kernel<<<(unsigned)((ngroups + 15) / 16), 256, 0, st>>>(x, ngroups, qx, sx);
@@ -190,13 +202,17 @@ cudaError_t launch_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, 
 
 cudaError_t launch_quantize_weight(ql_scheme scheme, const uint16_t* w, int64_t N, int64_t K,
                                    uint8_t* wq, float* sw, cudaStream_t st) {
+  cudaError_t e;
   switch (scheme) {
-    case QL_W8A8_INT8_ROW: return launch_rows<true, true>(w, N, K, wq, sw, st);
-    case QL_FP8_E4M3_ROW: return launch_rows<false, false>(w, N, K, wq, sw, st);
+    case QL_W8A8_INT8_ROW: e = launch_rows<true, true, false>(w, N, K, wq, sw, st); break;
+    case QL_FP8_E4M3_ROW: e = launch_rows<false, false, false>(w, N, K, wq, sw, st); break;
     default:
       quant_wblock_kernel<<<(unsigned)((N / 128) * (K / 128)), 256, 0, st>>>(w, K, wq, sw);
-      return cudaGetLastError();
+      e = cudaGetLastError();
   }
+  if (e != cudaSuccess) return e;
+  stream_order_kernel<<<1, 32, 0, st>>>();
+  return cudaGetLastError();
 }
 
 }  // namespace ql

@@ -1,0 +1,118 @@
+// ql_tc.cuh -- tcgen05 (5th-generation tensor core) and TMA tensor-copy helpers.
+//
+// Inline PTX for sm_100a: TMEM allocation, MMA issue (kind::i8 for int8 x int8
+// -> s32, kind::f8f6f4 for E4M3 x E4M3 -> f32), commit to mbarriers, TMEM
+// loads, and 2-D tiled TMA loads.  Operands are K-major tiles in shared
+// memory laid out with the 128-byte swizzle that TMA writes.  No multicast
+// form appears anywhere in this file.
+#pragma once
+
+#include <cuda.h>
+
+#include "ql_common.cuh"
+
+namespace ql {
+namespace tc {
+
+// ---- instruction descriptor (kind::i8 / kind::f8f6f4, dense, K-major A and B)
+//  bits [4,6)   D format: 1 = f32, 2 = s32
+//  bits [7,10)  A format: kind::i8 -> 1 = signed 8-bit; kind::f8f6f4 -> 0 = E4M3
+//  bits [10,13) B format: same encoding
+//  bit 15 / 16  A / B major: 0 = K-major
+//  bits [17,23) N >> 3
+//  bits [24,29) M >> 4
+__host__ __device__ constexpr uint32_t idesc(bool int8, int m, int n) {
+  return ((int8 ? 2u : 1u) << 4) | ((int8 ? 1u : 0u) << 7) | ((int8 ? 1u : 0u) << 10) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// ---- shared-memory matrix descriptor: K-major tile of 128-byte rows written
+// by TMA with the 128-byte swizzle; 8-row groups are 1024 bytes apart.
+//  bits [0,14)  start address >> 4
+//  bits [16,30) leading-dimension byte offset >> 4 (not used by this layout)
+//  bits [32,46) stride-dimension byte offset >> 4 (1024 B)
+//  bits [46,48) descriptor version (1 on sm_100)
+//  bits [61,64) layout: 2 = 128-byte swizzle
+QL_DEVINL uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// ---- TMEM
+QL_DEVINL void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+QL_DEVINL void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+QL_DEVINL void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+QL_DEVINL void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+QL_DEVINL void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Arrive on `bar` once every tcgen05 operation this thread issued so far has completed.
+QL_DEVINL void commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, one instruction covers K = 32 bytes.
+template <bool kInt8>
+QL_DEVINL void mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t id, uint32_t accumulate) {
+  if constexpr (kInt8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(id), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(id), "r"(accumulate)
+        : "memory");
+  }
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: lane i of the warp gets TMEM lane
+// (taddr.lane + i), columns [taddr.col, taddr.col + 32).
+QL_DEVINL void ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+QL_DEVINL void ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---- TMA tiled 2-D load (no multicast).  x is the innermost (byte) coordinate
+// and must be a multiple of 16; y is the row.
+QL_DEVINL void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y, uint64_t* bar,
+                           uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+QL_DEVINL void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// ---- programmatic dependent launch
+QL_DEVINL void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+QL_DEVINL void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+}  // namespace tc
+}  // namespace ql

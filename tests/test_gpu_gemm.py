@@ -1,0 +1,128 @@
+"""GPU parity: the large-M tcgen05 GEMM (pre-quantized activations) vs the oracle.
+
+Inputs are quantized by the oracle, so this file checks the product and the
+epilogue alone.  Small and ragged shapes (several tiles, partial M / N tiles,
+K not a multiple of the 128-byte stage) are compared output by output; the
+prefill configurations (M in {512, 1024} x gate/up, down, fused qkv, W8A8;
+Qwen3-8B FP8-block at M = 512) at full size on sampled outputs plus whole rows
+and columns.  int8: int32 accumulators and bf16 outputs bit-exact; E4M3:
+2^-7 |y| + 1e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fp8_linear_layers_b200 as ql
+import oracle
+from fp8_linear_layers_b200 import synthetic
+from tests._util import assert_y_close, bits, f32_dev, u8_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(scheme, M, N, K, seed=0, outliers=None):
+    if outliers is None:
+        outliers = synthetic.outlier_count(K) if scheme != ql.FP8_E4M3_BLOCK128 else 0
+    x = synthetic.make_x(M, K, seed=seed, tag="gemm-x", outliers=outliers)
+    w = synthetic.make_w(N, K, seed=seed, tag="gemm-w")
+    qx, sx = oracle.quantize_act(scheme, x)
+    wq, sw = oracle.quantize_weight(scheme, w)
+    return qx, sx, wq, sw
+
+
+def _gpu(scheme, qx, sx, wq, sw, want_acc=True):
+    M, K = qx.shape
+    N = wq.shape[0]
+    dbg = None
+    if want_acc:
+        dbg = ql.Debug(acc_i32=torch.empty((M, N), dtype=torch.int32, device="cuda")
+                       if scheme == ql.W8A8_INT8_ROW else None,
+                       acc_f32=torch.empty((M, N), dtype=torch.float32, device="cuda")
+                       if scheme == ql.FP8_E4M3_ROW else None)
+    ws_n = ql.workspace_bytes(scheme, M, N, K)
+    ws = ql.new_workspace(ws_n) if ws_n else None
+    ypad = torch.full((M * N + 64,), -7.0, dtype=torch.bfloat16, device="cuda")
+    y = ypad[:M * N].view(M, N)
+    ql.gemm(scheme, u8_dev(qx), f32_dev(sx), u8_dev(wq), f32_dev(sw), workspace=ws, y=y, debug=dbg)
+    st, detail = ql.device_status()
+    assert st == 0, f"device status {st} detail {detail:#x}"
+    assert np.all(bits(ypad[M * N:]) == bits(torch.tensor([-7.0], dtype=torch.bfloat16))[0]), \
+        "gemm wrote past the end of y"
+    return bits(y), dbg
+
+
+@pytest.mark.parametrize("scheme", [ql.W8A8_INT8_ROW, ql.FP8_E4M3_ROW])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (128, 256, 4096), (130, 300, 272), (33, 64, 48),
+                                   (1, 1000, 1024), (257, 520, 1040), (384, 768, 2048)])
+def test_gemm_small_shapes_full_compare(cuda, scheme, M, N, K):
+    qx, sx, wq, sw = _inputs(scheme, M, N, K)
+    gy, dbg = _gpu(scheme, qx, sx, wq, sw)
+    ry, racc_i, racc_d = oracle.linear(scheme, qx, sx, wq, sw, want_acc=True)
+    if scheme == ql.W8A8_INT8_ROW:
+        assert np.array_equal(dbg.acc_i32.cpu().numpy(), racc_i), "int32 accumulators differ"
+        assert np.array_equal(gy, ry), "int8 outputs must be bit-exact"
+    else:
+        acc = dbg.acc_f32.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(acc - racc_d) <= 1e-5 * np.abs(racc_d).max() + 1e-6)
+        assert_y_close(gy, ry, f"gemm {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (128, 256, 512), (200, 384, 640), (129, 1280, 1024),
+                                   (40, 256, 4096)])
+def test_gemm_block_small_shapes(cuda, M, N, K):
+    scheme = ql.FP8_E4M3_BLOCK128
+    qx, sx, wq, sw = _inputs(scheme, M, N, K, outliers=3)
+    gy, _ = _gpu(scheme, qx, sx, wq, sw, want_acc=False)
+    ry = oracle.linear(scheme, qx, sx, wq, sw)
+    assert_y_close(gy, ry, f"gemm block {M}x{N}x{K}")
+
+
+def _sampled_compare(scheme, M, N, K, nsamp=3000, seed=0):
+    qx, sx, wq, sw = _inputs(scheme, M, N, K, seed=seed)
+    gy, dbg = _gpu(scheme, qx, sx, wq, sw, want_acc=scheme == ql.W8A8_INT8_ROW)
+    rng = np.random.default_rng(seed + 99)
+    pm = np.concatenate([rng.integers(0, M, nsamp), np.full(N, M - 1), np.arange(M),
+                         [0, M - 1, 0, M - 1]])
+    pn = np.concatenate([rng.integers(0, N, nsamp), np.arange(N), np.full(M, N // 2 + 1),
+                         [0, 0, N - 1, N - 1]])
+    ry, racc_i, _ = oracle.linear_sampled(scheme, qx, sx, wq, sw, pm, pn, want_acc=True)
+    if scheme == ql.W8A8_INT8_ROW:
+        assert np.array_equal(dbg.acc_i32.cpu().numpy()[pm, pn], racc_i)
+        assert np.array_equal(gy[pm, pn], ry)
+    else:
+        assert_y_close(gy[pm, pn], ry, f"gemm {M}x{N}x{K} sampled")
+
+
+@pytest.mark.parametrize("M", [512, 1024])
+@pytest.mark.parametrize("name,N,K", synthetic.LLAMA31_8B_PREFILL)
+def test_gemm_prefill_w8a8_full_size(cuda, M, name, N, K):
+    _sampled_compare(ql.W8A8_INT8_ROW, M, N, K)
+
+
+@pytest.mark.parametrize("name,N,K", synthetic.LLAMA31_8B_PREFILL[::2])
+def test_gemm_prefill_fp8_row_full_size(cuda, name, N, K):
+    _sampled_compare(ql.FP8_E4M3_ROW, 512, N, K, nsamp=1500)
+
+
+@pytest.mark.parametrize("name,N,K", synthetic.QWEN3_8B)
+def test_gemm_qwen_block_m512_full_size(cuda, name, N, K):
+    _sampled_compare(ql.FP8_E4M3_BLOCK128, 512, N, K, nsamp=1500)
+
+
+def test_forward_dispatches_large_m_through_quant_and_gemm(cuda):
+    """qlinear_forward with M > 32: fused per-token quantization into the
+    workspace, then the GEMM; compared with the oracle's whole method."""
+    for scheme in ql.SCHEMES:
+        M, N, K = 96, 256, 512
+        x = synthetic.make_x(M, K, seed=3, tag="fwd-x", outliers=4)
+        w = synthetic.make_w(N, K, seed=3, tag="fwd-w")
+        wq, sw = oracle.quantize_weight(scheme, w)
+        ws = ql.new_workspace(ql.forward_workspace_bytes(scheme, M, N, K))
+        xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+        y = ql.forward(scheme, xd, u8_dev(wq), f32_dev(sw), workspace=ws)
+        torch.cuda.synchronize()
+        ry = oracle.forward(scheme, x, wq, sw)
+        if scheme == ql.W8A8_INT8_ROW:
+            assert np.array_equal(bits(y), ry)
+        else:
+            assert_y_close(bits(y), ry, "forward large M")
