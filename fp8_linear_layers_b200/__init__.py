@@ -39,7 +39,7 @@ STATUS = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED_SHAPE", 3:
 EXPORTS = ("qlinear_quantize_weight", "qlinear_quantize_act", "qlinear_gemv", "qlinear_gemm_small",
            "qlinear_gemm", "qlinear_forward", "qlinear_workspace_bytes",
            "qlinear_forward_workspace_bytes", "qlinear_get_device_status", "qlinear_status_string",
-           "qlinear_last_cuda_error")
+           "qlinear_last_cuda_error", "qlinear_gemm_small_noalloc")
 
 
 class QLinearError(RuntimeError):
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
         L.qlinear_gemm_small.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp, vp]
         L.qlinear_gemm.argtypes = [i32, vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp, vp]
         L.qlinear_forward.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]
+        L.qlinear_gemm_small_noalloc.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp]
         L.qlinear_workspace_bytes.argtypes = [i32, i64, i64, i64]
         L.qlinear_workspace_bytes.restype = sz
         L.qlinear_forward_workspace_bytes.argtypes = [i32, i64, i64, i64]
@@ -97,7 +98,7 @@ def lib() -> ctypes.CDLL:
         L.qlinear_last_cuda_error.restype = ctypes.c_char_p
         for name in ("qlinear_quantize_weight", "qlinear_quantize_act", "qlinear_gemv",
                      "qlinear_gemm_small", "qlinear_gemm", "qlinear_forward",
-                     "qlinear_get_device_status"):
+                     "qlinear_get_device_status", "qlinear_gemm_small_noalloc"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -205,6 +206,24 @@ def gemm_small(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
                                     _dev(y, torch.bfloat16, "y"), wp, wn,
                                     debug._c() if debug else None, _stream(stream)),
            "qlinear_gemm_small")
+    return y
+
+
+def gemm_small_noalloc(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor, y=None,
+                       stream=None):
+    """Same as ``gemm_small`` with the library's fixed device scratch instead of a
+    caller workspace (for callers that cannot allocate; calls must not overlap)."""
+    M, K = x.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    status = lib().qlinear_gemm_small_noalloc(scheme, _dev(x, torch.bfloat16, "x"),
+                                              _dev(wq, torch.uint8, "wq"), _dev(sw, torch.float32, "sw"),
+                                              M, N, K, _dev(y, torch.bfloat16, "y"), _stream(stream))
+    if status == 7:  # the shape needs more than the fixed scratch; the library says how much
+        raise QLinearError(status, "qlinear_gemm_small_noalloc",
+                           lib().qlinear_last_cuda_error().decode(errors="replace"))
+    _check(status, "qlinear_gemm_small_noalloc")
     return y
 
 

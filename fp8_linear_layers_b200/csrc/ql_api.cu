@@ -288,3 +288,73 @@ const char* qlinear_status_string(ql_status status) {
 const char* qlinear_last_cuda_error(void) { return g_last_cuda_error; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free small-M entry point.
+//
+// Scratch for qlinear_gemm_small_noalloc: a fixed array in device global
+// memory that every GPU loading the library holds until the process exits.
+// Host code must not hand `g_noalloc_scratch` itself to a kernel (on the host
+// it is only a stand-in symbol); it uses the device address looked up below.
+// ---------------------------------------------------------------------------
+static constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device, looked up once
+// per device with that device current.
+ql_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return QL_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return QL_OK;
+}
+}  // namespace
+
+extern "C" ql_status qlinear_gemm_small_noalloc(ql_scheme scheme, const uint16_t* x, const void* wq,
+                                                const float* sw, int64_t M, int64_t N, int64_t K,
+                                                uint16_t* y, void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_n(scheme, N, K));
+  QL_TRY(check_m(M, N, K));
+  if (M == 0) return QL_OK;
+  if (M > 32) return QL_ERR_UNSUPPORTED_SHAPE;
+  QL_TRY(need(x));
+  QL_TRY(need(wq));
+  QL_TRY(need(sw));
+  QL_TRY(need(y));
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  const size_t need_ws = ql::gemm_small_workspace_bytes(scheme, M, N, K, d.sms);
+  if (need_ws > kNoAllocScratchBytes) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "qlinear_gemm_small_noalloc: this shape needs %zu bytes of scratch, the static "
+                  "scratch holds %zu",
+                  need_ws, kNoAllocScratchBytes);
+    return QL_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  QL_TRY(noalloc_scratch(&scratch));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The split-tile arrival counters must start at zero; the scratch keeps
+  // whatever the previous call left, so clear them (no allocation involved).
+  const size_t counters = ql::gemm_small_counters_offset(scheme, M, N, K, d.sms);
+  cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(scratch) + counters, 0, need_ws - counters, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scratch counters)");
+  e = ql::launch_gemm_small(scheme, x, wq, sw, M, N, K, y, scratch, kNoAllocScratchBytes, nullptr,
+                            d.sms, d.status, st);
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm_small_noalloc");
+}

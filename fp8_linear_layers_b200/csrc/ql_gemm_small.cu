@@ -382,6 +382,10 @@ size_t gemm_small_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_
   return small_layout(scheme, M, N, K, num_sms).total;
 }
 
+size_t gemm_small_counters_offset(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms) {
+  return small_layout(scheme, M, N, K, num_sms).counters;
+}
+
 template <ql_scheme S, int NTOK>
 static cudaError_t launch_small_t(const SmallParams& p, const CUtensorMap& tw, const CUtensorMap& tx,
                                   int grid, cudaStream_t st) {

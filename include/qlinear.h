@@ -186,8 +186,38 @@ ql_status qlinear_get_device_status(void* stream, uint32_t* detail);
 /* Static description of a status code. */
 const char* qlinear_status_string(ql_status status);
 
-/* The CUDA error text behind the most recent QL_ERR_CUDA on this thread. */
+/* The CUDA error text behind the most recent QL_ERR_CUDA on this thread (and
+ * the reason for a QL_ERR_WORKSPACE from qlinear_gemm_small_noalloc). */
 const char* qlinear_last_cuda_error(void);
+
+/* qlinear_gemm_small without a caller-provided workspace.  The pages have no
+ * counterpart to this entry point: it exists for callers that cannot allocate
+ * device memory themselves -- plugin code inside a host framework that has
+ * reserved all device memory up front and hands out no allocator, a C caller
+ * with nowhere to keep a workspace pointer between calls, or a latency-
+ * critical path where cudaMalloc could stall or synchronise the device.
+ *
+ * The scratch (quantized tokens, per-SM partial sums, split-tile counters) is
+ * a fixed 8 MiB array in device global memory that the library declares at
+ * file scope; every GPU that loads the library holds it until the process
+ * exits.  This call allocates nothing and calls no allocating routine.
+ *   - Arguments, layouts, numerics and the 1 <= M <= 32 limit are those of
+ *     qlinear_gemm_small; the result is the same.
+ *   - A shape whose scratch need (qlinear_workspace_bytes) exceeds 8 MiB is
+ *     rejected with QL_ERR_WORKSPACE before anything is launched, and
+ *     qlinear_last_cuda_error() says how much it needed.  Every Llama-3.1-8B
+ *     and Qwen3-8B projection shape fits at M <= 32 on a 148-SM B200.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current (a one-time set-up); make that first call before
+ *     any stream capture.
+ *   - All calls share the one array and it keeps the previous call's
+ *     contents: each call clears the counters that must start at zero (an
+ *     asynchronous memset on `stream`).  Calls whose GPU work overlaps --
+ *     on different streams, or from different threads -- race on the array
+ *     and give wrong results; serialise them. */
+ql_status qlinear_gemm_small_noalloc(ql_scheme scheme, const uint16_t* x, const void* wq,
+                                     const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                     void* stream);
 
 #ifdef __cplusplus
 }
