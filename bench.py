@@ -1,26 +1,34 @@
 #!/usr/bin/env python3
 """Benchmark of the quantized decoder projection on B200.
 
-Default workload (one "step"): M = 1 decode through one Llama-3.1-8B layer's
-seven projections (q 4096x4096, k/v 1024x4096, o 4096x4096, gate/up
-14336x4096, down 4096x14336) in W8A8 int8 and in FP8 E4M3 per-row, i.e. 14
-GEMV launches (activation quantization fused) per step.  Metric: HBM GB/s of
-algorithmic bytes (weights + scales + x + y) per second, whole job.
+Default workload ("decode", one step): M = 1 decode through one
+Llama-3.1-8B layer's seven projections (q 4096x4096, k/v 1024x4096, o
+4096x4096, gate/up 14336x4096, down 4096x14336) in W8A8 int8 and in FP8 E4M3
+per-row: 14 GEMV launches (activation quantization fused) per step.  Metric:
+HBM GB/s of algorithmic bytes (weights + scales + x + y) per second, whole job.
 
-Legs:
-  value     device time of K steps, each step one CUDA graph replay of the 14
+Other workloads (``--workload``), same JSON line:
+  prefill       W8A8, M in {512, 1024} x gate/up/down/fused-qkv: TOPS
+  small         M in {2, 8, 16, 32} x the 7 Llama shapes x {W8A8, FP8 row}: GB/s
+  kproj         W8A8, M = 8, N = 1024, K = 4096 (8 outlier channels): GB/s
+  qwen-decode   FP8 128x128 block, M = 1 x the 7 Qwen3-8B shapes: GB/s
+  qwen-small    FP8 block, M = 32 x the Qwen shapes: GB/s
+  qwen-prefill  FP8 block, M = 512 x the Qwen shapes: TOPS
+
+Legs of the line:
+  value     device time of K steps, each one CUDA-graph replay of the step's
             launches (the pages decode under CUDA graphs); inputs resident in
-            HBM; 436 MB of weights per step, larger than L2, so every step
-            streams from HBM.
+            HBM; decode and small-M steps stream more than L2 every step.
   e2e       the same metric through the public API (``forward``) with the
-            step's tokens copied host->device from pinned memory and the
+            step's activations copied host->device from pinned memory and the
             outputs read back device->host every step (captured in a graph,
             host synchronised per step).
-  roofline  the GEMV kernel's algorithmic bytes per launch / its average
-            launch duration (step time / launches, CUDA events), against the
-            measured HBM copy bandwidth.
-  cpu_baseline  the CPU oracle (test infrastructure) on the same workload,
-            host cores, a bounded sample; reported, not the target.
+  roofline  the dominant kernel's algorithmic bytes (or ops) per launch over
+            its average launch duration, CUDA events, against the measured HBM
+            copy bandwidth or the measured bf16 GEMM rate x the nominal
+            8-bit/bf16 ratio of 2.
+  cpu_baseline  the CPU oracle (test infrastructure) on a bounded row sample
+            of the same workload, host cores; reported, not the target.
 
 ``--impl reference`` times the CPU oracle alone on the same metric (rank 0
 only).  Multi-GPU (torchrun): replicas, each rank runs the same step on its
@@ -36,23 +44,93 @@ import subprocess
 import sys
 import threading
 import time
+from dataclasses import dataclass, field
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "quantized linear: M=1 GEMV HBM GB/s; M≥512 int8/FP8 TOPS; % of B200 roofline"
-WORKLOAD = ("decode GEMV M=1: one Llama-3.1-8B layer's 7 projections "
-            "(q,k,v,o,gate,up,down) in W8A8 int8 and in FP8 E4M3 per-row, per-token dynamic "
-            "activation quantization fused")
 HBM_FALLBACK_GBS = 6650.0
+BF16_FALLBACK_TFLOPS = 1590.0
+INT8, FP8R, FP8B = 0, 1, 2
+SCHEME_NAME = {INT8: "w8a8_int8_row", FP8R: "fp8_e4m3_row", FP8B: "fp8_e4m3_block128"}
+
+
+# ------------------------------------------------------------------ workloads
+@dataclass
+class Product:
+    name: str
+    scheme: int
+    M: int
+    N: int
+    K: int
+    outliers: int
+
+
+@dataclass
+class Workload:
+    key: str
+    description: str
+    unit: str                # "GB/s" or "TOPS"
+    products: list = field(default_factory=list)
+
+    @property
+    def bound(self):
+        return "hbm" if self.unit == "GB/s" else "tensor"
+
+    @property
+    def kernel(self):
+        M = self.products[0].M
+        return "ql::gemv_kernel" if M == 1 else ("ql::gemm_small_kernel" if M <= 32 else "ql::gemm_kernel")
+
+    def amount(self, p: Product) -> float:
+        """Algorithmic bytes (HBM-bound regimes) or ops (tensor-bound) of one product."""
+        if self.unit == "TOPS":
+            return 2.0 * p.M * p.N * p.K
+        sw = 4 * (p.N // 128) * (p.K // 128) if p.scheme == FP8B else 4 * p.N
+        return p.N * p.K + sw + 2 * p.M * p.K + 2 * p.M * p.N
+
+
+def workloads():
+    from fp8_linear_layers_b200 import synthetic as S
+    oc = S.outlier_count
+    w = {}
+    w["decode"] = Workload(
+        "decode", "decode GEMV M=1: one Llama-3.1-8B layer's 7 projections (q,k,v,o,gate,up,down) "
+        "in W8A8 int8 and in FP8 E4M3 per-row, per-token dynamic activation quantization fused", "GB/s",
+        [Product(n, s, 1, N, K, oc(K)) for n, N, K in S.LLAMA31_8B for s in (INT8, FP8R)])
+    w["prefill"] = Workload(
+        "prefill", "prefill W8A8 int8 GEMM: M in {512, 1024} x Llama-3.1-8B gate/up 14336x4096, "
+        "down 4096x14336, fused qkv 6144x4096; per-token quantization + tcgen05 kind::i8", "TOPS",
+        [Product(n, INT8, M, N, K, oc(K)) for M in (512, 1024) for n, N, K in S.LLAMA31_8B_PREFILL])
+    w["small"] = Workload(
+        "small", "small-batch tensor-core path: M in {2, 8, 16, 32} x the 7 Llama-3.1-8B shapes x "
+        "{W8A8 int8, FP8 E4M3 per-row}, quantization fused", "GB/s",
+        [Product(n, s, M, N, K, oc(K)) for M in (2, 8, 16, 32) for s in (INT8, FP8R)
+         for n, N, K in S.LLAMA31_8B])
+    w["kproj"] = Workload(
+        "kproj", "W8A8 int8 k_proj shape: X [8, 4096] with 8 outlier channels, W [1024, 4096]",
+        "GB/s", [Product("k_proj", INT8, 8, 1024, 4096, 8)])
+    w["qwen-decode"] = Workload(
+        "qwen-decode", "Qwen3-8B FP8 128x128-block projections at M=1 (7 shapes)", "GB/s",
+        [Product(n, FP8B, 1, N, K, 0) for n, N, K in S.QWEN3_8B])
+    w["qwen-small"] = Workload(
+        "qwen-small", "Qwen3-8B FP8 128x128-block projections at M=32 (7 shapes)", "GB/s",
+        [Product(n, FP8B, 32, N, K, 0) for n, N, K in S.QWEN3_8B])
+    w["qwen-prefill"] = Workload(
+        "qwen-prefill", "Qwen3-8B FP8 128x128-block projections at M=512 (7 shapes), per-K-block "
+        "promotion", "TOPS", [Product(n, FP8B, 512, N, K, 0) for n, N, K in S.QWEN3_8B])
+    return w
 
 
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["qlinear", "reference"], default="qlinear")
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "prefill", "small", "kproj", "qwen-decode", "qwen-small", "qwen-prefill"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -60,21 +138,21 @@ def parse_args():
     return ap.parse_args()
 
 
-def algorithmic_bytes(scheme: int, N: int, K: int, M: int = 1) -> int:
-    """Bytes the method must move for one product: weights, weight scales,
-    bf16 activations in, bf16 outputs out."""
-    sw = 4 * (N // 128) * (K // 128) if scheme == 2 else 4 * N
-    return N * K + sw + 2 * M * K + 2 * M * N
-
-
 def measured_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
-        with open(p) as f:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             return json.load(f), "measured"
     except (OSError, ValueError):
-        return {"hbm_gbs": HBM_FALLBACK_GBS, "bf16_tflops": 1590.0,
+        return {"hbm_gbs": HBM_FALLBACK_GBS, "bf16_tflops": BF16_FALLBACK_TFLOPS,
                 "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def roofline_peak(wl: Workload):
+    peaks, src = measured_peaks()
+    if wl.unit == "GB/s":
+        return float(peaks["hbm_gbs"]), f"{src} HBM copy bandwidth (hbm_gbs)"
+    # 8-bit (int8 / E4M3) dense tensor rate = measured bf16 burst x nominal ratio 4.5/2.25
+    return 2.0 * float(peaks["bf16_tflops"]), f"{src} bf16 GEMM burst x 2 (nominal 8-bit/bf16 ratio)"
 
 
 # ------------------------------------------------------------------ clocks
@@ -85,10 +163,7 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
-        self.idx = gpu_index
-        self.proc = None
-        self.lines = []
-        self.thread = None
+        self.idx, self.proc, self.lines, self.thread = gpu_index, None, [], None
 
     def start(self):
         if self.idx is None:
@@ -155,127 +230,165 @@ def nvsmi_index(torch, dev: int):
     return None
 
 
-# ------------------------------------------------------------------ workload
-def build_decode(torch, ql, synthetic, device, tokens=2):
-    """Quantized weights (on the GPU, by the library's own quantizer) and a
-    small rotation of input tokens for each projection."""
-    work = []
-    for name, N, K in synthetic.LLAMA31_8B:
-        w = synthetic.make_w_device(N, K, seed=0, tag=f"llama31_8b.{name}", device=device)
-        xs = synthetic.make_x_device(tokens, K, seed=0, tag=f"llama31_8b.{name}.x",
-                                     outliers=synthetic.outlier_count(K), device=device)
-        for scheme in (ql.W8A8_INT8_ROW, ql.FP8_E4M3_ROW):
-            wq, sw = ql.quantize_weight(scheme, w)
-            work.append(dict(name=name, scheme=scheme, N=N, K=K, wq=wq, sw=sw, xs=xs,
-                             bytes=algorithmic_bytes(scheme, N, K)))
-        del w
-    torch.cuda.synchronize()
-    return work
+# ------------------------------------------------------------------ GPU legs
+class Runner:
+    """Device buffers and launch closures for one workload (public API calls only)."""
 
+    def __init__(self, torch, ql, synthetic, wl: Workload, tokens: int = 2):
+        self.torch, self.ql, self.wl, self.tokens = torch, ql, wl, tokens
+        self.items = []
+        weights = {}
+        for p in wl.products:
+            key = (p.name, p.N, p.K)
+            if key not in weights:
+                weights[key] = synthetic.make_w_device(p.N, p.K, seed=0, tag=f"bench.{p.name}")
+            wq, sw = ql.quantize_weight(p.scheme, weights[key])
+            xs = [synthetic.make_x_device(p.M, p.K, seed=t, tag=f"bench.{p.name}.x.M{p.M}",
+                                          outliers=p.outliers) for t in range(tokens)]
+            ys = [torch.empty((p.M, p.N), dtype=torch.bfloat16, device="cuda") for _ in range(tokens)]
+            ws_bytes = ql.forward_workspace_bytes(p.scheme, p.M, p.N, p.K)
+            ws = ql.new_workspace(ws_bytes) if ws_bytes else None
+            item = dict(p=p, wq=wq, sw=sw, xs=xs, ys=ys, ws=ws, amount=wl.amount(p))
+            if p.M > 32:  # pre-quantized activations for the dominant-kernel timing
+                item["q"] = [ql.quantize_act(p.scheme, x) for x in xs]
+            self.items.append(item)
+        del weights
+        torch.cuda.synchronize()
+        self.step_amount = sum(i["amount"] for i in self.items)
+        self.launches_per_step = sum(1 if i["p"].M == 1 else 2 for i in self.items)
 
-def capture_step_graphs(torch, ql, work, tokens, stream):
-    """One CUDA graph per token slot, each holding the step's 14 GEMV launches."""
-    for item in work:
-        item["ys"] = [torch.empty((1, item["N"]), dtype=torch.bfloat16, device="cuda")
-                      for _ in range(tokens)]
-    # warm the launch path (device info, shared-memory attribute) before capture
-    with torch.cuda.stream(stream):
-        for item in work:
-            ql.gemv(item["scheme"], item["xs"][0:1], item["wq"], item["sw"], y=item["ys"][0])
-    stream.synchronize()
-    graphs = []
-    for t in range(tokens):
+    def step(self, t):
+        ql = self.ql
+        for i in self.items:
+            ql.forward(i["p"].scheme, i["xs"][t], i["wq"], i["sw"], workspace=i["ws"], y=i["ys"][t])
+
+    def dominant(self, t):
+        """Launches of the dominant kernel alone (the product on quantized inputs)."""
+        ql = self.ql
+        for i in self.items:
+            p = i["p"]
+            if p.M == 1:
+                ql.gemv(p.scheme, i["xs"][t], i["wq"], i["sw"], y=i["ys"][t])
+            elif p.M <= 32:
+                ql.gemm_small(p.scheme, i["xs"][t], i["wq"], i["sw"], i["ws"], y=i["ys"][t])
+            else:
+                qx, sx = i["q"][t]
+                ql.gemm(p.scheme, qx, sx, i["wq"], i["sw"], y=i["ys"][t])
+
+    def capture(self, fn, stream):
+        torch = self.torch
+        with torch.cuda.stream(stream):
+            fn(0)  # warms the launch path (device info, attributes) before capture
+        stream.synchronize()
+        graphs = []
+        for t in range(self.tokens):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn(t)
+            graphs.append(g)
+        return graphs
+
+    def e2e_graph(self, stream):
+        """H2D of every product's activations (pinned host -> device), the
+        public forward() calls, D2H of every output."""
+        torch, ql = self.torch, self.ql
+        xs_tot = sum(i["p"].M * i["p"].K for i in self.items)
+        ys_tot = sum(i["p"].M * i["p"].N for i in self.items)
+        h_x = torch.empty(xs_tot, dtype=torch.bfloat16, pin_memory=True)
+        h_y = torch.empty(ys_tot, dtype=torch.bfloat16, pin_memory=True)
+        d_x = torch.empty(xs_tot, dtype=torch.bfloat16, device="cuda")
+        d_y = torch.empty(ys_tot, dtype=torch.bfloat16, device="cuda")
+        views, ox, oy = [], 0, 0
+        for i in self.items:
+            p = i["p"]
+            h_x[ox:ox + p.M * p.K].copy_(i["xs"][0].reshape(-1).cpu())
+            views.append((i, d_x[ox:ox + p.M * p.K].view(p.M, p.K), d_y[oy:oy + p.M * p.N].view(p.M, p.N)))
+            ox += p.M * p.K
+            oy += p.M * p.N
+
+        def body():
+            for i, xv, yv in views:
+                ql.forward(i["p"].scheme, xv, i["wq"], i["sw"], workspace=i["ws"], y=yv)
+
+        with torch.cuda.stream(stream):
+            body()
+        stream.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            for item in work:
-                ql.gemv(item["scheme"], item["xs"][t:t + 1], item["wq"], item["sw"], y=item["ys"][t])
-        graphs.append(g)
-    return graphs
+            d_x.copy_(h_x, non_blocking=True)
+            body()
+            h_y.copy_(d_y, non_blocking=True)
+        return g, 2 * xs_tot, 2 * ys_tot
 
 
-def capture_e2e_graph(torch, ql, work, stream):
-    """Graph of one end-to-end step: H2D of all 14 tokens (pinned host ->
-    device), 14 public-API forward() calls, D2H of all outputs."""
-    K_tot = sum(i["K"] for i in work)
-    N_tot = sum(i["N"] for i in work)
-    h_x = torch.empty(K_tot, dtype=torch.bfloat16, pin_memory=True)
-    h_y = torch.empty(N_tot, dtype=torch.bfloat16, pin_memory=True)
-    off = 0
-    for i in work:
-        h_x[off:off + i["K"]].copy_(i["xs"][0].cpu())
-        off += i["K"]
-    d_x = torch.empty(K_tot, dtype=torch.bfloat16, device="cuda")
-    d_y = torch.empty(N_tot, dtype=torch.bfloat16, device="cuda")
-    views = []
-    ox = oy = 0
-    for i in work:
-        views.append((i, d_x[ox:ox + i["K"]].view(1, -1), d_y[oy:oy + i["N"]].view(1, -1)))
-        ox += i["K"]
-        oy += i["N"]
+def timed(torch, stream, graphs, steps):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        for i, xv, yv in views:
-            ql.forward(i["scheme"], xv, i["wq"], i["sw"], y=yv)
-    stream.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        d_x.copy_(h_x, non_blocking=True)
-        for i, xv, yv in views:
-            ql.forward(i["scheme"], xv, i["wq"], i["sw"], y=yv)
-        h_y.copy_(d_y, non_blocking=True)
-    return g, 2 * K_tot, 2 * N_tot
+        e0.record(stream)
+        for i in range(steps):
+            graphs[i % len(graphs)].replay()
+        e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1)
 
 
 # ------------------------------------------------------------------ CPU oracle
-def oracle_decode_sample(budget_s: float, rows_cap=None):
-    """Time the CPU oracle on the decode step (or a row sample of it) for about
-    budget_s seconds.  Returns (GB/s, seconds, sample description)."""
-    import numpy as np
+def _oracle_items(wl: Workload, rows_cap: int):
     import oracle
     from fp8_linear_layers_b200 import synthetic
     items = []
-    for name, N, K in synthetic.LLAMA31_8B:
-        rows = N if rows_cap is None else min(N, rows_cap)
-        w = synthetic.make_w(rows, K, seed=0, tag=f"oracle.llama31_8b.{name}")
-        x = synthetic.make_x(1, K, seed=0, tag=f"oracle.llama31_8b.{name}.x",
-                             outliers=synthetic.outlier_count(K))
-        for scheme in (0, 1):
-            wq, sw = oracle.quantize_weight(scheme, w)
-            items.append((scheme, x, wq, sw, algorithmic_bytes(scheme, rows, K)))
-    done_bytes, t_used, reps = 0, 0.0, 0
-    while t_used < budget_s or reps == 0:
+    for p in wl.products:
+        rows = min(p.N, rows_cap)
+        if p.scheme == FP8B:
+            rows = max(128, rows // 128 * 128)
+        w = synthetic.make_w(rows, p.K, seed=0, tag=f"oracle.{p.name}")
+        x = synthetic.make_x(p.M, p.K, seed=0, tag=f"oracle.{p.name}.x", outliers=p.outliers)
+        wq, sw = oracle.quantize_weight(p.scheme, w)
+        items.append((p.scheme, x, wq, sw, wl.amount(Product(p.name, p.scheme, p.M, rows, p.K, 0))))
+    return items
+
+
+def oracle_sample(wl: Workload, budget_s: float, rows_cap: int):
+    """The CPU oracle (whole method from bf16 X) on the first rows_cap output
+    rows of every product of the workload, repeated for about budget_s.
+    Returns (throughput in the workload's unit, seconds, passes, amount per pass)."""
+    import oracle
+    items = _oracle_items(wl, rows_cap)
+    per_pass = sum(i[4] for i in items)
+    done, t_used, passes = 0.0, 0.0, 0
+    while t_used < budget_s or passes == 0:
         t0 = time.perf_counter()
-        for scheme, x, wq, sw, nb in items:
+        for scheme, x, wq, sw, amt in items:
             oracle.forward(scheme, x, wq, sw)
-            done_bytes += nb
+            done += amt
         t_used += time.perf_counter() - t0
-        reps += 1
-    what = "full step" if rows_cap is None else f"first {rows_cap} output rows of each projection"
-    return done_bytes / t_used / 1e9, t_used, f"{what} (14 GEMVs, M=1) x {reps} passes, {t_used:.1f} s"
+        passes += 1
+    scale = 1e9 if wl.unit == "GB/s" else 1e12
+    return done / t_used / scale, t_used, passes, per_pass
 
 
-# ------------------------------------------------------------------ main legs
+def pick_rows(wl: Workload, seconds: float) -> int:
+    """Rows per product so that one oracle pass takes about `seconds`."""
+    _, t, _, _ = oracle_sample(wl, 0.0, 8)
+    return max(1, int(8 * seconds / max(t, 1e-6)))
+
+
+def base_line(wl, args, world):
+    return {"metric": METRIC, "unit": wl.unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "s8*s8->s32 (W8A8), e4m3*e4m3->f32 (FP8)",
+            "data": "synthetic (seeded N(0,1) activations with outlier channels x20; N(0,0.02) weights)"}
+
+
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    if int(os.environ.get("RANK", "0")) != 0:
         return 0
-    # calibrate the per-step sample so that warmup + steps take about a minute
-    from fp8_linear_layers_b200 import synthetic
     import oracle
-    _, t64, _ = oracle_decode_sample(0.0, rows_cap=64)  # one pass over 64 rows per projection
-    per_step_target = max(0.002, 60.0 / max(1, args.steps + args.warmup))
-    rows = max(1, min(14336, int(64 * per_step_target / max(t64, 1e-6))))
-    full_bytes = sum(algorithmic_bytes(s, N, K) for _, N, K in synthetic.LLAMA31_8B for s in (0, 1))
-    import numpy as np
-    items = []
-    for name, N, K in synthetic.LLAMA31_8B:
-        r = min(N, rows)
-        w = synthetic.make_w(r, K, seed=0, tag=f"oracle.llama31_8b.{name}")
-        x = synthetic.make_x(1, K, seed=0, tag=f"oracle.llama31_8b.{name}.x",
-                             outliers=synthetic.outlier_count(K))
-        for scheme in (0, 1):
-            wq, sw = oracle.quantize_weight(scheme, w)
-            items.append((scheme, x, wq, sw, algorithmic_bytes(scheme, r, K)))
-    step_bytes = sum(i[4] for i in items)
+    wl = workloads()[args.workload]
+    per_step = max(0.002, 60.0 / max(1, args.steps + args.warmup))
+    rows = pick_rows(wl, per_step)
+    items = _oracle_items(wl, rows)
+    step_amount = sum(i[4] for i in items)
     for _ in range(args.warmup):
         for scheme, x, wq, sw, _ in items:
             oracle.forward(scheme, x, wq, sw)
@@ -284,20 +397,20 @@ def run_reference(args):
         for scheme, x, wq, sw, _ in items:
             oracle.forward(scheme, x, wq, sw)
     dt = time.perf_counter() - t0
-    value = step_bytes * args.steps / dt / 1e9
-    sample = (f"first {rows} output rows of each of the 14 projections (M=1), "
-              f"{step_bytes / full_bytes * 100:.2f}% of a full step, per step")
-    line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "s8*s8->s32 (int8), e4m3*e4m3 exact (int64 fixed point)",
-        "data": "synthetic (seeded N(0,1) tokens with 1% outlier channels x20; N(0,0.02) weights)",
-        "config": {"workload": WORKLOAD, "M": 1, "note": "CPU oracle, single thread"},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
-        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
+    scale = 1e9 if wl.unit == "GB/s" else 1e12
+    value = step_amount * args.steps / dt / scale
+    full = sum(wl.amount(p) for p in wl.products)
+    sample = (f"first {rows} output rows of each of the workload's {len(items)} products, "
+              f"{100 * step_amount / full:.3g}% of a full step, per step; single thread")
+    line = base_line(wl, args, args.gpus)
+    line.update({"value": value, "impl": "reference", "ms_per_step": dt / args.steps * 1e3,
+                 "dtype": "s8*s8->s32 (int8), e4m3*e4m3 exact (int64 fixed point)",
+                 "config": {"workload": wl.description, "key": wl.key,
+                            "note": "CPU oracle, the plain definition"},
+                 "cpu_baseline": {"value": value, "unit": wl.unit, "cores": 1, "kind": "oracle",
+                                  "sample": sample},
+                 "e2e": {"value": value, "unit": wl.unit, "h2d_bytes_per_step": 0,
+                         "d2h_bytes_per_step": 0}})
     print(json.dumps(line), flush=True)
     return 0
 
@@ -335,123 +448,103 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    peaks, peak_src = measured_peaks()
-    tokens = 2
+    wl = workloads()[args.workload]
+    scale = 1e9 if wl.unit == "GB/s" else 1e12
     stream = torch.cuda.Stream()
-    work = build_decode(torch, ql, synthetic, "cuda", tokens)
-    graphs = capture_step_graphs(torch, ql, work, tokens, stream)
-    launches_per_step = len(work)
-    step_bytes = sum(i["bytes"] for i in work)
+    run = Runner(torch, ql, synthetic, wl)
+    graphs = run.capture(run.step, stream)
 
+    # ---- timed region: K steps, one graph replay each
     sampler = ClockSampler(nvsmi_index(torch, dev) if rank == 0 else None).start()
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            graphs[i % tokens].replay()
+            graphs[i % len(graphs)].replay()
     stream.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        for i in range(args.steps):
-            graphs[i % tokens].replay()
-        ev1.record(stream)
-    ev1.synchronize()
+    ms_local = timed(torch, stream, graphs, args.steps)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    ms_local = ev0.elapsed_time(ev1)
     ms = max_over_ranks(ms_local)
-    value = world * step_bytes * args.steps / (ms / 1e3) / 1e9
+    value = world * run.step_amount * args.steps / (ms / 1e3) / scale
     status, detail = ql.device_status(stream)
     if status != 0:
         raise RuntimeError(f"device status {status} detail {detail:#x} after the timed region")
 
-    # per-projection kernel durations (outside the timed region), for the record
-    per_kernel = {}
-    for item in work:
-        g = torch.cuda.CUDAGraph()
-        y = item["ys"][0]
-        with torch.cuda.graph(g, stream=stream):
-            for _ in range(10):
-                ql.gemv(item["scheme"], item["xs"][0:1], item["wq"], item["sw"], y=y)
-        with torch.cuda.stream(stream):
-            g.replay()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(5):
-                g.replay()
-            b.record(stream)
-        b.synchronize()
-        us = a.elapsed_time(b) * 1e3 / 50
-        key = f"{ql.SCHEME_NAMES[item['scheme']]}.{item['name']}"
-        per_kernel[key] = {"us": round(us, 2), "GB/s": round(item["bytes"] / us / 1e3, 1)}
-        del g
-
-    # end-to-end through the public API with host buffers
-    e2e_steps = args.e2e_steps or max(10, min(args.steps, 2000))
-    g_e2e, h2d, d2h = capture_e2e_graph(torch, ql, work, stream)
+    # ---- the dominant kernel's own launches (for the roofline), same kind of timing
+    dgraphs = run.capture(run.dominant, stream)
+    dsteps = max(3, min(args.steps, 500))
     with torch.cuda.stream(stream):
-        for _ in range(min(args.warmup, 20)):
+        for i in range(min(args.warmup, 10)):
+            dgraphs[i % len(dgraphs)].replay()
+    d_ms = timed(torch, stream, dgraphs, dsteps)
+    n_dom = len(run.items)
+    per_launch_amount = run.step_amount / n_dom
+    per_launch_s = (d_ms / 1e3) / (dsteps * n_dom)
+    achieved = per_launch_amount / per_launch_s / scale
+    peak, peak_src = roofline_peak(wl)
+    roofline = {"bound": wl.bound, "achieved": round(achieved, 1), "peak": round(peak, 1),
+                "unit": wl.unit, "frac": round(achieved / peak, 4), "traffic": None,
+                "kernel": wl.kernel, "peak_source": peak_src,
+                "duration_source": "CUDA events over graph replays of this kernel's launches "
+                                   "(inputs already quantized where the step quantizes separately)"}
+    del dgraphs
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = args.e2e_steps or max(10, min(args.steps, 1000))
+    g_e2e, h2d, d2h = run.e2e_graph(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(min(args.warmup, 10)):
             g_e2e.replay()
             stream.synchronize()
     barrier()
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
         for _ in range(e2e_steps):
             g_e2e.replay()
-            stream.synchronize()  # the host reads each step's outputs
+            stream.synchronize()  # the host reads every step's outputs
         e1.record(stream)
     e1.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * step_bytes * e2e_steps / (e2e_ms / 1e3) / 1e9
+    e2e_value = world * run.step_amount * e2e_steps / (e2e_ms / 1e3) / scale
     del g_e2e
-
-    # roofline of the (only) kernel: average algorithmic bytes per launch over
-    # the average launch duration inside the timed region
-    per_launch_bytes = step_bytes / launches_per_step
-    per_launch_s = (ms_local / 1e3) / (args.steps * launches_per_step)
-    achieved = per_launch_bytes / per_launch_s / 1e9
-    peak = float(peaks["hbm_gbs"])
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
-                "kernel": "ql::gemv_kernel", "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
-                if peak_src == "measured" else "fallback 6.65 TB/s",
-                "duration_source": "timed-region step time / launches (graph gaps included)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, secs, sample = oracle_decode_sample(args.cpu_seconds)
-        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample}
+        rows = pick_rows(wl, min(args.cpu_seconds, 4.0))
+        v, secs, passes, per_pass = oracle_sample(wl, args.cpu_seconds, rows)
+        cpu = {"value": round(v, 6), "unit": wl.unit, "cores": 1, "kind": "oracle",
+               "sample": f"first {rows} output rows of each of the {len(wl.products)} products "
+                         f"({100 * per_pass / run.step_amount:.3g}% of a step) x {passes} passes, "
+                         f"{secs:.1f} s, single thread"}
 
     if rank == 0:
-        line = {
-            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "s8*s8->s32 (W8A8), e4m3*e4m3->f32 (FP8 row)",
-            "data": "synthetic (seeded N(0,1) tokens with 1% outlier channels x20; N(0,0.02) "
-                    "weights quantized on the GPU)",
-            "config": {"workload": WORKLOAD, "M": 1,
-                       "shapes": [f"{n} {N}x{K}" for n, N, K in synthetic.LLAMA31_8B],
-                       "schemes": ["w8a8_int8_row", "fp8_e4m3_row"], "launches_per_step": launches_per_step,
-                       "bytes_per_step": step_bytes, "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2: 436 MB of weights streamed per step (L2 126 MB)",
+        line = base_line(wl, args, world)
+        weight_bytes = sum(p.N * p.K for p in wl.products)
+        line.update({
+            "value": round(value, 1), "ms_per_step": ms / args.steps,
+            "config": {"workload": wl.description, "key": wl.key,
+                       "products": [f"{SCHEME_NAME[p.scheme]} M={p.M} {p.name} {p.N}x{p.K}"
+                                    for p in wl.products],
+                       "launches_per_step": run.launches_per_step,
+                       "amount_per_step": run.step_amount, "parallelism": f"replicas x{world}",
+                       "l2": (f"inputs larger than L2 (126 MB): {weight_bytes / 1e6:.0f} MB of weights "
+                              "per step") if weight_bytes > 126e6 else
+                             (f"{weight_bytes / 1e6:.0f} MB of weights per step, under the 126 MB L2: "
+                              "not flushed between steps"),
                        "timing": "one CUDA graph replay per step, CUDA events on the launch stream"},
             "roofline": roofline,
             "cpu_baseline": cpu,
-            "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": round(e2e_value, 1), "unit": wl.unit, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                    "how": "graph of H2D tokens + 14 forward() + D2H outputs, host sync per step"},
-            "gpu_launches": launches_per_step * args.steps,
+                    "how": "graph of H2D activations + forward() per product + D2H outputs, "
+                           "host sync per step"},
+            "gpu_launches": run.launches_per_step * args.steps,
             "clocks": clocks,
-            "per_kernel": per_kernel,
-        }
+        })
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -173,15 +173,115 @@ QL_DEVINL float f16_hi_to_f32(uint32_t h2) {
   return f;
 }
 
-// Activation / weight code for one value: int8 clamp(rne(x/s)) or E4M3(x/s).
-// The quotient is one IEEE f32 division (the library is built without fast
-// math), and a zero scale (all-zero token, group or row) gives code 0.
-QL_DEVINL int int8_code(float x, float s) {
-  float t = (s > 0.0f) ? (x / s) : 0.0f;
-  int q = __float2int_rn(t);
-  return max(-127, min(127, q));
+// Quantization of one 16-byte chunk (8 bf16 values) with one scale s:
+// int8 code clamp(rne(x/s), -127, 127) or E4M3 code of x/s, x/s the
+// correctly rounded f32 quotient (the value one IEEE division gives); a zero
+// scale (all-zero token, group or row) gives codes 0.
+//
+// For 2^-100 <= s <= 2^100 ("fast" scales) the quotient takes the correctly
+// rounded reciprocal r of s and two correction steps of Markstein's method
+// (P. W. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Develop. 34(1), 1990): q = x r, then
+// q <- q + (x - s q) r twice, the residual exact through an FMA.  The code is
+// branch-free, so the eight values of a chunk run side by side.  Other scales
+// take the IEEE division.  The GPU tests compare the codes bit for bit with
+// codes from IEEE division on every bf16 x at scales on both sides of the
+// range.
+struct Divisor {
+  float s, r;
+  bool fast;
+};
+QL_DEVINL Divisor make_divisor(float s) {
+  Divisor d;
+  d.s = s;
+  d.fast = s >= 0x1p-100f && s <= 0x1p100f;
+  d.r = d.fast ? __frcp_rn(s) : 0.0f;
+  return d;
 }
-QL_DEVINL float e4m3_quotient(float x, float s) { return (s > 0.0f) ? (x / s) : 0.0f; }
+
+// x / s for a fast scale; the sign of a zero result is not fixed here.
+QL_DEVINL float quotient_fast(float x, const Divisor& d) {
+  float q = __fmul_rn(x, d.r);
+  float e = __fmaf_rn(-q, d.s, x);
+  q = __fmaf_rn(e, d.r, q);
+  e = __fmaf_rn(-q, d.s, x);
+  return __fmaf_rn(e, d.r, q);
+}
+
+// int8 code in bits [7:0] (the other bits are not part of the result).
+// Fast scales: clamp first (the same code for every x), then adding 1.5 * 2^23
+// rounds to the nearest integer, ties to even, and leaves that integer in the
+// low bits of the sum (|t| <= 127, far inside 2^22).
+QL_DEVINL uint32_t int8_bits_fast(float x, const Divisor& d) {
+  const float t = fminf(fmaxf(quotient_fast(x, d), -127.0f), 127.0f);
+  return __float_as_uint(__fadd_rn(t, 0x1.8p23f));
+}
+QL_DEVINL uint32_t int8_bits_ieee(float x, const Divisor& d) {
+  const int q = __float2int_rn(d.s > 0.0f ? x / d.s : 0.0f);
+  return (uint32_t)max(-127, min(127, q));
+}
+// The correctly rounded quotient of a finite x by s > 0 has the sign of x,
+// which also decides the E4M3 code of a zero (0x00 / 0x80).
+QL_DEVINL float e4m3_quotient_fast(float x, const Divisor& d) {
+  return copysignf(quotient_fast(x, d), x);
+}
+QL_DEVINL float e4m3_quotient_ieee(float x, const Divisor& d) {
+  return d.s > 0.0f ? x / d.s : 0.0f;
+}
+
+// Bytes [7:0] of a, b, c, d -> one word, a in the lowest byte.
+QL_DEVINL uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+template <bool kInt8, bool kFast>
+QL_DEVINL uint2 quant_chunk8(const uint4& v, const Divisor& d) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float f[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    f[2 * j] = bf16_lo(w[j]);
+    f[2 * j + 1] = bf16_hi(w[j]);
+  }
+  uint32_t o[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float* g = f + 4 * h;
+    if constexpr (kInt8) {
+      if constexpr (kFast)
+        o[h] = pack_low_bytes(int8_bits_fast(g[0], d), int8_bits_fast(g[1], d),
+                              int8_bits_fast(g[2], d), int8_bits_fast(g[3], d));
+      else
+        o[h] = pack_low_bytes(int8_bits_ieee(g[0], d), int8_bits_ieee(g[1], d),
+                              int8_bits_ieee(g[2], d), int8_bits_ieee(g[3], d));
+    } else {
+      if constexpr (kFast)
+        o[h] = __byte_perm(f32x2_to_e4m3x2(e4m3_quotient_fast(g[0], d), e4m3_quotient_fast(g[1], d)),
+                           f32x2_to_e4m3x2(e4m3_quotient_fast(g[2], d), e4m3_quotient_fast(g[3], d)),
+                           0x5410);
+      else
+        o[h] = __byte_perm(f32x2_to_e4m3x2(e4m3_quotient_ieee(g[0], d), e4m3_quotient_ieee(g[1], d)),
+                           f32x2_to_e4m3x2(e4m3_quotient_ieee(g[2], d), e4m3_quotient_ieee(g[3], d)),
+                           0x5410);
+    }
+  }
+  return make_uint2(o[0], o[1]);
+}
+
+// Either path, chosen per chunk (uniform where the scale is).
+template <bool kInt8>
+QL_DEVINL uint2 quant_chunk8(const uint4& v, const Divisor& d) {
+  return d.fast ? quant_chunk8<kInt8, true>(v, d) : quant_chunk8<kInt8, false>(v, d);
+}
+
+// Largest |x| of one chunk of 8 bf16.
+QL_DEVINL float absmax_chunk8(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float a = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+  return a;
+}
 
 QL_DEVINL float warp_max(float v) {
 #pragma unroll

@@ -293,14 +293,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         float acc[Cfg::kHalf];
 #pragma unroll
         for (int j = 0; j < Cfg::kHalf; ++j) acc[j] = 0.0f;
+        // scales of K block kb+1 are loaded while the MMAs of block kb run
+        const bool live = live_m && live_n;
+        float sx_next = live ? __ldg(p.sx + (int64_t)m * KB) : 0.0f;
+        float sw_next = live ? __ldg(p.sw + (int64_t)nbw * KB) : 0.0f;
         for (int kb = 0; kb < p.nkb; ++kb) {
+          const float scale = sx_next * sw_next;
+          if (live && kb + 1 < p.nkb) {
+            sx_next = __ldg(p.sx + (int64_t)m * KB + kb + 1);
+            sw_next = __ldg(p.sw + (int64_t)nbw * KB + kb + 1);
+          }
           const uint32_t buf = jt % kBufs;
           ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kBufs) & 1, abort_flag));
           if (!ok) break;
           tc::fence_after();
-          const float scale = (live_m && live_n)
-                                  ? __ldg(p.sx + (int64_t)m * KB + kb) * __ldg(p.sw + (int64_t)nbw * KB + kb)
-                                  : 0.0f;
 #pragma unroll
           for (int c = 0; c < Cfg::kHalf / 32; ++c) {
             uint32_t r[32];

@@ -254,8 +254,23 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         ++jt;
       } else if (kBlock) {
         const float* swt = p.sw + (int64_t)t * KB;
+        // the next K block's scales are loaded while this block's MMAs run
+        float sx_next[NTOK];
+        float sw_next = __ldg(swt + (u - t * nkb));
+#pragma unroll
+        for (int m = 0; m < NTOK; ++m)
+          sx_next[m] = m < p.M ? __ldg(p.sx + (int64_t)m * KB + (u - t * nkb)) : 0.0f;
         for (int v = u; v < seg_end; ++v) {
           const int kb = v - t * nkb;
+          float sxv[NTOK];
+#pragma unroll
+          for (int m = 0; m < NTOK; ++m) sxv[m] = sx_next[m];
+          const float swv = sw_next;
+          if (v + 1 < seg_end) {
+            sw_next = __ldg(swt + kb + 1);
+#pragma unroll
+            for (int m = 0; m < NTOK; ++m) sx_next[m] = m < p.M ? __ldg(p.sx + (int64_t)m * KB + kb + 1) : 0.0f;
+          }
           const uint32_t buf = jt % kSmallBufs;
           ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kSmallBufs) & 1, abort_flag));
           if (!ok) break;
@@ -267,12 +282,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[buf]);
           ++jt;
-          const float swv = __ldg(swt + kb);
 #pragma unroll
-          for (int m = 0; m < NTOK; ++m) {
-            const float sxm = m < p.M ? __ldg(p.sx + (int64_t)m * KB + kb) : 0.0f;
-            acc[m] = fmaf(__uint_as_float(r[m]), sxm * swv, acc[m]);
-          }
+          for (int m = 0; m < NTOK; ++m) acc[m] = fmaf(__uint_as_float(r[m]), sxv[m] * swv, acc[m]);
         }
       }
       // every epilogue warp leaves together if any of them gave up a wait

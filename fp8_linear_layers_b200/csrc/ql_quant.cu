@@ -8,7 +8,10 @@
 //
 // Every kernel here is HBM-bound: it reads bf16 once and writes one byte per
 // element.  Absmax reductions are warp shuffles (plus one shared-memory step
-// for a whole row); the scale is one IEEE f32 division and each code one more.
+// for a whole row); the scale is one IEEE f32 division and each code takes the
+// correctly rounded quotient (quant_chunk8).
+#include <type_traits>
+
 #include "ql_common.cuh"
 #include "ql_internal.h"
 #include "ql_tc.cuh"
@@ -40,17 +43,11 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
     int64_t c = t + (int64_t)i * kThreads;
     if (c < nchunk) {
       cache[i] = __ldg(xr + c);
-      const uint32_t w[4] = {cache[i].x, cache[i].y, cache[i].z, cache[i].w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+      a = fmaxf(a, absmax_chunk8(cache[i]));
     }
   }
-  for (int64_t c = t + (int64_t)kCache * kThreads; c < nchunk; c += kThreads) {
-    uint4 v = __ldg(xr + c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
-  }
+  for (int64_t c = t + (int64_t)kCache * kThreads; c < nchunk; c += kThreads)
+    a = fmaxf(a, absmax_chunk8(__ldg(xr + c)));
 
   __shared__ float red[kThreads / 32];
   a = warp_max(a);
@@ -66,32 +63,23 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
   float s = a / (kInt8 ? 127.0f : 448.0f);
   if (kBf16Scale) s = __uint_as_float((uint32_t)f32_to_bf16_rn(s) << 16);
   if (t == 0) s_out[row] = s;
+  const Divisor dv = make_divisor(s);
 
   uint2* qr = reinterpret_cast<uint2*>(q + row * K);
-  auto emit = [&](int64_t c, const uint4& v) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[2];
+  auto emit_all = [&](auto fast) {
+    constexpr bool kFast = decltype(fast)::value;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const float f0 = bf16_lo(w[2 * h]), f1 = bf16_hi(w[2 * h]);
-      const float f2 = bf16_lo(w[2 * h + 1]), f3 = bf16_hi(w[2 * h + 1]);
-      if (kInt8) {
-        o[h] = (uint32_t)(int8_code(f0, s) & 0xFF) | ((uint32_t)(int8_code(f1, s) & 0xFF) << 8) |
-               ((uint32_t)(int8_code(f2, s) & 0xFF) << 16) |
-               ((uint32_t)(int8_code(f3, s) & 0xFF) << 24);
-      } else {
-        o[h] = f32x2_to_e4m3x2(e4m3_quotient(f0, s), e4m3_quotient(f1, s)) |
-               (f32x2_to_e4m3x2(e4m3_quotient(f2, s), e4m3_quotient(f3, s)) << 16);
-      }
+    for (int i = 0; i < kCache; ++i) {
+      int64_t c = t + (int64_t)i * kThreads;
+      if (c < nchunk) qr[c] = quant_chunk8<kInt8, kFast>(cache[i], dv);
     }
-    qr[c] = make_uint2(o[0], o[1]);
+    for (int64_t c = t + (int64_t)kCache * kThreads; c < nchunk; c += kThreads)
+      qr[c] = quant_chunk8<kInt8, kFast>(__ldg(xr + c), dv);
   };
-#pragma unroll
-  for (int i = 0; i < kCache; ++i) {
-    int64_t c = t + (int64_t)i * kThreads;
-    if (c < nchunk) emit(c, cache[i]);
-  }
-  for (int64_t c = t + (int64_t)kCache * kThreads; c < nchunk; c += kThreads) emit(c, __ldg(xr + c));
+  if (dv.fast)
+    emit_all(std::true_type{});
+  else
+    emit_all(std::false_type{});
 }
 
 // Per-(token, 128-group) E4M3 quantization: 16 lanes per group, each lane one
@@ -108,22 +96,13 @@ __global__ void __launch_bounds__(256) quant_groups_kernel(const uint16_t* __res
   // group g covers elements [128 g, 128 g + 128) of the flattened [M, K]
   // (K is a multiple of 128, so groups never straddle tokens)
   if (live) v = __ldg(reinterpret_cast<const uint4*>(x + g * 128) + lane16);
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float a = 0.0f;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+  float a = absmax_chunk8(v);
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
   if (!live) return;
   const float s = a / 448.0f;
-  uint32_t o2[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h)
-    o2[h] = f32x2_to_e4m3x2(e4m3_quotient(bf16_lo(w[2 * h]), s), e4m3_quotient(bf16_hi(w[2 * h]), s)) |
-            (f32x2_to_e4m3x2(e4m3_quotient(bf16_lo(w[2 * h + 1]), s),
-                             e4m3_quotient(bf16_hi(w[2 * h + 1]), s))
-             << 16);
-  reinterpret_cast<uint2*>(q + g * 128)[lane16] = make_uint2(o2[0], o2[1]);
+  const Divisor dv = make_divisor(s);
+  reinterpret_cast<uint2*>(q + g * 128)[lane16] = quant_chunk8<false>(v, dv);
   if (lane16 == 0) s_out[g] = s;
 }
 
@@ -141,9 +120,7 @@ __global__ void __launch_bounds__(256) quant_wblock_kernel(const uint16_t* __res
     const int c = t + i * 256;  // 2048 chunks: 128 rows x 16 chunks
     const int64_t r = nb * 128 + (c >> 4);
     v[i] = __ldg(reinterpret_cast<const uint4*>(w + r * K + kb * 128) + (c & 15));
-    const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16_lo(u[j])), fabsf(bf16_hi(u[j]))));
+    a = fmaxf(a, absmax_chunk8(v[i]));
   }
   __shared__ float red[8];
   a = warp_max(a);
@@ -154,20 +131,20 @@ __global__ void __launch_bounds__(256) quant_wblock_kernel(const uint16_t* __res
   for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
   const float s = m / 448.0f;
   if (t == 0) s_out[nb * KB + kb] = s;
+  const Divisor dv = make_divisor(s);
+  auto emit_all = [&](auto fast) {
+    constexpr bool kFast = decltype(fast)::value;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int c = t + i * 256;
-    const int64_t r = nb * 128 + (c >> 4);
-    const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-    uint32_t o2[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-      o2[h] = f32x2_to_e4m3x2(e4m3_quotient(bf16_lo(u[2 * h]), s), e4m3_quotient(bf16_hi(u[2 * h]), s)) |
-              (f32x2_to_e4m3x2(e4m3_quotient(bf16_lo(u[2 * h + 1]), s),
-                               e4m3_quotient(bf16_hi(u[2 * h + 1]), s))
-               << 16);
-    reinterpret_cast<uint2*>(q + r * K + kb * 128)[c & 15] = make_uint2(o2[0], o2[1]);
-  }
+    for (int i = 0; i < 8; ++i) {
+      const int c = t + i * 256;
+      const int64_t r = nb * 128 + (c >> 4);
+      reinterpret_cast<uint2*>(q + r * K + kb * 128)[c & 15] = quant_chunk8<false, kFast>(v[i], dv);
+    }
+  };
+  if (dv.fast)
+    emit_all(std::true_type{});
+  else
+    emit_all(std::false_type{});
 }
 
 template <bool kInt8, bool kBf16Scale, bool kTrigger>

@@ -88,11 +88,20 @@ def test_int8_rounding_every_bf16_value(cuda):
     _check_act(ql.W8A8_INT8_ROW, _all_bf16_with_pin(127.0, 127.0))
 
 
-@pytest.mark.parametrize("pin", [448.0, 1.0, 3.0e-3])
+@pytest.mark.parametrize("pin", [448.0, 1.0, 3.0e-3, 0.7, 1.37, 5.9, 123.4, 1.1e4, 7.3e-20, 2.2e25,
+                                 3.3e29, 1.0e-35])
 def test_e4m3_rounding_every_bf16_value(cuda, pin):
     # pin 448 -> s = 1: the hardware E4M3 conversion meets the oracle's encoder on
     # every bf16 value; other pins push every value through a non-trivial quotient
+    # (scales on both sides of the kernels' reciprocal fast path, 2^-100..2^100)
     _check_act(ql.FP8_E4M3_ROW, _all_bf16_with_pin(pin, pin))
+
+
+@pytest.mark.parametrize("pin", [1.0, 0.37, 9.9, 300.5, 7.3e-20, 2.2e25, 3.3e29, 1.0e-35])
+def test_int8_quotient_every_bf16_value(cuda, pin):
+    # s = pin / 127: every bf16 x with |x| <= pin through rne(x / s), with the
+    # rounding ties and the clamp decided by the correctly rounded quotient
+    _check_act(ql.W8A8_INT8_ROW, _all_bf16_with_pin(pin, pin))
 
 
 @pytest.mark.parametrize("scheme", SCHEMES)
