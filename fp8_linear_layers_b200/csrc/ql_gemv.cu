@@ -58,11 +58,10 @@ struct GemvParams {
   const float* sw;
   uint16_t* y;
   int64_t N, K;
-  int rows_per_stage;  // R_s: whole rows per ring stage (<= 8)
+  int rows_per_stage;  // R_s: whole rows per ring stage (1, 2, 4 or 8; the kernel's kRs)
   int stage_bytes;     // R_s * K rounded up to 128
   int stages;          // ring depth
-  int q_segs;          // K segments per row carried by separate MMA columns (8 / rows)
-  int64_t seg_len;     // bytes per segment (multiple of 64, or of 128 for blocks)
+  int64_t seg_len;     // bytes per unit segment: ceil(K R_s / 8) rounded up to 128
   ql_debug dbg;
   DevStatus* status;
 };
@@ -94,25 +93,21 @@ __host__ __device__ inline GemvSmemLayout gemv_layout(int64_t K, int stage_bytes
   return L;
 }
 
-QL_DEVINL uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
+// Plain 16-byte shared-memory load: ordered after the barrier waits (which
+// clobber memory), free to be scheduled ahead of the tensor-core instructions.
+QL_DEVINL uint4 ld_s128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
 
 // D[16x8] += A[16x32] * B[32x8]; A rows 1..15 are zero here (one token).
 template <bool kInt8>
 QL_DEVINL void mma_16832(uint32_t (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
   if constexpr (kInt8) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
         "{%8, %9}, {%0, %1, %2, %3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
   } else {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
         "{%8, %9}, {%0, %1, %2, %3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
@@ -120,7 +115,7 @@ QL_DEVINL void mma_16832(uint32_t (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0
   }
 }
 
-template <ql_scheme kScheme, int Q>
+template <ql_scheme kScheme, int kRs>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams p) {
   constexpr bool kInt8 = kScheme == QL_W8A8_INT8_ROW;
   constexpr bool kBlock = kScheme == QL_FP8_E4M3_BLOCK128;
@@ -150,8 +145,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int Rs = p.rows_per_stage;
-  const int nstages = (int)((row_end - row_begin + Rs - 1) / Rs);
+  const int nstages = (int)((row_end - row_begin + kRs - 1) / kRs);
 
   if (tid == 0) {
     tc::launch_dependents();  // the next kernel's CTAs may start as SMs free up
@@ -177,8 +171,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
           *abort_flag = 1;
           break;
         }
-        const int64_t r0 = row_begin + (int64_t)i * Rs;
-        const int64_t nr = min((int64_t)Rs, row_end - r0);
+        const int64_t r0 = row_begin + (int64_t)i * kRs;
+        const int64_t nr = min((int64_t)kRs, row_end - r0);
         const uint32_t bytes = (uint32_t)(nr * K);
         mbar_arrive_expect_tx(&full[slot], bytes);
         bulk_g2s(ring + slot * p.stage_bytes, p.wq + r0 * K, bytes, &full[slot], policy);
@@ -269,117 +263,120 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       if (p.dbg.sx) p.dbg.sx[i] = sx_s[i];
   }
 
-  // 2. Work split.  A stage holds Rs (<= 8) whole rows and the MMA has 8
-  //    columns.  With Q = 8 / Rs' (Rs' = Rs rounded up to 1, 2, 4 or 8),
-  //    row r's K range is cut into Q segments of seg_len bytes: column
-  //    j = r * Q + q of B carries segment q of row r, row q of A carries
-  //    segment q of x, so D[q][j] with q == j % Q is row r's partial over
-  //    segment q (the other products are discarded).  Every column carries
-  //    real bytes whatever Rs is.  Each warp owns the same local 64-byte
-  //    windows [lw0, lw1) of every segment; the block scheme splits whole
-  //    128-byte groups so that each group's partial is scaled alone.
-  const int64_t seg = p.seg_len;  // Q (segments per row) is a template parameter
-  const int64_t NWs = seg / 64;
-  int64_t lw0, lw1;
+  // 2. Work split.  A stage holds kRs (1, 2, 4 or 8) whole rows and the
+  //    MMA's 8 columns are the stage's 8 units: unit j = (row j / kQ, segment
+  //    j % kQ), kQ = 8 / kRs, segment q covering bytes [q seg, (q+1) seg) of
+  //    its row.  Row j of A carries the x bytes that unit j meets, so D[j][j]
+  //    is unit j's partial, held by one lane, and the other products are
+  //    discarded.  A step feeds one 64-byte window of every unit; odd units
+  //    take the two windows of each pair in swapped order, so that the lanes
+  //    of one shared-memory phase (units 2p and 2p+1) read opposite halves of
+  //    the banks.  Each warp owns the same steps of every stage, so its x
+  //    fragments stay in registers for the whole kernel.  The block scheme
+  //    splits whole window pairs (128-byte groups) so that each group's
+  //    partial is scaled alone.
+  constexpr int kQ = 8 / kRs;
+  constexpr int kMaxSteps = 8;
+  const int64_t seg = p.seg_len;     // a multiple of 128
+  const int segW = (int)(seg / 64);  // windows per unit (even)
+  int st0, st1;                      // this warp's steps [st0, st1)
   if (kBlock) {
-    const int64_t GS = seg / 128;  // groups per segment
-    lw0 = 2 * ((warp * GS) / kGemvWarps);
-    lw1 = 2 * (((warp + 1) * GS) / kGemvWarps);
+    st0 = 2 * ((warp * (segW / 2)) / kGemvWarps);
+    st1 = 2 * (((warp + 1) * (segW / 2)) / kGemvWarps);
   } else {
-    lw0 = (warp * NWs) / kGemvWarps;
-    lw1 = ((warp + 1) * NWs) / kGemvWarps;
+    st0 = (warp * segW) / kGemvWarps;
+    st1 = ((warp + 1) * segW) / kGemvWarps;
   }
+  const int nsteps = st1 - st0;           // <= kMaxSteps (segW <= 64)
   const int g = lane >> 2, t = lane & 3;  // MMA fragment coordinates
-  const int rB = g / Q, qB = g % Q;       // this lane's B column: row rB, segment qB
-  const bool useful0 = g == (2 * t) % Q;      // D[g][2t] is a kept product
-  const bool useful1 = g == (2 * t + 1) % Q;  // D[g][2t+1] is a kept product
+  const int ur = g / kQ, uq = g % kQ;     // this lane's unit: row ur, segment uq
+  const int flip = g & 1;                 // odd units swap the windows of each pair
+  const int e = g & 1;                    // D[g][g] is element e of this lane's pair
+  const bool diag = t == (g >> 1);        // this lane holds D[g][g]
+  const int64_t ulen = min(seg, K - (int64_t)uq * seg);  // unit bytes inside K
+  uint4 xr[kMaxSteps];
+  uint32_t vmask = 0;  // steps whose 16 bytes of this lane lie inside the unit
+#pragma unroll
+  for (int s = 0; s < kMaxSteps; ++s) {
+    const int64_t off = (int64_t)((st0 + s) ^ flip) * 64 + t * 16;
+    const bool v = s < nsteps && off < ulen;
+    xr[s] = v ? ld_s128(qx_s + (int64_t)uq * seg + off) : make_uint4(0, 0, 0, 0);
+    vmask |= (uint32_t)v << s;
+  }
   const float sx_tok = kBlock ? 0.0f : sx_s[0];
-  const uint32_t qx_a = smem_u32(qx_s);
-  const uint32_t ring_a = smem_u32(ring);
-  // per-lane 32-bit bases and limits of the two fragments (bytes past the
-  // lane's first window that still lie inside K; <= 0 means no data)
-  const int x_lim = (g < Q) ? (int)(K - (int64_t)g * seg - t * 16) : 0;
-  const int w_lim = (int)(K - (int64_t)qB * seg - t * 16);
-  const uint32_t x_base = qx_a + (uint32_t)((int64_t)g * seg + t * 16);
-  const uint32_t w_off = (uint32_t)(rB * K + (int64_t)qB * seg + t * 16);
+  float sxr[kMaxSteps / 2];  // block scheme: x scale of each pair's 128-wide group
+  int64_t grp0 = 0;
+  if constexpr (kBlock) {
+    grp0 = ((int64_t)uq * seg + (int64_t)st0 * 64) / 128;
+#pragma unroll
+    for (int m = 0; m < kMaxSteps / 2; ++m) sxr[m] = sx_s[min(grp0 + m, KB - 1)];
+  }
+  const uint32_t w_lane = (uint32_t)(ur * K + (int64_t)uq * seg + t * 16);
 
   // 3. Stream the ring.
   for (int i = 0; i < nstages; ++i) {
     const int slot = i % nst;
-    const int64_t r0 = row_begin + (int64_t)i * Rs;
-    const int nr = (int)min((int64_t)Rs, row_end - r0);
+    const int64_t r0 = row_begin + (int64_t)i * kRs;
+    const int nr = (int)min((int64_t)kRs, row_end - r0);
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], (i / nst) & 1, abort_flag))) {
       if (lane == 0 && !*abort_flag) record_timeout(p.status, KID_GEMV, 2);
       *abort_flag = 1;
       break;
     }
-    const int wl = rB < nr ? w_lim : 0;  // zero unless this B column is a real row of the stage
-    const uint32_t w_base = ring_a + slot * p.stage_bytes + w_off;
-    float res0 = 0.0f, res1 = 0.0f;  // kept products D[g][2t], D[g][2t+1]
+    const uint8_t* wb = ring + slot * p.stage_bytes + w_lane;
+    const uint32_t vm = ur < nr ? vmask : 0u;  // a unit past the stage's rows has no data
+    float kept;                                // this lane's unit partial (diagonal lanes)
     if constexpr (!kBlock) {
-      // four independent accumulators: consecutive MMAs do not wait on each other
+      // four accumulators: consecutive MMAs do not wait on each other
+      // Always kMaxSteps steps: a step past this warp's range has zero x and
+      // W fragments and adds nothing (a uniform branch per step measured 2x
+      // slower than the spare MMAs).
       uint32_t d[4][4] = {};
-      int64_t lw = lw0;
-      for (; lw + 1 < lw1; lw += 2) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int off = (int)(lw + h) * 64;
-          const uint4 xv = off < x_lim ? lds128(x_base + off) : make_uint4(0, 0, 0, 0);
-          const uint4 wv = off < wl ? lds128(w_base + off) : make_uint4(0, 0, 0, 0);
-          mma_16832<kInt8>(d[2 * h], xv.x, xv.y, wv.x, wv.y);
-          mma_16832<kInt8>(d[2 * h + 1], xv.z, xv.w, wv.z, wv.w);
-        }
+      for (int s = 0; s < kMaxSteps; ++s) {
+        const uint4 wv = (vm >> s) & 1u ? ld_s128(wb + ((st0 + s) ^ flip) * 64) : make_uint4(0, 0, 0, 0);
+        mma_16832<kInt8>(d[2 * (s & 1)], xr[s].x, xr[s].y, wv.x, wv.y);
+        mma_16832<kInt8>(d[2 * (s & 1) + 1], xr[s].z, xr[s].w, wv.z, wv.w);
       }
-      if (lw < lw1) {
-        const int off = (int)lw * 64;
-        const uint4 xv = off < x_lim ? lds128(x_base + off) : make_uint4(0, 0, 0, 0);
-        const uint4 wv = off < wl ? lds128(w_base + off) : make_uint4(0, 0, 0, 0);
-        mma_16832<kInt8>(d[0], xv.x, xv.y, wv.x, wv.y);
-        mma_16832<kInt8>(d[1], xv.z, xv.w, wv.z, wv.w);
-      }
-      if constexpr (kInt8) {
-        // carried bit-for-bit through the float slot, summed as int32
-        res0 = __int_as_float((int)(d[0][0] + d[1][0] + d[2][0] + d[3][0]));
-        res1 = __int_as_float((int)(d[0][1] + d[1][1] + d[2][1] + d[3][1]));
-      } else {
-        res0 = (__uint_as_float(d[0][0]) + __uint_as_float(d[1][0])) +
-               (__uint_as_float(d[2][0]) + __uint_as_float(d[3][0]));
-        res1 = (__uint_as_float(d[0][1]) + __uint_as_float(d[1][1])) +
-               (__uint_as_float(d[2][1]) + __uint_as_float(d[3][1]));
-      }
+      uint32_t de[4];  // element e of each accumulator (selects: no local memory)
+#pragma unroll
+      for (int a = 0; a < 4; ++a) de[a] = e ? d[a][1] : d[a][0];
+      if constexpr (kInt8)  // carried bit-for-bit through the float slot, summed as int32
+        kept = __int_as_float((int)(de[0] + de[1] + de[2] + de[3]));
+      else
+        kept = (__uint_as_float(de[0]) + __uint_as_float(de[1])) +
+               (__uint_as_float(de[2]) + __uint_as_float(de[3]));
     } else {
-      // per 128-wide group: its own partial, scaled by s_x[group] * s_w[block, group]
-      const int64_t GS = seg / 128;
-      const int64_t rowA = r0 + (2 * t) / Q, rowB = r0 + (2 * t + 1) / Q;
-      const int64_t bA = (min(rowA, row_end - 1) >> 7) * KB - sw_first;
-      const int64_t bB = (min(rowB, row_end - 1) >> 7) * KB - sw_first;
-      for (int64_t lw = lw0; lw < lw1; lw += 2) {
-        uint32_t d[4][4] = {};  // independent chains inside the 128-wide group
+      // per 128-wide group (a window pair): its own partial, scaled by
+      // s_x[group] * s_w[row block, group]
+      const int64_t ublk = (min(r0 + ur, row_end - 1) >> 7) * KB - sw_first;
+      float res = 0.0f;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int off = (int)(lw + h) * 64;
-          const uint4 xv = off < x_lim ? lds128(x_base + off) : make_uint4(0, 0, 0, 0);
-          const uint4 wv = off < wl ? lds128(w_base + off) : make_uint4(0, 0, 0, 0);
-          mma_16832<false>(d[2 * h], xv.x, xv.y, wv.x, wv.y);
-          mma_16832<false>(d[2 * h + 1], xv.z, xv.w, wv.z, wv.w);
+      for (int m = 0; m < kMaxSteps / 2; ++m) {
+        {  // pairs past this warp's range have zero fragments and add nothing
+          uint32_t d[4][4] = {};
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int s = 2 * m + h;
+            const uint4 wv = (vm >> s) & 1u ? ld_s128(wb + ((st0 + s) ^ flip) * 64) : make_uint4(0, 0, 0, 0);
+            mma_16832<false>(d[2 * h], xr[s].x, xr[s].y, wv.x, wv.y);
+            mma_16832<false>(d[2 * h + 1], xr[s].z, xr[s].w, wv.z, wv.w);
+          }
+          uint32_t de[4];
+#pragma unroll
+          for (int a = 0; a < 4; ++a) de[a] = e ? d[a][1] : d[a][0];
+          const float pg = (__uint_as_float(de[0]) + __uint_as_float(de[1])) +
+                           (__uint_as_float(de[2]) + __uint_as_float(de[3]));
+          const int64_t si = ublk + min(grp0 + m, KB - 1);
+          const float swv = si < sw_cached ? sw_s[si] : __ldg(p.sw + sw_first + si);
+          res = fmaf(pg, sxr[m] * swv, res);
         }
-        // the kept products of this lane belong to segment g: global group g*GS + lw/2
-        const int64_t grp = min((int64_t)g * GS + (lw >> 1), KB - 1);
-        const float sxg = sx_s[grp];
-        const float swA = bA + grp < sw_cached ? sw_s[bA + grp] : __ldg(p.sw + sw_first + bA + grp);
-        const float swB = bB + grp < sw_cached ? sw_s[bB + grp] : __ldg(p.sw + sw_first + bB + grp);
-        const float pA = (__uint_as_float(d[0][0]) + __uint_as_float(d[1][0])) +
-                         (__uint_as_float(d[2][0]) + __uint_as_float(d[3][0]));
-        const float pB = (__uint_as_float(d[0][1]) + __uint_as_float(d[1][1])) +
-                         (__uint_as_float(d[2][1]) + __uint_as_float(d[3][1]));
-        res0 = fmaf(pA, sxg * swA, res0);
-        res1 = fmaf(pB, sxg * swB, res1);
       }
+      kept = res;
     }
-    // Park the kept partials (column j = r * Q + q), then count in.
+    // Park the unit partial, then count in.
     float* ps = part + slot * kGemvWarps * kGemvRows;
-    if (useful0) ps[warp * kGemvRows + 2 * t] = res0;
-    if (useful1) ps[warp * kGemvRows + 2 * t + 1] = res1;
+    if (diag) ps[warp * kGemvRows + g] = kept;
     __syncwarp();
     int before = 0;
     if (lane == 0) {
@@ -388,31 +385,43 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     }
     before = __shfl_sync(0xffffffffu, before, 0);
     if (before == kGemvWarps - 1) {
-      // last warp of this stage: every warp has read the stage and written its slot
+      // last warp of this stage: every warp has read the stage and parked its
+      // partials.  Lane (wg, u) adds warps wg and wg + 4 of unit u; the lanes
+      // then add across warp groups and across the kQ units of each row, in a
+      // fixed order.
       __threadfence_block();
-      if (lane < nr) {
-        const int64_t n = r0 + lane;
-        const int c0 = lane * Q;  // this row's columns c0 .. c0 + Q - 1
+      const int u = lane & 7, wg = lane >> 3;
+      const float p0 = ps[wg * kGemvRows + u], p1 = ps[(wg + 4) * kGemvRows + u];
+      int vi = 0;
+      float vf = 0.0f;
+      if constexpr (kInt8) {
+        vi = __float_as_int(p0) + __float_as_int(p1);
+        vi += __shfl_xor_sync(0xffffffffu, vi, 8);
+        vi += __shfl_xor_sync(0xffffffffu, vi, 16);
+#pragma unroll
+        for (int o = 1; o < kQ; o <<= 1) vi += __shfl_xor_sync(0xffffffffu, vi, o);
+      } else {
+        vf = p0 + p1;
+        vf += __shfl_xor_sync(0xffffffffu, vf, 8);
+        vf += __shfl_xor_sync(0xffffffffu, vf, 16);
+#pragma unroll
+        for (int o = 1; o < kQ; o <<= 1) vf += __shfl_xor_sync(0xffffffffu, vf, o);
+      }
+      const int r = u / kQ;
+      if (wg == 0 && u % kQ == 0 && r < nr) {
+        const int64_t n = r0 + r;
         float yv;
-        if constexpr (kInt8) {
-          int v = 0;
-          for (int w = 0; w < kGemvWarps; ++w)
-            for (int q = 0; q < Q; ++q) v += __float_as_int(ps[w * kGemvRows + c0 + q]);
-          if (p.dbg.acc_i32) p.dbg.acc_i32[n] = v;
+        if constexpr (kBlock) {
+          yv = vf;
+        } else {
           const int64_t si = n - row_begin;
           const float swn = si < sw_cached ? sw_s[si] : __ldg(p.sw + n);
-          yv = __fmul_rn(__fmul_rn(__int2float_rn(v), sx_tok), swn);
-        } else {
-          float v = 0.0f;
-          for (int w = 0; w < kGemvWarps; ++w)
-            for (int q = 0; q < Q; ++q) v += ps[w * kGemvRows + c0 + q];
-          if constexpr (kBlock) {
-            yv = v;
+          if constexpr (kInt8) {
+            if (p.dbg.acc_i32) p.dbg.acc_i32[n] = vi;
+            yv = __fmul_rn(__fmul_rn(__int2float_rn(vi), sx_tok), swn);
           } else {
-            if (p.dbg.acc_f32) p.dbg.acc_f32[n] = v;
-            const int64_t si = n - row_begin;
-            const float swn = si < sw_cached ? sw_s[si] : __ldg(p.sw + n);
-            yv = __fmul_rn(__fmul_rn(v, sx_tok), swn);
+            if (p.dbg.acc_f32) p.dbg.acc_f32[n] = vf;
+            yv = __fmul_rn(__fmul_rn(vf, sx_tok), swn);
           }
         }
         p.y[n] = f32_to_bf16_rn(yv);
@@ -428,9 +437,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 
 int gemv_max_k() { return kGemvMaxK; }
 
-template <ql_scheme S, int Q>
-static cudaError_t launch_gemv_q(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
-  cudaError_t e = ensure_smem<gemv_kernel<S, Q>>((int)smem);
+template <ql_scheme S, int kRs>
+static cudaError_t launch_gemv_r(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
+  cudaError_t e = ensure_smem<gemv_kernel<S, kRs>>((int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -442,16 +451,16 @@ static cudaError_t launch_gemv_q(const GemvParams& p, int grid, size_t smem, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<S, Q>, p);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<S, kRs>, p);
 }
 
 template <ql_scheme S>
 static cudaError_t launch_gemv_t(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
-  switch (p.q_segs) {
-    case 1: return launch_gemv_q<S, 1>(p, grid, smem, st);
-    case 2: return launch_gemv_q<S, 2>(p, grid, smem, st);
-    case 4: return launch_gemv_q<S, 4>(p, grid, smem, st);
-    case 8: return launch_gemv_q<S, 8>(p, grid, smem, st);
+  switch (p.rows_per_stage) {
+    case 1: return launch_gemv_r<S, 1>(p, grid, smem, st);
+    case 2: return launch_gemv_r<S, 2>(p, grid, smem, st);
+    case 4: return launch_gemv_r<S, 4>(p, grid, smem, st);
+    case 8: return launch_gemv_r<S, 8>(p, grid, smem, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -466,15 +475,19 @@ cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, con
   p.y = y;
   p.N = N;
   p.K = K;
-  p.rows_per_stage = (int)std::max<int64_t>(1, std::min<int64_t>(kGemvRows, kGemvStageTarget / K));
-  p.stage_bytes = (int)(((int64_t)p.rows_per_stage * K + 127) / 128 * 128);
+  // rows per stage: the largest power of two <= 8 whose stage fits the
+  // ~32 KB copy size; the 8 MMA columns are then R_s rows x 8/R_s segments
+  int rs = 1;
+  while (rs < kGemvRows && (int64_t)(2 * rs) * K <= kGemvStageTarget) rs *= 2;
+  p.rows_per_stage = rs;
+  p.stage_bytes = (int)(((int64_t)rs * K + 127) / 128 * 128);
   const int fixed = gemv_layout(K, p.stage_bytes, 0, kGemvSwCache).total;
   p.stages = (int)std::min<int64_t>(kGemvMaxStages, (kGemvSmemBudget - fixed) / p.stage_bytes);
   if (p.stages < 2) return cudaErrorInvalidConfiguration;
-  const int rq = p.rows_per_stage <= 1 ? 1 : p.rows_per_stage <= 2 ? 2 : p.rows_per_stage <= 4 ? 4 : 8;
-  p.q_segs = kGemvRows / rq;
-  const int64_t unit = scheme == QL_FP8_E4M3_BLOCK128 ? 128 : 64;
-  p.seg_len = ((K + p.q_segs - 1) / p.q_segs + unit - 1) / unit * unit;
+  const int q = kGemvRows / rs;
+  p.seg_len = ((K + q - 1) / q + 127) / 128 * 128;
+  // the kernel keeps at most 8 steps of 64-byte windows per warp: seg <= 4096
+  if (p.seg_len > 64 * 64) return cudaErrorInvalidValue;
   p.dbg = dbg ? *dbg : ql_debug{nullptr, nullptr, nullptr, nullptr};
   p.status = status;
   const int64_t stage_rows_total = (N + p.rows_per_stage - 1) / p.rows_per_stage;
