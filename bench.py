@@ -83,6 +83,11 @@ class Workload:
         M = self.products[0].M
         return "ql::gemv_kernel" if M == 1 else ("ql::gemm_small_kernel" if M <= 32 else "ql::gemm_kernel")
 
+    def bytes_touched(self, p: Product) -> float:
+        """Bytes one product reads and writes in HBM (weights, scales, x, y)."""
+        sw = 4 * (p.N // 128) * (p.K // 128) if p.scheme == FP8B else 4 * p.N
+        return p.N * p.K + sw + 2 * p.M * p.K + 2 * p.M * p.N + p.M * p.K
+
     def amount(self, p: Product) -> float:
         """Algorithmic bytes (HBM-bound regimes) or ops (tensor-bound) of one product."""
         if self.unit == "TOPS":
@@ -231,24 +236,64 @@ def nvsmi_index(torch, dev: int):
 
 
 # ------------------------------------------------------------------ GPU legs
-class Runner:
-    """Device buffers and launch closures for one workload (public API calls only)."""
+L2_BYTES = 126e6
 
-    def __init__(self, torch, ql, synthetic, wl: Workload, tokens: int = 2):
-        self.torch, self.ql, self.wl, self.tokens = torch, ql, wl, tokens
+# DRAM bytes per launch of the dominant kernel from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum), with the hash of the kernel sources it was taken on: when the
+# sources differ the figure no longer describes the kernel and the line reports null.
+KERNEL_SOURCES = {"ql::gemv_kernel": ["ql_gemv.cu", "ql_common.cuh", "ql_tc.cuh", "ql_internal.h"]}
+TRAFFIC = {
+    # workload: (bytes per launch, kernel source hash, summary file)
+    "decode": (31259502, "51b8a2aef1415563", "profiles/gemv_decode_dram.md"),
+}
+
+
+def kernel_source_hash(kernel: str):
+    import hashlib
+    files = KERNEL_SOURCES.get(kernel)
+    if not files:
+        return None
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "fp8_linear_layers_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(wl):
+    t = TRAFFIC.get(wl.key)
+    if t is None or kernel_source_hash(wl.kernel) != t[1]:
+        return None, None
+    return t[0], t[2]
+
+
+class Runner:
+    """Device buffers and launch closures for one workload (public API calls only).
+
+    Steps cycle through `copies` independent sets of quantized weights,
+    activations and outputs, enough that the bytes touched by consecutive
+    steps exceed twice the L2: no step finds its inputs in L2 from an earlier
+    one, so no flush is needed between timed steps.
+    """
+
+    def __init__(self, torch, ql, synthetic, wl: Workload):
+        self.torch, self.ql, self.wl = torch, ql, wl
+        per_step = sum(wl.bytes_touched(p) for p in wl.products)
+        self.copies = max(2, -(-int(2 * L2_BYTES) // int(per_step)))
         self.items = []
         weights = {}
         for p in wl.products:
             key = (p.name, p.N, p.K)
             if key not in weights:
                 weights[key] = synthetic.make_w_device(p.N, p.K, seed=0, tag=f"bench.{p.name}")
-            wq, sw = ql.quantize_weight(p.scheme, weights[key])
+            n_w = 1 if per_step >= 2 * L2_BYTES else self.copies
+            wqs = [ql.quantize_weight(p.scheme, weights[key]) for _ in range(n_w)]
             xs = [synthetic.make_x_device(p.M, p.K, seed=t, tag=f"bench.{p.name}.x.M{p.M}",
-                                          outliers=p.outliers) for t in range(tokens)]
-            ys = [torch.empty((p.M, p.N), dtype=torch.bfloat16, device="cuda") for _ in range(tokens)]
+                                          outliers=p.outliers) for t in range(self.copies)]
+            ys = [torch.empty((p.M, p.N), dtype=torch.bfloat16, device="cuda") for _ in range(self.copies)]
             ws_bytes = ql.forward_workspace_bytes(p.scheme, p.M, p.N, p.K)
             ws = ql.new_workspace(ws_bytes) if ws_bytes else None
-            item = dict(p=p, wq=wq, sw=sw, xs=xs, ys=ys, ws=ws, amount=wl.amount(p))
+            item = dict(p=p, wqs=wqs, xs=xs, ys=ys, ws=ws, amount=wl.amount(p))
             if p.M > 32:  # pre-quantized activations for the dominant-kernel timing
                 item["q"] = [ql.quantize_act(p.scheme, x) for x in xs]
             self.items.append(item)
@@ -257,23 +302,28 @@ class Runner:
         self.step_amount = sum(i["amount"] for i in self.items)
         self.launches_per_step = sum(1 if i["p"].M == 1 else 2 for i in self.items)
 
+    def _w(self, i, t):
+        return i["wqs"][t % len(i["wqs"])]
+
     def step(self, t):
         ql = self.ql
         for i in self.items:
-            ql.forward(i["p"].scheme, i["xs"][t], i["wq"], i["sw"], workspace=i["ws"], y=i["ys"][t])
+            wq, sw = self._w(i, t)
+            ql.forward(i["p"].scheme, i["xs"][t], wq, sw, workspace=i["ws"], y=i["ys"][t])
 
     def dominant(self, t):
         """Launches of the dominant kernel alone (the product on quantized inputs)."""
         ql = self.ql
         for i in self.items:
             p = i["p"]
+            wq, sw = self._w(i, t)
             if p.M == 1:
-                ql.gemv(p.scheme, i["xs"][t], i["wq"], i["sw"], y=i["ys"][t])
+                ql.gemv(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
             elif p.M <= 32:
-                ql.gemm_small(p.scheme, i["xs"][t], i["wq"], i["sw"], i["ws"], y=i["ys"][t])
+                ql.gemm_small(p.scheme, i["xs"][t], wq, sw, i["ws"], y=i["ys"][t])
             else:
                 qx, sx = i["q"][t]
-                ql.gemm(p.scheme, qx, sx, i["wq"], i["sw"], y=i["ys"][t])
+                ql.gemm(p.scheme, qx, sx, wq, sw, y=i["ys"][t])
 
     def capture(self, fn, stream):
         torch = self.torch
@@ -281,7 +331,7 @@ class Runner:
             fn(0)  # warms the launch path (device info, attributes) before capture
         stream.synchronize()
         graphs = []
-        for t in range(self.tokens):
+        for t in range(self.copies):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 fn(t)
@@ -306,19 +356,44 @@ class Runner:
             ox += p.M * p.K
             oy += p.M * p.N
 
-        def body():
+        def body(c):
             for i, xv, yv in views:
-                ql.forward(i["p"].scheme, xv, i["wq"], i["sw"], workspace=i["ws"], y=yv)
+                wq, sw = self._w(i, c)
+                ql.forward(i["p"].scheme, xv, wq, sw, workspace=i["ws"], y=yv)
 
         with torch.cuda.stream(stream):
-            body()
+            body(0)
         stream.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            d_x.copy_(h_x, non_blocking=True)
-            body()
-            h_y.copy_(d_y, non_blocking=True)
-        return g, 2 * xs_tot, 2 * ys_tot
+        graphs = []
+        for c in range(self.copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                d_x.copy_(h_x, non_blocking=True)
+                body(c)
+                h_y.copy_(d_y, non_blocking=True)
+            graphs.append(g)
+        return graphs, 2 * xs_tot, 2 * ys_tot
+
+
+def max_over_ranks_of(torch, dist, v: float, device) -> float:
+    """The largest of every rank's v (the job's time is its slowest rank's)."""
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, amount_per_step: float, steps: int, ms: float, scale: float) -> float:
+    """Replicas: every rank runs the same step, so the job moves world x the
+    step's amount in the max-over-ranks time."""
+    return world * amount_per_step * steps / (ms / 1e3) / scale
+
+
+def workload_config(wl):
+    return {"workload": wl.description, "key": wl.key,
+            "products": [f"{SCHEME_NAME[p.scheme]} M={p.M} {p.name} {p.N}x{p.K}" for p in wl.products],
+            "amount_per_step": sum(wl.amount(p) for p in wl.products)}
 
 
 def timed(torch, stream, graphs, steps):
@@ -405,8 +480,8 @@ def run_reference(args):
     line = base_line(wl, args, args.gpus)
     line.update({"value": value, "impl": "reference", "ms_per_step": dt / args.steps * 1e3,
                  "dtype": "s8*s8->s32 (int8), e4m3*e4m3 exact (int64 fixed point)",
-                 "config": {"workload": wl.description, "key": wl.key,
-                            "note": "CPU oracle, the plain definition"},
+                 "config": {**workload_config(wl), "parallelism": f"replicas x{args.gpus}",
+                            "note": "CPU oracle, the plain definition, on a row sample per step"},
                  "cpu_baseline": {"value": value, "unit": wl.unit, "cores": 1, "kind": "oracle",
                                   "sample": sample},
                  "e2e": {"value": value, "unit": wl.unit, "h2d_bytes_per_step": 0,
@@ -442,11 +517,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_of(torch, dist if world > 1 else None, v, "cuda")
 
     wl = workloads()[args.workload]
     scale = 1e9 if wl.unit == "GB/s" else 1e12
@@ -467,7 +538,7 @@ def main():
     barrier()
     clocks = sampler.stop()
     ms = max_over_ranks(ms_local)
-    value = world * run.step_amount * args.steps / (ms / 1e3) / scale
+    value = whole_job_value(world, run.step_amount, args.steps, ms, scale)
     status, detail = ql.device_status(stream)
     if status != 0:
         raise RuntimeError(f"device status {status} detail {detail:#x} after the timed region")
@@ -484,8 +555,10 @@ def main():
     per_launch_s = (d_ms / 1e3) / (dsteps * n_dom)
     achieved = per_launch_amount / per_launch_s / scale
     peak, peak_src = roofline_peak(wl)
+    traffic, traffic_src = measured_traffic(wl)
     roofline = {"bound": wl.bound, "achieved": round(achieved, 1), "peak": round(peak, 1),
-                "unit": wl.unit, "frac": round(achieved / peak, 4), "traffic": None,
+                "unit": wl.unit, "frac": round(achieved / peak, 4), "traffic": traffic,
+                "traffic_source": traffic_src,
                 "kernel": wl.kernel, "peak_source": peak_src,
                 "duration_source": "CUDA events over graph replays of this kernel's launches "
                                    "(inputs already quantized where the step quantizes separately)"}
@@ -495,21 +568,21 @@ def main():
     e2e_steps = args.e2e_steps or max(10, min(args.steps, 1000))
     g_e2e, h2d, d2h = run.e2e_graph(stream)
     with torch.cuda.stream(stream):
-        for _ in range(min(args.warmup, 10)):
-            g_e2e.replay()
+        for i in range(min(args.warmup, 10)):
+            g_e2e[i % len(g_e2e)].replay()
             stream.synchronize()
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for _ in range(e2e_steps):
-            g_e2e.replay()
+        for i in range(e2e_steps):
+            g_e2e[i % len(g_e2e)].replay()
             stream.synchronize()  # the host reads every step's outputs
         e1.record(stream)
     e1.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * run.step_amount * e2e_steps / (e2e_ms / 1e3) / scale
+    e2e_value = whole_job_value(world, run.step_amount, e2e_steps, e2e_ms, scale)
     del g_e2e
 
     cpu = None
@@ -526,15 +599,13 @@ def main():
         weight_bytes = sum(p.N * p.K for p in wl.products)
         line.update({
             "value": round(value, 1), "ms_per_step": ms / args.steps,
-            "config": {"workload": wl.description, "key": wl.key,
-                       "products": [f"{SCHEME_NAME[p.scheme]} M={p.M} {p.name} {p.N}x{p.K}"
-                                    for p in wl.products],
+            "config": {**workload_config(wl),
                        "launches_per_step": run.launches_per_step,
-                       "amount_per_step": run.step_amount, "parallelism": f"replicas x{world}",
-                       "l2": (f"inputs larger than L2 (126 MB): {weight_bytes / 1e6:.0f} MB of weights "
-                              "per step") if weight_bytes > 126e6 else
-                             (f"{weight_bytes / 1e6:.0f} MB of weights per step, under the 126 MB L2: "
-                              "not flushed between steps"),
+                       "parallelism": f"replicas x{world}",
+                       "l2": (f"inputs larger than L2 (126 MB): consecutive steps cycle through "
+                              f"{run.copies} sets of weights/activations/outputs, "
+                              f"{run.copies * sum(wl.bytes_touched(p) for p in wl.products) / 1e6:.0f} MB "
+                              f"touched per cycle ({weight_bytes / 1e6:.0f} MB of weights per step); no flush"),
                        "timing": "one CUDA graph replay per step, CUDA events on the launch stream"},
             "roofline": roofline,
             "cpu_baseline": cpu,
