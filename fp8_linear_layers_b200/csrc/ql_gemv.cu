@@ -21,7 +21,9 @@
 //    block scheduler then stacks two CTAs of one kernel on some SMs.)
 //  * 8 consumer warps first quantize x (fused per-token or per-128-group
 //    absmax, IEEE-divided scale, correctly rounded quotients, codes) into
-//    shared memory.
+//    shared memory.  Until they are done the producer has only two stages in
+//    flight (measured: a full ring fill from every SM at kernel start delays
+//    the quantization's own x reads and instruction fetches by microseconds).
 //  * The products run on the tensor cores with mma.sync m16n8k32 (s8 x s8 ->
 //    s32, exact; or E4M3 x E4M3 -> f32): the stage's rows are the MMA's 8
 //    columns, the token is row 0 of its 16 rows.  The k order inside each
@@ -45,6 +47,7 @@ constexpr int kGemvWarps = 8;                  // consumer warps
 constexpr int kGemvConsumers = kGemvWarps * 32;
 constexpr int kGemvThreads = kGemvConsumers + 32;
 constexpr int kGemvMaxStages = 6;
+constexpr int kEarlyStages = 2;                 // stages copied before x is quantized
 constexpr int kGemvStageTarget = 32768;
 constexpr int kGemvSmemBudget = 200 * 1024;     // one CTA per SM
 constexpr int kGemvMaxK = 32768;
@@ -85,8 +88,8 @@ __host__ __device__ inline GemvSmemLayout gemv_layout(int64_t K, int stage_bytes
   off += (sw_floats + 31) / 32 * 128;
   L.part = off;  // [stages][8 warps][8 rows] partial sums
   off += kGemvMaxStages * kGemvWarps * kGemvRows * 4;
-  L.bars = off;  // full[stages], empty[stages]
-  off += 2 * kGemvMaxStages * 8;
+  L.bars = off;  // full[stages], empty[stages], x ready
+  off += 2 * kGemvMaxStages * 8 + 8;
   L.flags = off;  // abort flag, per-stage arrival counters, block reduction scratch
   off += 16 + kGemvMaxStages * 4 + kGemvWarps * 4;
   L.total = (off + 127) / 128 * 128;
@@ -139,6 +142,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   float* part = reinterpret_cast<float*>(smem + L.part);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + kGemvMaxStages;
+  uint64_t* xready = full + 2 * kGemvMaxStages;  // consumers have quantized x
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.flags);
   int* arrivals = reinterpret_cast<int*>(smem + L.flags + 16);
   float* blockred = reinterpret_cast<float*>(smem + L.flags + 16 + kGemvMaxStages * 4);
@@ -155,6 +159,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       arrivals[s] = 0;
     }
     *abort_flag = 0;
+    mbar_init(xready, 1);
     fence_barrier_init();
   }
   __syncthreads();
@@ -166,6 +171,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       int issued = 0;
       for (int i = 0; i < nstages; ++i) {
         const int slot = i % nst;
+        // Only kEarlyStages copies go out before x is quantized: a full ring
+        // fill from every SM at once queues the consumers' x reads and
+        // instruction fetches behind ~25 MB of weight requests.
+        if (i == kEarlyStages && !mbar_wait_bounded(xready, 0, abort_flag)) {
+          if (!*abort_flag) record_timeout(p.status, KID_GEMV, 3);
+          *abort_flag = 1;
+          break;
+        }
         if (i >= nst && !mbar_wait_bounded(&empty[slot], ((i / nst) - 1) & 1, abort_flag)) {
           if (!*abort_flag) record_timeout(p.status, KID_GEMV, 1);
           *abort_flag = 1;
@@ -192,14 +205,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   for (int i = tid; i < sw_cached; i += kGemvConsumers) sw_s[i] = __ldg(p.sw + sw_first + i);
 
   tc::grid_dependency_wait();  // x may be produced by the previous kernel
-  // 1. Fused activation quantization of x [1, K] into shared memory.  Up to
-  //    kXCache 16-byte chunks per thread stay in registers between the absmax
-  //    and the rounding; longer rows re-read the rest (x sits in L2).
+  // 1. Fused activation quantization of x [1, K] into shared memory: one pass
+  //    for the absmax (the first kXLoads chunks per thread loaded together),
+  //    one for the codes (x is L2-resident by then).
   {
     const int64_t nchunk8 = K / 8;  // 16-byte chunks of 8 bf16
-    constexpr int kXCache = 8;
+    constexpr int kXLoads = 8;
     const uint4* xg = reinterpret_cast<const uint4*>(p.x);
-    uint4 xc[kXCache];
     if (kBlock) {
       // 16 consecutive chunks (lanes) form one 128-wide group: no CTA barrier
       for (int64_t base = 0; base < nchunk8; base += kGemvConsumers) {
@@ -217,12 +229,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     } else {
       float a_tok = 0.0f;
 #pragma unroll
-      for (int i = 0; i < kXCache; ++i) {
+      for (int i = 0; i < kXLoads; ++i) {
         const int64_t c = tid + (int64_t)i * kGemvConsumers;
-        xc[i] = c < nchunk8 ? __ldg(xg + c) : make_uint4(0, 0, 0, 0);
-        a_tok = fmaxf(a_tok, absmax_chunk8(xc[i]));
+        a_tok = fmaxf(a_tok, absmax_chunk8(c < nchunk8 ? __ldg(xg + c) : make_uint4(0, 0, 0, 0)));
       }
-      for (int64_t c = tid + (int64_t)kXCache * kGemvConsumers; c < nchunk8; c += kGemvConsumers)
+      for (int64_t c = tid + (int64_t)kXLoads * kGemvConsumers; c < nchunk8; c += kGemvConsumers)
         a_tok = fmaxf(a_tok, absmax_chunk8(__ldg(xg + c)));
       a_tok = warp_max(a_tok);
       if (lane == 0) blockred[warp] = a_tok;
@@ -236,14 +247,18 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       // one uniform branch: the eight values of every chunk run side by side
       auto emit_all = [&](auto fast) {
         constexpr bool kFast = decltype(fast)::value;
+        // a rolled loop re-reading x (L2-resident): the straight-line form
+        // measured slower inside a step, where its instructions are fetched
+        // while the weight stream congests L2
         uint2* q2 = reinterpret_cast<uint2*>(qx_s);
-#pragma unroll
-        for (int i = 0; i < kXCache; ++i) {
-          const int64_t c = tid + (int64_t)i * kGemvConsumers;
-          if (c < nchunk8) q2[c] = quant_chunk8<kInt8, kFast>(xc[i], dv);
+#pragma unroll 1
+        for (int64_t c = tid; c < nchunk8; c += 2 * kGemvConsumers) {
+          const int64_t c2 = c + kGemvConsumers;
+          const uint4 v0 = __ldg(xg + c);
+          const uint4 v1 = c2 < nchunk8 ? __ldg(xg + c2) : make_uint4(0, 0, 0, 0);
+          q2[c] = quant_chunk8<kInt8, kFast>(v0, dv);
+          if (c2 < nchunk8) q2[c2] = quant_chunk8<kInt8, kFast>(v1, dv);
         }
-        for (int64_t c = tid + (int64_t)kXCache * kGemvConsumers; c < nchunk8; c += kGemvConsumers)
-          q2[c] = quant_chunk8<kInt8, kFast>(__ldg(xg + c), dv);
       };
       if (dv.fast)
         emit_all(std::true_type{});
@@ -255,6 +270,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       *reinterpret_cast<uint4*>(qx_s + b) = make_uint4(0, 0, 0, 0);
     named_bar_sync(kBarConsumers, kGemvConsumers);
   }
+  if (tid == 0) mbar_arrive(xready);  // the producer may fill the whole ring now
   if (blockIdx.x == 0 && (p.dbg.qx || p.dbg.sx)) {
     for (int64_t c = tid; c < K / 16; c += kGemvConsumers)
       if (p.dbg.qx) reinterpret_cast<uint4*>(p.dbg.qx)[c] = reinterpret_cast<const uint4*>(qx_s)[c];
