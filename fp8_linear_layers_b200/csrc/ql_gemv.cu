@@ -43,7 +43,7 @@
 
 namespace ql {
 
-constexpr int kGemvWarps = 8;                  // consumer warps
+constexpr int kGemvWarps = 8;                  // consumer warps (a multiple of 4)
 constexpr int kGemvConsumers = kGemvWarps * 32;
 constexpr int kGemvThreads = kGemvConsumers + 32;
 constexpr int kGemvMaxStages = 6;
@@ -150,6 +150,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int nstages = (int)((row_end - row_begin + kRs - 1) / kRs);
+  // A ragged row count puts its partial stage first, so that it streams with
+  // the first full stages instead of adding one stage of latency at the end.
+  const int lead = (int)((row_end - row_begin) % kRs);
+  auto stage_r0 = [&](int i) -> int64_t {
+    return lead == 0 ? row_begin + (int64_t)i * kRs
+                     : (i == 0 ? row_begin : row_begin + lead + (int64_t)(i - 1) * kRs);
+  };
+  auto stage_rows = [&](int i) -> int { return (lead != 0 && i == 0) ? lead : kRs; };
 
   if (tid == 0) {
     tc::launch_dependents();  // the next kernel's CTAs may start as SMs free up
@@ -184,8 +192,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
           *abort_flag = 1;
           break;
         }
-        const int64_t r0 = row_begin + (int64_t)i * kRs;
-        const int64_t nr = min((int64_t)kRs, row_end - r0);
+        const int64_t r0 = stage_r0(i);
+        const int64_t nr = stage_rows(i);
         const uint32_t bytes = (uint32_t)(nr * K);
         mbar_arrive_expect_tx(&full[slot], bytes);
         bulk_g2s(ring + slot * p.stage_bytes, p.wq + r0 * K, bytes, &full[slot], policy);
@@ -292,7 +300,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   //    splits whole window pairs (128-byte groups) so that each group's
   //    partial is scaled alone.
   constexpr int kQ = 8 / kRs;
-  constexpr int kMaxSteps = 8;
+  constexpr int kMaxSteps = 64 / kGemvWarps;  // steps per warp (a unit has <= 64 windows)
   const int64_t seg = p.seg_len;     // a multiple of 128
   const int segW = (int)(seg / 64);  // windows per unit (even)
   int st0, st1;                      // this warp's steps [st0, st1)
@@ -332,8 +340,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   // 3. Stream the ring.
   for (int i = 0; i < nstages; ++i) {
     const int slot = i % nst;
-    const int64_t r0 = row_begin + (int64_t)i * kRs;
-    const int nr = (int)min((int64_t)kRs, row_end - r0);
+    const int64_t r0 = stage_r0(i);
+    const int nr = stage_rows(i);
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], (i / nst) & 1, abort_flag))) {
       if (lane == 0 && !*abort_flag) record_timeout(p.status, KID_GEMV, 2);
       *abort_flag = 1;
@@ -402,22 +410,26 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     before = __shfl_sync(0xffffffffu, before, 0);
     if (before == kGemvWarps - 1) {
       // last warp of this stage: every warp has read the stage and parked its
-      // partials.  Lane (wg, u) adds warps wg and wg + 4 of unit u; the lanes
-      // then add across warp groups and across the kQ units of each row, in a
-      // fixed order.
+      // partials.  Lane (wg, u) adds warps wg, wg + 4, ... of unit u; the
+      // lanes then add across warp groups and across the kQ units of each
+      // row, in a fixed order.
       __threadfence_block();
       const int u = lane & 7, wg = lane >> 3;
-      const float p0 = ps[wg * kGemvRows + u], p1 = ps[(wg + 4) * kGemvRows + u];
       int vi = 0;
       float vf = 0.0f;
+#pragma unroll
+      for (int w = wg; w < kGemvWarps; w += 4) {
+        if constexpr (kInt8)
+          vi += __float_as_int(ps[w * kGemvRows + u]);
+        else
+          vf += ps[w * kGemvRows + u];
+      }
       if constexpr (kInt8) {
-        vi = __float_as_int(p0) + __float_as_int(p1);
         vi += __shfl_xor_sync(0xffffffffu, vi, 8);
         vi += __shfl_xor_sync(0xffffffffu, vi, 16);
 #pragma unroll
         for (int o = 1; o < kQ; o <<= 1) vi += __shfl_xor_sync(0xffffffffu, vi, o);
       } else {
-        vf = p0 + p1;
         vf += __shfl_xor_sync(0xffffffffu, vf, 8);
         vf += __shfl_xor_sync(0xffffffffu, vf, 16);
 #pragma unroll
