@@ -349,11 +349,11 @@ extern "C" ql_status qlinear_gemm_small_noalloc(ql_scheme scheme, const uint16_t
   void* scratch = nullptr;
   QL_TRY(noalloc_scratch(&scratch));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // The split-tile arrival counters must start at zero; the scratch keeps
-  // whatever the previous call left, so clear them (no allocation involved).
-  const size_t counters = ql::gemm_small_counters_offset(scheme, M, N, K, d.sms);
-  cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(scratch) + counters, 0, need_ws - counters, st);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scratch counters)");
+  // The split-tile sums and arrival counters must start at zero; the scratch
+  // keeps whatever the previous call left, so clear them (no allocation).
+  const size_t zeroed = ql::gemm_small_zeroed_bytes(scheme, M, N, K, d.sms);
+  cudaError_t e = cudaMemsetAsync(scratch, 0, zeroed, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scratch sums and counters)");
   e = ql::launch_gemm_small(scheme, x, wq, sw, M, N, K, y, scratch, kNoAllocScratchBytes, nullptr,
                             d.sms, d.status, st);
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm_small_noalloc");

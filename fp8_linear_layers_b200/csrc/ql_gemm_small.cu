@@ -31,6 +31,8 @@ constexpr int kSmallThreads = 64 + kSmallEpiWarps * 32;
 constexpr int kSmallTmemCols = 128;
 constexpr int kSmallBufs = 4;  // TMEM accumulators of 32 columns
 constexpr int kSmallBufCols = 32;
+constexpr int kSmallSlots = 2;  // parked partials per split tile (more contributors: atomics)
+constexpr int kSmallEarlyStages = 2;  // weight stages issued before the tokens
 constexpr uint32_t kSmallEpiBar = 1;
 
 template <int NTOK>
@@ -52,7 +54,7 @@ struct SmallParams {
   int ntn;          // 128-row tiles of W_q
   int nkb;          // 128-byte K blocks
   int units;        // ntn * nkb
-  float* partials;  // [G][2][NTOK][128] 32-bit partial sums
+  void* accum;         // [ntn][kSmallSlots][NTOK][128] int32 or f32: parked partials, or atomic sums (zero between calls)
   unsigned* counters;  // [ntn], zero between calls
   int32_t* acc_i32;
   float* acc_f32;
@@ -134,8 +136,11 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
       const int n = u1 - u0;
-      const int pre = n < kStages ? n : kStages;
-      // weights first: they do not depend on the quantization kernel
+      // weights first: they do not depend on the quantization kernel.  Only a
+      // couple of stages go out before the quantized tokens are requested: a
+      // full ring fill from every SM would queue those (L2-resident) loads
+      // behind ~30 MB of weight reads.
+      const int pre = n < kSmallEarlyStages ? n : kSmallEarlyStages;
       for (int j = 0; j < pre; ++j) {
         const int u = u0 + j;
         mbar_arrive_expect_tx(&full[j], Cfg::kStage);
@@ -149,7 +154,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       int issued = pre;
       for (int j = pre; j < n; ++j) {
         const int s = j % kStages;
-        if (!mbar_wait_bounded(&empty[s], ((j / kStages) - 1) & 1, abort_flag)) {
+        if (j >= kStages && !mbar_wait_bounded(&empty[s], ((j / kStages) - 1) & 1, abort_flag)) {
           if (!*abort_flag) record_timeout(p.status, KID_GEMM_SMALL, 1);
           *abort_flag = 1;
           break;
@@ -294,17 +299,27 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
 
       bool do_epilogue = whole;
       if (!whole) {
-        // park this segment's partial, then let the last contributor finish the tile
+        // A tile split between two CTAs: each parks its partial in its own
+        // slot and the second to arrive adds the two in a fixed order.  A tile
+        // with more contributors (small N: up to ~20) adds into one slot with
+        // L2 atomics (int32 exact for int8; f32 for E4M3, whose order of
+        // addition then varies from call to call), and the last to arrive
+        // reads the sums and zeroes them for the next call -- summing parked
+        // partials there took one L2 round trip per contributor.
         const int c_first = unit_owner(t * nkb, p.units, G);
         const int c_last = unit_owner((t + 1) * nkb - 1, p.units, G);
-        const int my_slot = 2 * c + ((unit_begin(c, p.units, G) / nkb) == t ? 0 : 1);
-        float* slot = p.partials + (int64_t)my_slot * NTOK * 128;
+        const int ncon = c_last - c_first + 1;
+        const bool few = ncon <= kSmallSlots;
+        Acc* tacc = reinterpret_cast<Acc*>(p.accum) + (int64_t)t * kSmallSlots * NTOK * 128;
+        if (few) {
+          Acc* slot = tacc + (c - c_first) * NTOK * 128;
 #pragma unroll
-        for (int m = 0; m < NTOK; ++m) {
-          if constexpr (kInt8)
-            reinterpret_cast<int*>(slot)[m * 128 + et] = acc[m];
-          else
-            slot[m * 128 + et] = acc[m];
+          for (int m = 0; m < NTOK; ++m)
+            if (m < p.M) slot[m * 128 + et] = acc[m];
+        } else {
+#pragma unroll
+          for (int m = 0; m < NTOK; ++m)
+            if (m < p.M) atomicAdd(tacc + m * 128 + et, acc[m]);
         }
         __threadfence();
         named_bar_sync(kSmallEpiBar, kSmallEpiWarps * 32);
@@ -316,18 +331,22 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         do_epilogue = *last_flag != 0;
         if (do_epilogue) {
           __threadfence();
-#pragma unroll
-          for (int m = 0; m < NTOK; ++m) acc[m] = 0;
-          for (int cc = c_first; cc <= c_last; ++cc) {
-            const int sl = 2 * cc + ((unit_begin(cc, p.units, G) / nkb) == t ? 0 : 1);
-            const float* src = p.partials + (int64_t)sl * NTOK * 128;
+          if (few) {
 #pragma unroll
             for (int m = 0; m < NTOK; ++m) {
-              if constexpr (kInt8)
-                acc[m] += __ldcg(reinterpret_cast<const int*>(src) + m * 128 + et);
-              else
-                acc[m] += __ldcg(src + m * 128 + et);
+              Acc v = 0;
+              if (m < p.M) {
+                // fixed order: the first contributor's part, then the second's
+                v = __ldcg(tacc + m * 128 + et) + __ldcg(tacc + NTOK * 128 + m * 128 + et);
+              }
+              acc[m] = v;
             }
+          } else {
+#pragma unroll
+            for (int m = 0; m < NTOK; ++m) acc[m] = m < p.M ? __ldcg(tacc + m * 128 + et) : (Acc)0;
+#pragma unroll
+            for (int m = 0; m < NTOK; ++m)
+              if (m < p.M) tacc[m * 128 + et] = (Acc)0;  // zero again for the next call
           }
           if (et == 0) p.counters[t] = 0u;  // every contributor has arrived: reset for the next call
         }
@@ -371,20 +390,20 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
 
 namespace {
 struct SmallLayout {
-  size_t qx, sx, partials, counters, total;
+  size_t qx, sx, accum, counters, total;
 };
 
 SmallLayout small_layout(ql_scheme s, int64_t M, int64_t N, int64_t K, int sms) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
   const int ntok = M <= 16 ? 16 : 32;
-  const int64_t units = ((N + 127) / 128) * ((K + 127) / 128);
-  const int64_t G = std::min<int64_t>(units, sms);
+  (void)sms;
+  // the region that must be zero when a call starts comes first
   SmallLayout L;
-  L.qx = 0;
-  L.sx = up((size_t)(M * K));
-  L.partials = L.sx + up((size_t)M * (s == QL_FP8_E4M3_BLOCK128 ? K / 128 : 1) * 4);
-  L.counters = L.partials + up((size_t)G * 2 * ntok * 128 * 4);
-  L.total = L.counters + up((size_t)((N + 127) / 128) * 4);
+  L.counters = 0;
+  L.accum = up((size_t)((N + 127) / 128) * 4);
+  L.qx = L.accum + up((size_t)((N + 127) / 128) * kSmallSlots * ntok * 128 * 4);
+  L.sx = L.qx + up((size_t)(M * K));
+  L.total = L.sx + up((size_t)M * (s == QL_FP8_E4M3_BLOCK128 ? K / 128 : 1) * 4);
   return L;
 }
 }  // namespace
@@ -393,8 +412,8 @@ size_t gemm_small_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_
   return small_layout(scheme, M, N, K, num_sms).total;
 }
 
-size_t gemm_small_counters_offset(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms) {
-  return small_layout(scheme, M, N, K, num_sms).counters;
+size_t gemm_small_zeroed_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms) {
+  return small_layout(scheme, M, N, K, num_sms).qx;
 }
 
 template <ql_scheme S, int NTOK>
@@ -438,7 +457,7 @@ cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* w
   p.ntn = (int)((N + 127) / 128);
   p.nkb = (int)((K + 127) / 128);
   p.units = p.ntn * p.nkb;
-  p.partials = reinterpret_cast<float*>(ws + L.partials);
+  p.accum = ws + L.accum;
   p.counters = reinterpret_cast<unsigned*>(ws + L.counters);
   p.acc_i32 = dbg ? dbg->acc_i32 : nullptr;
   p.acc_f32 = dbg ? dbg->acc_f32 : nullptr;

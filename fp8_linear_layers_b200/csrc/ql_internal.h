@@ -57,7 +57,9 @@ cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const
 // Small-M (1..32) tensor-core GEMM, K split across the SMs.
 size_t gemm_small_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);
 // Byte offset of the arrival counters inside that workspace (they run to its end).
-size_t gemm_small_counters_offset(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);
+// Bytes at the start of the workspace that must be zero when a call starts
+// (split-tile arrival counters and sums); a completed call leaves them zero.
+size_t gemm_small_zeroed_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq,
                               const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
                               void* workspace, size_t ws_bytes, const ql_debug* dbg, int num_sms,

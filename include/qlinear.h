@@ -137,10 +137,14 @@ ql_status qlinear_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, cons
  * overlapped with the weight stream by programmatic dependent launch).
  *   x          device, bf16 [M,K]
  *   workspace  device, at least qlinear_workspace_bytes(scheme, M, N, K)
- *              bytes, 256-byte aligned, ZERO-FILLED before its first use; a
- *              call that completes leaves it zero-filled again (after a
- *              QL_ERR_TIMEOUT, zero it again).  Two calls in flight at the
- *              same time must not share a workspace.
+ *              bytes, 256-byte aligned, ZERO-FILLED before its first use.
+ *              Its leading part (split-tile partial sums and arrival
+ *              counters) must be zero when a call starts; a call that
+ *              completes leaves it ready for the next call of the same shape,
+ *              so one workspace serves call after call of one shape.  Zero it
+ *              again before a call of another (M, N, K) or after a
+ *              QL_ERR_TIMEOUT.  Two calls in flight at the same time
+ *              must not share a workspace.
  *   dbg        optional (NULL): q_x, s_x, acc_i32 (int8) / acc_f32 (E4M3 row) */
 ql_status qlinear_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
                              int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
@@ -197,7 +201,7 @@ const char* qlinear_last_cuda_error(void);
  * with nowhere to keep a workspace pointer between calls, or a latency-
  * critical path where cudaMalloc could stall or synchronise the device.
  *
- * The scratch (quantized tokens, per-SM partial sums, split-tile counters) is
+ * The scratch (quantized tokens, split-tile sums and counters) is
  * a fixed 8 MiB array in device global memory that the library declares at
  * file scope; every GPU that loads the library holds it until the process
  * exits.  This call allocates nothing and calls no allocating routine.
@@ -211,7 +215,7 @@ const char* qlinear_last_cuda_error(void);
  *     that device current (a one-time set-up); make that first call before
  *     any stream capture.
  *   - All calls share the one array and it keeps the previous call's
- *     contents: each call clears the counters that must start at zero (an
+ *     contents: each call clears the sums and counters that must start at zero (an
  *     asynchronous memset on `stream`).  Calls whose GPU work overlaps --
  *     on different streams, or from different threads -- race on the array
  *     and give wrong results; serialise them. */

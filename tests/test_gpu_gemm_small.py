@@ -99,14 +99,18 @@ def test_small_qwen_block_m32_full_size(cuda, name, N, K):
 
 
 def test_workspace_reused_across_calls(cuda):
-    """The split-tile counters are left at zero, so one workspace serves call
-    after call (and different shapes that fit in it)."""
-    ws = _run(ql.FP8_E4M3_ROW, 8, 1024, 4096, tag="reuse")
-    nbytes = ws.numel()
-    for _ in range(3):
-        _run(ql.FP8_E4M3_ROW, 8, 1024, 4096, tag="reuse", ws=ws)
-    need = ql.workspace_bytes(ql.W8A8_INT8_ROW, 4, 512, 2048)
-    if need <= nbytes:
+    """The split-tile sums and counters are left at zero, so one workspace
+    serves call after call of one shape; re-zeroed, it serves another shape
+    that fits in it."""
+    for scheme in (ql.FP8_E4M3_ROW, ql.W8A8_INT8_ROW):
+        ws = _run(scheme, 8, 1024, 4096, tag="reuse")
+        nbytes = ws.numel()
+        for _ in range(3):
+            _run(scheme, 8, 1024, 4096, tag="reuse", ws=ws)
+        need = ql.workspace_bytes(ql.W8A8_INT8_ROW, 4, 512, 2048)
+        assert need <= nbytes
+        ws.zero_()
+        _run(ql.W8A8_INT8_ROW, 4, 512, 2048, tag="reuse2", ws=ws)
         _run(ql.W8A8_INT8_ROW, 4, 512, 2048, tag="reuse2", ws=ws)
 
 
