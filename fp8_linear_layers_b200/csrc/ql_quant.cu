@@ -23,14 +23,19 @@ namespace ql {
 //   kBf16Scale  the scale is rounded to bf16 before use (W8A8 weight scales)
 // Each thread keeps up to kCache 16-byte chunks of the row in registers so the
 // row is read from HBM once; longer rows re-read the remainder from L2.
-//   kTrigger    let a dependent kernel launched with programmatic dependent
-//               launch start early (activations only: the dependents stream
-//               their weights before waiting, so weight writers never trigger)
+//   kTrigger    activations: the kernel is itself launched with programmatic
+//               dependent launch (its CTAs may start while the previous kernel
+//               drains; x is read only after the grid dependency wait) and lets
+//               its own dependents start early (they stream their weights
+//               before waiting; weight writers never trigger)
 template <bool kInt8, bool kBf16Scale, bool kTrigger, int kThreads, int kCache>
 __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __restrict__ x,
                                                               int64_t K, uint8_t* __restrict__ q,
                                                               float* __restrict__ s_out) {
-  if (kTrigger && threadIdx.x == 0) tc::launch_dependents();
+  if (kTrigger) {
+    if (threadIdx.x == 0) tc::launch_dependents();
+    tc::grid_dependency_wait();  // x may be produced by the previous kernel
+  }
   const int64_t row = blockIdx.x;
   const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
   const int64_t nchunk = K / 8;  // 8 bf16 per 16-byte chunk
@@ -89,6 +94,7 @@ __global__ void __launch_bounds__(256) quant_groups_kernel(const uint16_t* __res
                                                            uint8_t* __restrict__ q,
                                                            float* __restrict__ s_out) {
   if (threadIdx.x == 0) tc::launch_dependents();  // activations: dependents may start early
+  tc::grid_dependency_wait();                      // x may be produced by the previous kernel
   const int64_t g = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4);
   const int lane16 = threadIdx.x & 15;
   const bool live = g < ngroups;
@@ -147,13 +153,35 @@ __global__ void __launch_bounds__(256) quant_wblock_kernel(const uint16_t* __res
     emit_all(std::false_type{});
 }
 
+// Launch with programmatic dependent launch allowed (activation quantizers).
+template <typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(Args...), unsigned grid, unsigned block, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <bool kInt8, bool kBf16Scale, bool kTrigger>
 static cudaError_t launch_rows(const uint16_t* x, int64_t rows, int64_t K, uint8_t* q, float* s,
                                cudaStream_t st) {
-  if (K <= 8 * 8 * 256)
-    quant_rows_kernel<kInt8, kBf16Scale, kTrigger, 256, 8><<<(unsigned)rows, 256, 0, st>>>(x, K, q, s);
-  else
-    quant_rows_kernel<kInt8, kBf16Scale, kTrigger, 512, 8><<<(unsigned)rows, 512, 0, st>>>(x, K, q, s);
+  if (K <= 8 * 8 * 256) {
+    auto* k = quant_rows_kernel<kInt8, kBf16Scale, kTrigger, 256, 8>;
+    if (kTrigger) return launch_pdl(k, (unsigned)rows, 256u, st, x, K, q, s);
+    k<<<(unsigned)rows, 256, 0, st>>>(x, K, q, s);
+  } else {
+    auto* k = quant_rows_kernel<kInt8, kBf16Scale, kTrigger, 512, 8>;
+    if (kTrigger) return launch_pdl(k, (unsigned)rows, 512u, st, x, K, q, s);
+    k<<<(unsigned)rows, 512, 0, st>>>(x, K, q, s);
+  }
   return cudaGetLastError();
 }
 
@@ -171,8 +199,7 @@ cudaError_t launch_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, 
     case QL_FP8_E4M3_ROW: return launch_rows<false, false, true>(x, M, K, qx, sx, st);
     default: {
       const int64_t ngroups = M * (K / 128);
-      quant_groups_kernel<<<(unsigned)((ngroups + 15) / 16), 256, 0, st>>>(x, ngroups, qx, sx);
-      return cudaGetLastError();
+      return launch_pdl(quant_groups_kernel, (unsigned)((ngroups + 15) / 16), 256u, st, x, ngroups, qx, sx);
     }
   }
 }
