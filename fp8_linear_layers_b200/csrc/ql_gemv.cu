@@ -24,12 +24,16 @@
 //    shared memory.  Until they are done the producer has only two stages in
 //    flight (measured: a full ring fill from every SM at kernel start delays
 //    the quantization's own x reads and instruction fetches by microseconds).
-//  * The products run on the tensor cores with mma.sync m16n8k32 (s8 x s8 ->
-//    s32, exact; or E4M3 x E4M3 -> f32): the stage's rows are the MMA's 8
-//    columns, the token is row 0 of its 16 rows.  The k order inside each
-//    64-byte window is permuted identically for x and W so that every lane
-//    loads 16 contiguous bytes; a dot product does not depend on the order.
-//    Each warp owns a fixed range of 64-byte k windows of every row.
+//  * The products run on the tensor cores with mma.sync: the weights are the
+//    16-row A operand (16 units of the stage: rows x K segments) and x the
+//    8-column B operand, so that units j and j + 8 meet x segment j and every
+//    MMA keeps 16 products (512 weight bytes per s8 m16n8k32, exact; E4M3
+//    converts exactly to f16 for m16n8k16 with f32 accumulation, 256 bytes
+//    per instruction -- an E4M3 k32 MMA costs the same issue time for the same
+//    bytes).  The k order inside each 64-byte window is permuted identically
+//    for x and W so that every lane loads 16 contiguous bytes; a dot product
+//    does not depend on the order.  Each warp owns a fixed range of 64-byte
+//    k windows of every unit.
 //  * No CTA-wide barrier per stage: each warp parks its 8 row partials in a
 //    per-stage slot and counts itself in; the last warp adds the slots in a
 //    fixed order, applies the scales, writes y and releases the stage.
@@ -51,7 +55,7 @@ constexpr int kEarlyStages = 2;                 // stages copied before x is qua
 constexpr int kGemvStageTarget = 32768;
 constexpr int kGemvSmemBudget = 200 * 1024;     // one CTA per SM
 constexpr int kGemvMaxK = 32768;
-constexpr int kGemvRows = 8;                    // rows per stage at most (the MMA's N)
+constexpr int kGemvUnits = 16;                  // units per stage (the MMA's 16 A rows)
 constexpr int kGemvSwCache = 2048;              // row scales kept in shared memory
 constexpr uint32_t kBarConsumers = 1;           // named barrier of the consumer warps
 
@@ -61,7 +65,7 @@ struct GemvParams {
   const float* sw;
   uint16_t* y;
   int64_t N, K;
-  int rows_per_stage;  // R_s: whole rows per ring stage (1, 2, 4 or 8; the kernel's kRs)
+  int rows_per_stage;  // 2 kRs whole rows per ring stage (kRs = 1, 2 or 4: the kernel's template)
   int stage_bytes;     // R_s * K rounded up to 128
   int stages;          // ring depth
   int64_t seg_len;     // bytes per unit segment: ceil(K R_s / 8) rounded up to 128
@@ -87,7 +91,7 @@ __host__ __device__ inline GemvSmemLayout gemv_layout(int64_t K, int stage_bytes
   L.swc = off;
   off += (sw_floats + 31) / 32 * 128;
   L.part = off;  // [stages][8 warps][8 rows] partial sums
-  off += kGemvMaxStages * kGemvWarps * kGemvRows * 4;
+  off += kGemvMaxStages * kGemvWarps * kGemvUnits * 4;
   L.bars = off;  // full[stages], empty[stages], x ready
   off += 2 * kGemvMaxStages * 8 + 8;
   L.flags = off;  // abort flag, per-stage arrival counters, block reduction scratch
@@ -100,25 +104,38 @@ __host__ __device__ inline GemvSmemLayout gemv_layout(int64_t K, int stage_bytes
 // clobber memory), free to be scheduled ahead of the tensor-core instructions.
 QL_DEVINL uint4 ld_s128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
 
-// D[16x8] += A[16x32] * B[32x8]; A rows 1..15 are zero here (one token).
-template <bool kInt8>
-QL_DEVINL void mma_16832(uint32_t (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-  if constexpr (kInt8) {
-    asm(
-        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-        "{%8, %9}, {%0, %1, %2, %3};"
-        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
-  } else {
-    asm(
-        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-        "{%8, %9}, {%0, %1, %2, %3};"
-        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+// D[16x8] += A[16x32] * B[32x8], s8 x s8 -> s32 (exact).
+QL_DEVINL void mma_s8(uint32_t (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                      uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D[16x8] += A[16x16] * B[16x8], f16 x f16 -> f32.  E4M3 codes convert to f16
+// exactly and the products of two are exact in f32, so this computes what an
+// E4M3 MMA does with f32 accumulation, with half the tensor instructions per
+// weight byte (measured: one f16 k16 MMA costs what one E4M3 k32 MMA does).
+QL_DEVINL void mma_f16(uint32_t (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                       uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Eight f16x2 registers from 16 E4M3 codes (byte order kept).
+QL_DEVINL void e4m3x16_to_f16(const uint4& v, uint32_t (&h)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    h[2 * q] = e4m3x2_to_f16x2((uint16_t)(w[q] & 0xFFFFu));
+    h[2 * q + 1] = e4m3x2_to_f16x2((uint16_t)(w[q] >> 16));
   }
 }
 
-template <ql_scheme kScheme, int kRs>
+template <ql_scheme kScheme, int kRs, int kMaxSteps>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams p) {
   constexpr bool kInt8 = kScheme == QL_W8A8_INT8_ROW;
   constexpr bool kBlock = kScheme == QL_FP8_E4M3_BLOCK128;
@@ -149,15 +166,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int nstages = (int)((row_end - row_begin + kRs - 1) / kRs);
+  constexpr int kStageRows = 2 * kRs;  // rows per full stage
+  const int nstages = (int)((row_end - row_begin + kStageRows - 1) / kStageRows);
   // A ragged row count puts its partial stage first, so that it streams with
   // the first full stages instead of adding one stage of latency at the end.
-  const int lead = (int)((row_end - row_begin) % kRs);
+  const int lead = (int)((row_end - row_begin) % kStageRows);
   auto stage_r0 = [&](int i) -> int64_t {
-    return lead == 0 ? row_begin + (int64_t)i * kRs
-                     : (i == 0 ? row_begin : row_begin + lead + (int64_t)(i - 1) * kRs);
+    return lead == 0 ? row_begin + (int64_t)i * kStageRows
+                     : (i == 0 ? row_begin : row_begin + lead + (int64_t)(i - 1) * kStageRows);
   };
-  auto stage_rows = [&](int i) -> int { return (lead != 0 && i == 0) ? lead : kRs; };
+  auto stage_rows = [&](int i) -> int { return (lead != 0 && i == 0) ? lead : kStageRows; };
 
   if (tid == 0) {
     tc::launch_dependents();  // the next kernel's CTAs may start as SMs free up
@@ -287,20 +305,22 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       if (p.dbg.sx) p.dbg.sx[i] = sx_s[i];
   }
 
-  // 2. Work split.  A stage holds kRs (1, 2, 4 or 8) whole rows and the
-  //    MMA's 8 columns are the stage's 8 units: unit j = (row j / kQ, segment
-  //    j % kQ), kQ = 8 / kRs, segment q covering bytes [q seg, (q+1) seg) of
-  //    its row.  Row j of A carries the x bytes that unit j meets, so D[j][j]
-  //    is unit j's partial, held by one lane, and the other products are
-  //    discarded.  A step feeds one 64-byte window of every unit; odd units
-  //    take the two windows of each pair in swapped order, so that the lanes
-  //    of one shared-memory phase (units 2p and 2p+1) read opposite halves of
-  //    the banks.  Each warp owns the same steps of every stage, so its x
+  // 2. Work split.  A stage holds 2 kRs whole rows (kRs = 1, 2 or 4) cut into
+  //    16 units of the MMA's 16 A rows: unit u = (row (u / 8) kRs + (u % 8) / kQ,
+  //    segment u % kQ), kQ = 8 / kRs, segment q covering bytes [q seg,
+  //    (q+1) seg) of its row.  The weights are the A operand and the 8 B columns
+  //    carry x: column j holds the x bytes of segment j % kQ at the window the
+  //    units j and j + 8 read, so D[j][j] and D[j+8][j] are those units'
+  //    partials (held by one lane) and the other products are discarded.  A
+  //    step feeds one 64-byte window of every unit; odd units take the two
+  //    windows of each pair in swapped order, so that the lanes of one
+  //    shared-memory phase (units 2p and 2p+1) read opposite halves of the
+  //    banks.  Each warp owns the same steps of every stage, so its x
   //    fragments stay in registers for the whole kernel.  The block scheme
   //    splits whole window pairs (128-byte groups) so that each group's
-  //    partial is scaled alone.
+  //    partial is scaled alone.  E4M3 runs as f16 MMAs (exact conversion).
   constexpr int kQ = 8 / kRs;
-  constexpr int kMaxSteps = 64 / kGemvWarps;  // steps per warp (a unit has <= 64 windows)
+  // kMaxSteps: steps per warp, >= ceil(windows per unit / warps) (host-chosen)
   const int64_t seg = p.seg_len;     // a multiple of 128
   const int segW = (int)(seg / 64);  // windows per unit (even)
   int st0, st1;                      // this warp's steps [st0, st1)
@@ -311,12 +331,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     st0 = (warp * segW) / kGemvWarps;
     st1 = ((warp + 1) * segW) / kGemvWarps;
   }
-  const int nsteps = st1 - st0;           // <= kMaxSteps (segW <= 64)
+  const int nsteps = st1 - st0;           // <= kMaxSteps
   const int g = lane >> 2, t = lane & 3;  // MMA fragment coordinates
-  const int ur = g / kQ, uq = g % kQ;     // this lane's unit: row ur, segment uq
+  const int ur = g / kQ, uq = g % kQ;     // units g and g + 8: rows ur and kRs + ur, segment uq
   const int flip = g & 1;                 // odd units swap the windows of each pair
-  const int e = g & 1;                    // D[g][g] is element e of this lane's pair
-  const bool diag = t == (g >> 1);        // this lane holds D[g][g]
+  const int e = g & 1;                    // D[g][g], D[g+8][g] are elements e, 2 + e
+  const bool diag = t == (g >> 1);        // this lane holds D[g][g] and D[g+8][g]
   const int64_t ulen = min(seg, K - (int64_t)uq * seg);  // unit bytes inside K
   uint4 xr[kMaxSteps];
   uint32_t vmask = 0;  // steps whose 16 bytes of this lane lie inside the unit
@@ -327,6 +347,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     xr[s] = v ? ld_s128(qx_s + (int64_t)uq * seg + off) : make_uint4(0, 0, 0, 0);
     vmask |= (uint32_t)v << s;
   }
+  uint32_t xh[kInt8 ? 1 : kMaxSteps][8];  // E4M3 schemes: x fragments as f16
+  if constexpr (!kInt8) {
+#pragma unroll
+    for (int s = 0; s < kMaxSteps; ++s) e4m3x16_to_f16(xr[s], xh[s]);
+  }
   const float sx_tok = kBlock ? 0.0f : sx_s[0];
   float sxr[kMaxSteps / 2];  // block scheme: x scale of each pair's 128-wide group
   int64_t grp0 = 0;
@@ -336,6 +361,25 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     for (int m = 0; m < kMaxSteps / 2; ++m) sxr[m] = sx_s[min(grp0 + m, KB - 1)];
   }
   const uint32_t w_lane = (uint32_t)(ur * K + (int64_t)uq * seg + t * 16);
+  const uint32_t w_half = (uint32_t)(kRs * K);  // units g + 8: kRs rows further
+
+  // One step: the 16-byte fragments of units g and g + 8, 2 s8 MMAs or 4 f16 MMAs.
+  auto step = [&](uint32_t (&dd)[2][4], int s, const uint8_t* wb, uint32_t vm0, uint32_t vm1) {
+    const int off = ((st0 + s) ^ flip) * 64;
+    const uint4 w0 = (vm0 >> s) & 1u ? ld_s128(wb + off) : make_uint4(0, 0, 0, 0);
+    const uint4 w1 = (vm1 >> s) & 1u ? ld_s128(wb + w_half + off) : make_uint4(0, 0, 0, 0);
+    if constexpr (kInt8) {
+      mma_s8(dd[0], w0.x, w1.x, w0.y, w1.y, xr[s].x, xr[s].y);
+      mma_s8(dd[1], w0.z, w1.z, w0.w, w1.w, xr[s].z, xr[s].w);
+    } else {
+      uint32_t h0[8], h1[8];
+      e4m3x16_to_f16(w0, h0);
+      e4m3x16_to_f16(w1, h1);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        mma_f16(dd[q & 1], h0[2 * q], h1[2 * q], h0[2 * q + 1], h1[2 * q + 1], xh[s][2 * q], xh[s][2 * q + 1]);
+    }
+  };
 
   // 3. Stream the ring.
   for (int i = 0; i < nstages; ++i) {
@@ -348,59 +392,60 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       break;
     }
     const uint8_t* wb = ring + slot * p.stage_bytes + w_lane;
-    const uint32_t vm = ur < nr ? vmask : 0u;  // a unit past the stage's rows has no data
-    float kept;                                // this lane's unit partial (diagonal lanes)
+    const uint32_t vm0 = ur < nr ? vmask : 0u;        // a unit past the stage's rows has no data
+    const uint32_t vm1 = kRs + ur < nr ? vmask : 0u;
+    float kept0, kept1;                               // units g and g + 8 (diagonal lanes)
     if constexpr (!kBlock) {
-      // four accumulators: consecutive MMAs do not wait on each other
-      // Always kMaxSteps steps: a step past this warp's range has zero x and
-      // W fragments and adds nothing (a uniform branch per step measured 2x
-      // slower than the spare MMAs).
-      uint32_t d[4][4] = {};
+      // Always kMaxSteps steps: a step past this warp's range has zero x and W
+      // fragments and adds nothing (a uniform branch per step measured 2x
+      // slower than the spare MMAs).  Two accumulator pairs alternate by step.
+      uint32_t d[2][2][4] = {};
 #pragma unroll
-      for (int s = 0; s < kMaxSteps; ++s) {
-        const uint4 wv = (vm >> s) & 1u ? ld_s128(wb + ((st0 + s) ^ flip) * 64) : make_uint4(0, 0, 0, 0);
-        mma_16832<kInt8>(d[2 * (s & 1)], xr[s].x, xr[s].y, wv.x, wv.y);
-        mma_16832<kInt8>(d[2 * (s & 1) + 1], xr[s].z, xr[s].w, wv.z, wv.w);
+      for (int s = 0; s < kMaxSteps; ++s) step(d[s & 1], s, wb, vm0, vm1);
+      uint32_t k0[4], k1[4];  // elements e and 2 + e of each accumulator (selects, no local memory)
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        k0[a] = e ? d[a >> 1][a & 1][1] : d[a >> 1][a & 1][0];
+        k1[a] = e ? d[a >> 1][a & 1][3] : d[a >> 1][a & 1][2];
       }
-      uint32_t de[4];  // element e of each accumulator (selects: no local memory)
-#pragma unroll
-      for (int a = 0; a < 4; ++a) de[a] = e ? d[a][1] : d[a][0];
-      if constexpr (kInt8)  // carried bit-for-bit through the float slot, summed as int32
-        kept = __int_as_float((int)(de[0] + de[1] + de[2] + de[3]));
-      else
-        kept = (__uint_as_float(de[0]) + __uint_as_float(de[1])) +
-               (__uint_as_float(de[2]) + __uint_as_float(de[3]));
+      if constexpr (kInt8) {  // carried bit-for-bit through the float slot, summed as int32
+        kept0 = __int_as_float((int)(k0[0] + k0[1] + k0[2] + k0[3]));
+        kept1 = __int_as_float((int)(k1[0] + k1[1] + k1[2] + k1[3]));
+      } else {
+        kept0 = (__uint_as_float(k0[0]) + __uint_as_float(k0[1])) +
+                (__uint_as_float(k0[2]) + __uint_as_float(k0[3]));
+        kept1 = (__uint_as_float(k1[0]) + __uint_as_float(k1[1])) +
+                (__uint_as_float(k1[2]) + __uint_as_float(k1[3]));
+      }
     } else {
-      // per 128-wide group (a window pair): its own partial, scaled by
-      // s_x[group] * s_w[row block, group]
-      const int64_t ublk = (min(r0 + ur, row_end - 1) >> 7) * KB - sw_first;
-      float res = 0.0f;
+      // per 128-wide group (a window pair): its own partials, scaled by
+      // s_x[group] * s_w[row block, group] for each of the two units
+      const int64_t blk0 = (min(r0 + ur, row_end - 1) >> 7) * KB - sw_first;
+      const int64_t blk1 = (min(r0 + kRs + ur, row_end - 1) >> 7) * KB - sw_first;
+      float res0 = 0.0f, res1 = 0.0f;
 #pragma unroll
       for (int m = 0; m < kMaxSteps / 2; ++m) {
-        {  // pairs past this warp's range have zero fragments and add nothing
-          uint32_t d[4][4] = {};
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int s = 2 * m + h;
-            const uint4 wv = (vm >> s) & 1u ? ld_s128(wb + ((st0 + s) ^ flip) * 64) : make_uint4(0, 0, 0, 0);
-            mma_16832<false>(d[2 * h], xr[s].x, xr[s].y, wv.x, wv.y);
-            mma_16832<false>(d[2 * h + 1], xr[s].z, xr[s].w, wv.z, wv.w);
-          }
-          uint32_t de[4];
-#pragma unroll
-          for (int a = 0; a < 4; ++a) de[a] = e ? d[a][1] : d[a][0];
-          const float pg = (__uint_as_float(de[0]) + __uint_as_float(de[1])) +
-                           (__uint_as_float(de[2]) + __uint_as_float(de[3]));
-          const int64_t si = ublk + min(grp0 + m, KB - 1);
-          const float swv = si < sw_cached ? sw_s[si] : __ldg(p.sw + sw_first + si);
-          res = fmaf(pg, sxr[m] * swv, res);
-        }
+        // pairs past this warp's range have zero fragments and add nothing
+        uint32_t d[2][4] = {};
+        step(d, 2 * m, wb, vm0, vm1);
+        step(d, 2 * m + 1, wb, vm0, vm1);
+        const float p0 = __uint_as_float(e ? d[0][1] : d[0][0]) + __uint_as_float(e ? d[1][1] : d[1][0]);
+        const float p1 = __uint_as_float(e ? d[0][3] : d[0][2]) + __uint_as_float(e ? d[1][3] : d[1][2]);
+        const int64_t grp = min(grp0 + m, KB - 1);
+        const float sw0 = blk0 + grp < sw_cached ? sw_s[blk0 + grp] : __ldg(p.sw + sw_first + blk0 + grp);
+        const float sw1 = blk1 + grp < sw_cached ? sw_s[blk1 + grp] : __ldg(p.sw + sw_first + blk1 + grp);
+        res0 = fmaf(p0, sxr[m] * sw0, res0);
+        res1 = fmaf(p1, sxr[m] * sw1, res1);
       }
-      kept = res;
+      kept0 = res0;
+      kept1 = res1;
     }
-    // Park the unit partial, then count in.
-    float* ps = part + slot * kGemvWarps * kGemvRows;
-    if (diag) ps[warp * kGemvRows + g] = kept;
+    // Park the unit partials, then count in.
+    float* ps = part + slot * kGemvWarps * kGemvUnits;
+    if (diag) {
+      ps[warp * kGemvUnits + g] = kept0;
+      ps[warp * kGemvUnits + 8 + g] = kept1;
+    }
     __syncwarp();
     int before = 0;
     if (lane == 0) {
@@ -410,32 +455,30 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     before = __shfl_sync(0xffffffffu, before, 0);
     if (before == kGemvWarps - 1) {
       // last warp of this stage: every warp has read the stage and parked its
-      // partials.  Lane (wg, u) adds warps wg, wg + 4, ... of unit u; the
-      // lanes then add across warp groups and across the kQ units of each
+      // partials.  Lane (wg, u) adds warps wg, wg + 2, ... of unit u; the lanes
+      // then add across the two warp groups and across the kQ units of each
       // row, in a fixed order.
       __threadfence_block();
-      const int u = lane & 7, wg = lane >> 3;
+      const int u = lane & 15, wg = lane >> 4;
       int vi = 0;
       float vf = 0.0f;
 #pragma unroll
-      for (int w = wg; w < kGemvWarps; w += 4) {
+      for (int w = wg; w < kGemvWarps; w += 2) {
         if constexpr (kInt8)
-          vi += __float_as_int(ps[w * kGemvRows + u]);
+          vi += __float_as_int(ps[w * kGemvUnits + u]);
         else
-          vf += ps[w * kGemvRows + u];
+          vf += ps[w * kGemvUnits + u];
       }
       if constexpr (kInt8) {
-        vi += __shfl_xor_sync(0xffffffffu, vi, 8);
         vi += __shfl_xor_sync(0xffffffffu, vi, 16);
 #pragma unroll
         for (int o = 1; o < kQ; o <<= 1) vi += __shfl_xor_sync(0xffffffffu, vi, o);
       } else {
-        vf += __shfl_xor_sync(0xffffffffu, vf, 8);
         vf += __shfl_xor_sync(0xffffffffu, vf, 16);
 #pragma unroll
         for (int o = 1; o < kQ; o <<= 1) vf += __shfl_xor_sync(0xffffffffu, vf, o);
       }
-      const int r = u / kQ;
+      const int r = (u >> 3) * kRs + (u & 7) / kQ;
       if (wg == 0 && u % kQ == 0 && r < nr) {
         const int64_t n = r0 + r;
         float yv;
@@ -465,9 +508,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 
 int gemv_max_k() { return kGemvMaxK; }
 
-template <ql_scheme S, int kRs>
+template <ql_scheme S, int kRs, int kSteps>
 static cudaError_t launch_gemv_r(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
-  cudaError_t e = ensure_smem<gemv_kernel<S, kRs>>((int)smem);
+  cudaError_t e = ensure_smem<gemv_kernel<S, kRs, kSteps>>((int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -479,16 +522,18 @@ static cudaError_t launch_gemv_r(const GemvParams& p, int grid, size_t smem, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<S, kRs>, p);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<S, kRs, kSteps>, p);
 }
 
+// Steps per warp: 4 when a unit has at most 32 windows of 64 bytes, else 8.
 template <ql_scheme S>
 static cudaError_t launch_gemv_t(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
-  switch (p.rows_per_stage) {
-    case 1: return launch_gemv_r<S, 1>(p, grid, smem, st);
-    case 2: return launch_gemv_r<S, 2>(p, grid, smem, st);
-    case 4: return launch_gemv_r<S, 4>(p, grid, smem, st);
-    case 8: return launch_gemv_r<S, 8>(p, grid, smem, st);
+  const bool long_units = p.seg_len > 32 * 64;
+  switch (p.rows_per_stage / 2) {
+    case 1:
+      return long_units ? launch_gemv_r<S, 1, 8>(p, grid, smem, st) : launch_gemv_r<S, 1, 4>(p, grid, smem, st);
+    case 2: return launch_gemv_r<S, 2, 4>(p, grid, smem, st);
+    case 4: return launch_gemv_r<S, 4, 4>(p, grid, smem, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -503,19 +548,20 @@ cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, con
   p.y = y;
   p.N = N;
   p.K = K;
-  // rows per stage: the largest power of two <= 8 whose stage fits the
-  // ~32 KB copy size; the 8 MMA columns are then R_s rows x 8/R_s segments
+  // kRs: the largest power of two <= 4 whose stage of 2 kRs rows fits the
+  // ~32 KB copy size (kRs = 1 above 16 KB rows: stages of two rows); the 16
+  // MMA rows are then 2 kRs rows x 8 / kRs segments
   int rs = 1;
-  while (rs < kGemvRows && (int64_t)(2 * rs) * K <= kGemvStageTarget) rs *= 2;
-  p.rows_per_stage = rs;
-  p.stage_bytes = (int)(((int64_t)rs * K + 127) / 128 * 128);
+  while (rs < 4 && (int64_t)(4 * rs) * K <= kGemvStageTarget) rs *= 2;
+  p.rows_per_stage = 2 * rs;
+  p.stage_bytes = (int)(((int64_t)p.rows_per_stage * K + 127) / 128 * 128);
   const int fixed = gemv_layout(K, p.stage_bytes, 0, kGemvSwCache).total;
   p.stages = (int)std::min<int64_t>(kGemvMaxStages, (kGemvSmemBudget - fixed) / p.stage_bytes);
   if (p.stages < 2) return cudaErrorInvalidConfiguration;
-  const int q = kGemvRows / rs;
+  const int q = 8 / rs;
   p.seg_len = ((K + q - 1) / q + 127) / 128 * 128;
-  // the kernel keeps at most 8 steps of 64-byte windows per warp: seg <= 4096
-  if (p.seg_len > 64 * 64) return cudaErrorInvalidValue;
+  // the kernel keeps at most 64 (kRs = 1) or 32 windows of 64 bytes per unit
+  if (p.seg_len > (rs == 1 ? 64 : 32) * 64) return cudaErrorInvalidValue;
   p.dbg = dbg ? *dbg : ql_debug{nullptr, nullptr, nullptr, nullptr};
   p.status = status;
   const int64_t stage_rows_total = (N + p.rows_per_stage - 1) / p.rows_per_stage;
