@@ -162,7 +162,7 @@ ql_status qlinear_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, cons
   QL_TRY(check_debug(dbg));
   DeviceInfo d;
   QL_TRY(current_device(&d));
-  cudaError_t e = ql::launch_gemv(scheme, x, wq, sw, N, K, y, dbg, d.sms, d.status,
+  cudaError_t e = ql::launch_gemv(scheme, x, wq, sw, 1, N, K, y, dbg, d.sms, d.status,
                                   static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemv");
 }

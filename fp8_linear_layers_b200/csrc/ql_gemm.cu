@@ -1,9 +1,9 @@
 // ql_gemm.cu -- large-M product on pre-quantized activations, tcgen05 + TMA.
 //
-// "Llama 3.1 8B Instruct W8A8", "Loading": longer inputs are rounded to int8 a
-// row at a time and multiplied in int8, summing in int32.  "Qwen3 8B FP8",
-// "Loading": longer inputs rounded to FP8 128 inputs at a time and multiplied
-// with block scales.  Here:
+// "Llama 3.1 8B Instruct W8A8", "Loading": larger batches quantize the
+// activations to int8 per token and accumulate the int8 products in int32.
+// "Qwen3 8B FP8", "Loading": larger batches quantize them to E4M3 in groups of
+// 128 along K and apply the block scales.  Here:
 //   acc[m,n] = sum_k q_x[m,k] q_w[n,k]       tcgen05.mma kind::i8  -> s32 TMEM
 //                                            tcgen05.mma kind::f8f6f4 (E4M3) -> f32 TMEM
 //   y[m,n]   = bf16(((f32)acc * s_x[m]) * s_w[n])                (row schemes)

@@ -1,6 +1,7 @@
 // ql_gemm_small.cu -- 1 <= M <= 32 tokens on the tensor cores (tcgen05).
 //
-// "Llama 3.1 8B Instruct W8A8", "Loading": "up to 32 rows on tensor cores";
+// "Llama 3.1 8B Instruct W8A8", "Loading": batches of at most 32 tokens run on
+// the tensor cores;
 // "Qwen3 8B FP8", "Loading": the same for the FP8 block scheme.  With at most
 // 32 tokens the product is still bound by the weight stream (<= 64 ops per
 // weight byte), so the design spreads W_q evenly over every SM:
@@ -441,6 +442,11 @@ cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* w
                               DevStatus* status, cudaStream_t st) {
   const SmallLayout L = small_layout(scheme, M, N, K, num_sms);
   if (ws_bytes < L.total) return cudaErrorInvalidValue;
+  // Up to four tokens: the GEMV kernel carries them on its MMA's B columns
+  // with the activation quantization fused, at the weight traffic of one
+  // token and without the split-K reduction (the workspace is not used).
+  if (K <= gemv_max_k_tokens(M))
+    return launch_gemv(scheme, x, wq, sw, M, N, K, y, dbg, num_sms, status, st);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint8_t* qx = ws + L.qx;
   float* sx = reinterpret_cast<float*>(ws + L.sx);

@@ -1,7 +1,7 @@
 // ql_gemv.cu -- M = 1 decode product y = (s_x s_w) . (Q(x) . W_q^T), one kernel.
 //
-// "Llama 3.1 8B Instruct W8A8", "Loading": a single token runs "one row in a
-// kernel that reads each byte once"; "Qwen3 8B FP8", "Loading": the same for
+// "Llama 3.1 8B Instruct W8A8", "Loading": a single token runs in a kernel
+// that touches every weight byte once; "Qwen3 8B FP8", "Loading": the same for
 // the FP8 block scheme.  The kernel is bound by the weight stream: N*K bytes
 // from HBM, everything else is L2/shared-memory traffic.
 //
@@ -55,6 +55,8 @@ constexpr int kEarlyStages = 2;                 // stages copied before x is qua
 constexpr int kGemvStageTarget = 32768;
 constexpr int kGemvSmemBudget = 200 * 1024;     // one CTA per SM
 constexpr int kGemvMaxK = 32768;
+constexpr int64_t kGemvMaxK2 = 16384;           // two tokens: units of at most 64 windows
+constexpr int64_t kGemvMaxK4 = 8192;            // three or four tokens: stages of 8 rows
 constexpr int kGemvUnits = 16;                  // units per stage (the MMA's 16 A rows)
 constexpr int kGemvSwCache = 2048;              // row scales kept in shared memory
 constexpr uint32_t kBarConsumers = 1;           // named barrier of the consumer warps
@@ -65,6 +67,7 @@ struct GemvParams {
   const float* sw;
   uint16_t* y;
   int64_t N, K;
+  int M;               // tokens: 1 to 4 (extra tokens ride on the MMA's B columns)
   int rows_per_stage;  // 2 kRs whole rows per ring stage (kRs = 1, 2 or 4: the kernel's template)
   int stage_bytes;     // R_s * K rounded up to 128
   int stages;          // ring depth
@@ -79,19 +82,19 @@ struct GemvSmemLayout {
 
 // Shared-memory carve-up; `sw_floats` is the number of weight scales cached.
 __host__ __device__ inline GemvSmemLayout gemv_layout(int64_t K, int stage_bytes, int stages,
-                                                      int sw_floats) {
+                                                      int sw_floats, int M = 1) {
   GemvSmemLayout L;
   int off = 0;
   L.ring = off;
   off += stages * stage_bytes;
-  L.qx = off;  // K codes, padded to whole 64-byte windows
-  off += (int)((K + 127) / 128) * 128;
+  L.qx = off;  // M rows of K codes, each padded to whole 128-byte blocks
+  off += M * (int)((K + 127) / 128) * 128;
   L.sx = off;
-  off += (int)((K / 128 + 1 + 31) / 32) * 128;
+  off += (int)((M * (K / 128 + 1) + 31) / 32) * 128;
   L.swc = off;
   off += (sw_floats + 31) / 32 * 128;
   L.part = off;  // [stages][8 warps][8 rows] partial sums
-  off += kGemvMaxStages * kGemvWarps * kGemvUnits * 4;
+  off += kGemvMaxStages * kGemvWarps * kGemvUnits * M * 4;
   L.bars = off;  // full[stages], empty[stages], x ready
   off += 2 * kGemvMaxStages * 8 + 8;
   L.flags = off;  // abort flag, per-stage arrival counters, block reduction scratch
@@ -135,8 +138,10 @@ QL_DEVINL void e4m3x16_to_f16(const uint4& v, uint32_t (&h)[8]) {
   }
 }
 
-template <ql_scheme kScheme, int kRs, int kMaxSteps>
+template <ql_scheme kScheme, int kRs, int kMaxSteps, int kM>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams p) {
+  // kM tokens x kQ = 8 / kRs segment classes must fit the 8 B columns
+  static_assert(kM == 1 || (kM * (8 / kRs) <= 8 && kRs >= 2), "tokens do not fit the B columns");
   constexpr bool kInt8 = kScheme == QL_W8A8_INT8_ROW;
   constexpr bool kBlock = kScheme == QL_FP8_E4M3_BLOCK128;
 
@@ -151,7 +156,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   const int64_t sw_count = kBlock ? (((row_end - 1) >> 7) - (row_begin >> 7) + 1) * KB : row_end - row_begin;
   const int sw_cached = (int)min(sw_count, (int64_t)kGemvSwCache);
   const int nst = p.stages;
-  const GemvSmemLayout L = gemv_layout(K, p.stage_bytes, nst, kGemvSwCache);
+  const GemvSmemLayout L = gemv_layout(K, p.stage_bytes, nst, kGemvSwCache, kM);
+  const int64_t xstride = (K + 127) / 128 * 128;  // bytes between the tokens' codes
   uint8_t* ring = smem + L.ring;
   uint8_t* qx_s = smem + L.qx;
   float* sx_s = reinterpret_cast<float*>(smem + L.sx);
@@ -234,10 +240,21 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   // 1. Fused activation quantization of x [1, K] into shared memory: one pass
   //    for the absmax (the first kXLoads chunks per thread loaded together),
   //    one for the codes (x is L2-resident by then).
-  {
+  for (int tok = 0; tok < kM; ++tok) {
     const int64_t nchunk8 = K / 8;  // 16-byte chunks of 8 bf16
     constexpr int kXLoads = 8;
-    const uint4* xg = reinterpret_cast<const uint4*>(p.x);
+    const uint4* xg = reinterpret_cast<const uint4*>(p.x + tok * K);
+    uint8_t* qx_t = qx_s + tok * xstride;
+    float* sx_t = sx_s + tok * (kBlock ? KB : 1);
+    if (tok >= p.M) {
+      // a padding token (three tokens on the four-token kernel): zero codes
+      // and scales, so its products are zero; its outputs are not written
+      for (int64_t b = tid * 16; b < xstride; b += kGemvConsumers * 16)
+        *reinterpret_cast<uint4*>(qx_t + b) = make_uint4(0, 0, 0, 0);
+      for (int i = tid; i < (kBlock ? (int)KB : 1); i += kGemvConsumers) sx_t[i] = 0.0f;
+      named_bar_sync(kBarConsumers, kGemvConsumers);
+      continue;
+    }
     if (kBlock) {
       // 16 consecutive chunks (lanes) form one 128-wide group: no CTA barrier
       for (int64_t base = 0; base < nchunk8; base += kGemvConsumers) {
@@ -248,8 +265,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
         const float s = a / 448.0f;
         if (c < nchunk8) {
-          if ((lane & 15) == 0) sx_s[c >> 4] = s;
-          reinterpret_cast<uint2*>(qx_s)[c] = quant_chunk8<false>(v, make_divisor(s));
+          if ((lane & 15) == 0) sx_t[c >> 4] = s;
+          reinterpret_cast<uint2*>(qx_t)[c] = quant_chunk8<false>(v, make_divisor(s));
         }
       }
     } else {
@@ -268,7 +285,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 #pragma unroll
       for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, blockred[w]);
       const float s = a / (kInt8 ? 127.0f : 448.0f);
-      if (tid == 0) sx_s[0] = s;
+      if (tid == 0) sx_t[0] = s;
       const Divisor dv = make_divisor(s);
       // one uniform branch: the eight values of every chunk run side by side
       auto emit_all = [&](auto fast) {
@@ -276,7 +293,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         // a rolled loop re-reading x (L2-resident): the straight-line form
         // measured slower inside a step, where its instructions are fetched
         // while the weight stream congests L2
-        uint2* q2 = reinterpret_cast<uint2*>(qx_s);
+        uint2* q2 = reinterpret_cast<uint2*>(qx_t);
 #pragma unroll 1
         for (int64_t c = tid; c < nchunk8; c += 2 * kGemvConsumers) {
           const int64_t c2 = c + kGemvConsumers;
@@ -293,16 +310,20 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     }
     // zero the padding of the last 64-byte window so it adds nothing
     for (int64_t b = K + tid * 16; b < (K + 63) / 64 * 64; b += kGemvConsumers * 16)
-      *reinterpret_cast<uint4*>(qx_s + b) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(qx_t + b) = make_uint4(0, 0, 0, 0);
     named_bar_sync(kBarConsumers, kGemvConsumers);
   }
   if (tid == 0) mbar_arrive(xready);  // the producer may fill the whole ring now
   if (blockIdx.x == 0 && (p.dbg.qx || p.dbg.sx)) {
-    for (int64_t c = tid; c < K / 16; c += kGemvConsumers)
-      if (p.dbg.qx) reinterpret_cast<uint4*>(p.dbg.qx)[c] = reinterpret_cast<const uint4*>(qx_s)[c];
-    const int ns = kBlock ? (int)KB : 1;
-    for (int i = tid; i < ns; i += kGemvConsumers)
-      if (p.dbg.sx) p.dbg.sx[i] = sx_s[i];
+    for (int tok = 0; tok < p.M; ++tok) {
+      for (int64_t c = tid; c < K / 16; c += kGemvConsumers)
+        if (p.dbg.qx)
+          reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.dbg.qx) + tok * K)[c] =
+              reinterpret_cast<const uint4*>(qx_s + tok * xstride)[c];
+      const int ns = kBlock ? (int)KB : 1;
+      for (int i = tid; i < ns; i += kGemvConsumers)
+        if (p.dbg.sx) p.dbg.sx[tok * ns + i] = sx_s[tok * ns + i];
+    }
   }
 
   // 2. Work split.  A stage holds 2 kRs whole rows (kRs = 1, 2 or 4) cut into
@@ -336,7 +357,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   const int ur = g / kQ, uq = g % kQ;     // units g and g + 8: rows ur and kRs + ur, segment uq
   const int flip = g & 1;                 // odd units swap the windows of each pair
   const int e = g & 1;                    // D[g][g], D[g+8][g] are elements e, 2 + e
-  const bool diag = t == (g >> 1);        // this lane holds D[g][g] and D[g+8][g]
+  // The lane's B column g carries token xtok.  One token: every column holds
+  // x of segment class g % kQ, and the lane keeps D[g][g], D[g+8][g] when it
+  // holds column g (t = g / 2).  kM tokens: column kQ tok + c holds token tok,
+  // class c (columns past kM kQ repeat the last token and are discarded), and
+  // the products of units g, g + 8 with token tok sit in column kQ tok + uq,
+  // held by lane t = (kQ tok + uq) / 2 as element uq % 2 = e (kQ is even).
+  const int c0 = 2 * t + e;  // the column whose products this lane may keep
+  const int xtok = kM == 1 ? 0 : min(g / kQ, kM - 1);
+  const bool diag = kM == 1 ? t == (g >> 1) : (c0 % kQ == uq && c0 / kQ < kM);
+  const int ktok = kM == 1 ? 0 : min(c0 / kQ, kM - 1);  // token of the kept products
   const int64_t ulen = min(seg, K - (int64_t)uq * seg);  // unit bytes inside K
   uint4 xr[kMaxSteps];
   uint32_t vmask = 0;  // steps whose 16 bytes of this lane lie inside the unit
@@ -344,7 +374,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   for (int s = 0; s < kMaxSteps; ++s) {
     const int64_t off = (int64_t)((st0 + s) ^ flip) * 64 + t * 16;
     const bool v = s < nsteps && off < ulen;
-    xr[s] = v ? ld_s128(qx_s + (int64_t)uq * seg + off) : make_uint4(0, 0, 0, 0);
+    xr[s] = v ? ld_s128(qx_s + xtok * xstride + (int64_t)uq * seg + off) : make_uint4(0, 0, 0, 0);
     vmask |= (uint32_t)v << s;
   }
   uint32_t xh[kInt8 ? 1 : kMaxSteps][8];  // E4M3 schemes: x fragments as f16
@@ -352,13 +382,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 #pragma unroll
     for (int s = 0; s < kMaxSteps; ++s) e4m3x16_to_f16(xr[s], xh[s]);
   }
-  const float sx_tok = kBlock ? 0.0f : sx_s[0];
   float sxr[kMaxSteps / 2];  // block scheme: x scale of each pair's 128-wide group
   int64_t grp0 = 0;
   if constexpr (kBlock) {
     grp0 = ((int64_t)uq * seg + (int64_t)st0 * 64) / 128;
 #pragma unroll
-    for (int m = 0; m < kMaxSteps / 2; ++m) sxr[m] = sx_s[min(grp0 + m, KB - 1)];
+    for (int m = 0; m < kMaxSteps / 2; ++m) sxr[m] = sx_s[ktok * KB + min(grp0 + m, KB - 1)];
   }
   const uint32_t w_lane = (uint32_t)(ur * K + (int64_t)uq * seg + t * 16);
   const uint32_t w_half = (uint32_t)(kRs * K);  // units g + 8: kRs rows further
@@ -441,10 +470,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       kept1 = res1;
     }
     // Park the unit partials, then count in.
-    float* ps = part + slot * kGemvWarps * kGemvUnits;
+    float* ps = part + slot * kM * kGemvWarps * kGemvUnits;  // [token][warp][unit]
     if (diag) {
-      ps[warp * kGemvUnits + g] = kept0;
-      ps[warp * kGemvUnits + 8 + g] = kept1;
+      ps[(ktok * kGemvWarps + warp) * kGemvUnits + g] = kept0;
+      ps[(ktok * kGemvWarps + warp) * kGemvUnits + 8 + g] = kept1;
     }
     __syncwarp();
     int before = 0;
@@ -455,47 +484,56 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     before = __shfl_sync(0xffffffffu, before, 0);
     if (before == kGemvWarps - 1) {
       // last warp of this stage: every warp has read the stage and parked its
-      // partials.  Lane (wg, u) adds warps wg, wg + 2, ... of unit u; the lanes
-      // then add across the two warp groups and across the kQ units of each
-      // row, in a fixed order.
+      // partials.
       __threadfence_block();
+      // One token: lane (wg, u) adds warps wg, wg + 2, ... of unit u and the
+      // two warp groups are then added.  kM tokens: lane (wg, u) adds all
+      // warps of unit u for tokens wg, wg + 2, ...  Then across the kQ units
+      // of each row; every order is fixed.
       const int u = lane & 15, wg = lane >> 4;
-      int vi = 0;
-      float vf = 0.0f;
-#pragma unroll
-      for (int w = wg; w < kGemvWarps; w += 2) {
-        if constexpr (kInt8)
-          vi += __float_as_int(ps[w * kGemvUnits + u]);
-        else
-          vf += ps[w * kGemvUnits + u];
-      }
-      if constexpr (kInt8) {
-        vi += __shfl_xor_sync(0xffffffffu, vi, 16);
-#pragma unroll
-        for (int o = 1; o < kQ; o <<= 1) vi += __shfl_xor_sync(0xffffffffu, vi, o);
-      } else {
-        vf += __shfl_xor_sync(0xffffffffu, vf, 16);
-#pragma unroll
-        for (int o = 1; o < kQ; o <<= 1) vf += __shfl_xor_sync(0xffffffffu, vf, o);
-      }
       const int r = (u >> 3) * kRs + (u & 7) / kQ;
-      if (wg == 0 && u % kQ == 0 && r < nr) {
-        const int64_t n = r0 + r;
-        float yv;
-        if constexpr (kBlock) {
-          yv = vf;
-        } else {
-          const int64_t si = n - row_begin;
-          const float swn = si < sw_cached ? sw_s[si] : __ldg(p.sw + n);
-          if constexpr (kInt8) {
-            if (p.dbg.acc_i32) p.dbg.acc_i32[n] = vi;
-            yv = __fmul_rn(__fmul_rn(__int2float_rn(vi), sx_tok), swn);
-          } else {
-            if (p.dbg.acc_f32) p.dbg.acc_f32[n] = vf;
-            yv = __fmul_rn(__fmul_rn(vf, sx_tok), swn);
-          }
+#pragma unroll
+      for (int tt = 0; tt < (kM + 1) / 2; ++tt) {
+        const int otok = kM == 1 ? 0 : wg + 2 * tt;  // output token of this lane
+        int vi = 0;
+        float vf = 0.0f;
+#pragma unroll
+        for (int w = (kM == 1 ? wg : 0); w < kGemvWarps; w += (kM == 1 ? 2 : 1)) {
+          const float pv = ps[(otok * kGemvWarps + w) * kGemvUnits + u];
+          if constexpr (kInt8)
+            vi += __float_as_int(pv);
+          else
+            vf += pv;
         }
-        p.y[n] = f32_to_bf16_rn(yv);
+        if constexpr (kInt8) {
+          if (kM == 1) vi += __shfl_xor_sync(0xffffffffu, vi, 16);
+#pragma unroll
+          for (int o = 1; o < kQ; o <<= 1) vi += __shfl_xor_sync(0xffffffffu, vi, o);
+        } else {
+          if (kM == 1) vf += __shfl_xor_sync(0xffffffffu, vf, 16);
+#pragma unroll
+          for (int o = 1; o < kQ; o <<= 1) vf += __shfl_xor_sync(0xffffffffu, vf, o);
+        }
+        if ((kM == 1 ? wg == 0 : otok < p.M) && u % kQ == 0 && r < nr) {
+          const int64_t n = r0 + r;
+          const int64_t o = otok * N + n;  // y and debug index [token, row]
+          float yv;
+          if constexpr (kBlock) {
+            yv = vf;
+          } else {
+            const int64_t si = n - row_begin;
+            const float swn = si < sw_cached ? sw_s[si] : __ldg(p.sw + n);
+            const float sxt = sx_s[otok];
+            if constexpr (kInt8) {
+              if (p.dbg.acc_i32) p.dbg.acc_i32[o] = vi;
+              yv = __fmul_rn(__fmul_rn(__int2float_rn(vi), sxt), swn);
+            } else {
+              if (p.dbg.acc_f32) p.dbg.acc_f32[o] = vf;
+              yv = __fmul_rn(__fmul_rn(vf, sxt), swn);
+            }
+          }
+          p.y[o] = f32_to_bf16_rn(yv);
+        }
       }
       __syncwarp();
       if (lane == 0) {
@@ -508,9 +546,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 
 int gemv_max_k() { return kGemvMaxK; }
 
-template <ql_scheme S, int kRs, int kSteps>
+template <ql_scheme S, int kRs, int kSteps, int kM>
 static cudaError_t launch_gemv_r(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
-  cudaError_t e = ensure_smem<gemv_kernel<S, kRs, kSteps>>((int)smem);
+  cudaError_t e = ensure_smem<gemv_kernel<S, kRs, kSteps, kM>>((int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -522,25 +560,37 @@ static cudaError_t launch_gemv_r(const GemvParams& p, int grid, size_t smem, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<S, kRs, kSteps>, p);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<S, kRs, kSteps, kM>, p);
 }
 
 // Steps per warp: 4 when a unit has at most 32 windows of 64 bytes, else 8.
 template <ql_scheme S>
 static cudaError_t launch_gemv_t(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
   const bool long_units = p.seg_len > 32 * 64;
+  if (p.M > 2)
+    return long_units ? launch_gemv_r<S, 4, 8, 4>(p, grid, smem, st) : launch_gemv_r<S, 4, 4, 4>(p, grid, smem, st);
+  if (p.M == 2) {
+    if (p.rows_per_stage == 8)
+      return long_units ? launch_gemv_r<S, 4, 8, 2>(p, grid, smem, st) : launch_gemv_r<S, 4, 4, 2>(p, grid, smem, st);
+    return long_units ? launch_gemv_r<S, 2, 8, 2>(p, grid, smem, st) : launch_gemv_r<S, 2, 4, 2>(p, grid, smem, st);
+  }
   switch (p.rows_per_stage / 2) {
     case 1:
-      return long_units ? launch_gemv_r<S, 1, 8>(p, grid, smem, st) : launch_gemv_r<S, 1, 4>(p, grid, smem, st);
-    case 2: return launch_gemv_r<S, 2, 4>(p, grid, smem, st);
-    case 4: return launch_gemv_r<S, 4, 4>(p, grid, smem, st);
+      return long_units ? launch_gemv_r<S, 1, 8, 1>(p, grid, smem, st) : launch_gemv_r<S, 1, 4, 1>(p, grid, smem, st);
+    case 2: return launch_gemv_r<S, 2, 4, 1>(p, grid, smem, st);
+    case 4: return launch_gemv_r<S, 4, 4, 1>(p, grid, smem, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
+int gemv_max_k_tokens(int64_t M) {
+  return M == 1 ? (int)kGemvMaxK : M == 2 ? (int)kGemvMaxK2 : M <= 4 ? (int)kGemvMaxK4 : 0;
+}
+
 cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
-                        int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg, int num_sms,
-                        DevStatus* status, cudaStream_t st) {
+                        int64_t M, int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg,
+                        int num_sms, DevStatus* status, cudaStream_t st) {
+  if (M < 1 || M > 4 || K > gemv_max_k_tokens(M)) return cudaErrorInvalidValue;
   GemvParams p;
   p.x = x;
   p.wq = static_cast<const uint8_t*>(wq);
@@ -548,25 +598,30 @@ cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, con
   p.y = y;
   p.N = N;
   p.K = K;
+  p.M = (int)M;
   // kRs: the largest power of two <= 4 whose stage of 2 kRs rows fits the
   // ~32 KB copy size (kRs = 1 above 16 KB rows: stages of two rows); the 16
-  // MMA rows are then 2 kRs rows x 8 / kRs segments
+  // MMA rows are then 2 kRs rows x 8 / kRs segments.  M tokens need M x 8 / kRs
+  // B columns: kRs >= 2 for two tokens, kRs = 4 for three or four.
   int rs = 1;
   while (rs < 4 && (int64_t)(4 * rs) * K <= kGemvStageTarget) rs *= 2;
+  if (M == 2) rs = std::max(rs, 2);
+  if (M > 2) rs = 4;
+  const int km = M <= 2 ? (int)M : 4;  // the kernel's token count (three tokens pad to four)
   p.rows_per_stage = 2 * rs;
   p.stage_bytes = (int)(((int64_t)p.rows_per_stage * K + 127) / 128 * 128);
-  const int fixed = gemv_layout(K, p.stage_bytes, 0, kGemvSwCache).total;
+  const int fixed = gemv_layout(K, p.stage_bytes, 0, kGemvSwCache, km).total;
   p.stages = (int)std::min<int64_t>(kGemvMaxStages, (kGemvSmemBudget - fixed) / p.stage_bytes);
   if (p.stages < 2) return cudaErrorInvalidConfiguration;
   const int q = 8 / rs;
   p.seg_len = ((K + q - 1) / q + 127) / 128 * 128;
-  // the kernel keeps at most 64 (kRs = 1) or 32 windows of 64 bytes per unit
-  if (p.seg_len > (rs == 1 ? 64 : 32) * 64) return cudaErrorInvalidValue;
+  // the kernel keeps at most 64 windows of 64 bytes per unit
+  if (p.seg_len > 64 * 64) return cudaErrorInvalidValue;
   p.dbg = dbg ? *dbg : ql_debug{nullptr, nullptr, nullptr, nullptr};
   p.status = status;
   const int64_t stage_rows_total = (N + p.rows_per_stage - 1) / p.rows_per_stage;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms, stage_rows_total));
-  const size_t smem = gemv_layout(K, p.stage_bytes, p.stages, kGemvSwCache).total;
+  const size_t smem = gemv_layout(K, p.stage_bytes, p.stages, kGemvSwCache, km).total;
   switch (scheme) {
     case QL_W8A8_INT8_ROW: return launch_gemv_t<QL_W8A8_INT8_ROW>(p, grid, smem, st);
     case QL_FP8_E4M3_ROW: return launch_gemv_t<QL_FP8_E4M3_ROW>(p, grid, smem, st);

@@ -43,9 +43,11 @@ cudaError_t launch_quantize_weight(ql_scheme scheme, const uint16_t* w, int64_t 
                                    uint8_t* wq, float* sw, cudaStream_t st);
 
 int gemv_max_k();
+int gemv_max_k_tokens(int64_t M);  // largest K the GEMV takes for M tokens (0: none)
+// M = 1 to 4 tokens (extra tokens ride on the MMA's B columns at no extra weight traffic).
 cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
-                        int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg, int num_sms,
-                        DevStatus* status, cudaStream_t st);
+                        int64_t M, int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg,
+                        int num_sms, DevStatus* status, cudaStream_t st);
 
 // Large-M tcgen05 GEMM on pre-quantized activations.
 size_t gemm_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);

@@ -1,10 +1,10 @@
 // ql_quant.cu -- activation and weight quantization kernels.
 //
-// Activations ("Llama 3.1 8B Instruct W8A8", intro and "Loading": inputs
-// rounded to int8 a token at a time; "Meta-Llama-3.1-8B-Instruct-FP8-dynamic"
-// recipe: per-token dynamic symmetric FP8; "Qwen3 8B FP8", "Loading": FP8 128
-// inputs at a time) and weights (the same pages' weight formats: one scale per
-// output row, or one per 128x128 block).
+// Activations ("Llama 3.1 8B Instruct W8A8", intro and "Loading": int8 per
+// token; "Meta-Llama-3.1-8B-Instruct-FP8-dynamic" recipe: per-token dynamic
+// symmetric FP8; "Qwen3 8B FP8", "Loading": E4M3 in groups of 128 along K) and
+// weights (the same pages' weight formats: a scale for each output row, or for
+// each 128x128 block).
 //
 // Every kernel here is HBM-bound: it reads bf16 once and writes one byte per
 // element.  Absmax reductions are warp shuffles (plus one shared-memory step

@@ -4,17 +4,17 @@
  *
  * Three schemes, as the model pages define them:
  *   QL_W8A8_INT8_ROW      "Llama 3.1 8B Instruct W8A8", intro and "Loading":
- *                         int8 weights with one (bf16) scale per output row,
- *                         inputs rounded to int8 a token at a time, int8
- *                         products summed in int32.
+ *                         int8 weights with a bf16 scale for each output row,
+ *                         activations quantized to int8 per token, the int8
+ *                         products accumulated in int32.
  *   QL_FP8_E4M3_ROW       "Meta-Llama-3.1-8B-Instruct-FP8-dynamic" README,
  *                         "Model Optimizations" and the "Creation" recipe: E4M3
  *                         weights per output channel (static, symmetric), E4M3
  *                         activations per token (dynamic, symmetric).
  *   QL_FP8_E4M3_BLOCK128  "Qwen3 8B FP8", intro and "Loading": E4M3 weights with
- *                         one scale per 128x128 block (a multiplier), inputs
- *                         rounded to E4M3 128 inputs at a time; widths must be
- *                         multiples of 128.
+ *                         a multiplying scale for each 128x128 block,
+ *                         activations quantized to E4M3 in groups of 128 along
+ *                         K; widths must be multiples of 128.
  *
  * Numerics (identical in every entry point):
  *   activation scale  s = absmax / 127 (int8) or absmax / 448 (E4M3), one IEEE
@@ -96,7 +96,7 @@ typedef struct ql_debug {
 /* ---------------------------------------------------------------------- */
 
 /* Weight quantization (offline, checkpoint side), on the GPU.
- * Pages: W8A8 intro (int8, one bf16 scale per output row); FP8-dynamic README
+ * Pages: W8A8 intro (int8, a bf16 scale for each output row); FP8-dynamic README
  * "Model Optimizations" / recipe (E4M3, per channel, static, symmetric); Qwen3
  * FP8 intro (E4M3, one multiplier per 128x128 block).
  *   w    device, bf16 [N,K]
@@ -109,9 +109,8 @@ ql_status qlinear_quantize_weight(ql_scheme scheme, const uint16_t* w, int64_t N
 
 /* Dynamic activation quantization (a per-token or per-128-group absmax by warp
  * shuffles, the scale, the rounded codes).  Pages: W8A8 intro and "Loading"
- * ("rounded to int8 a token at a time"); FP8-dynamic recipe (per token,
- * dynamic, symmetric); Qwen3 FP8 "Loading" ("rounded to FP8 128 inputs at a
- * time").
+ * (int8 per token); FP8-dynamic recipe (per token, dynamic, symmetric); Qwen3
+ * FP8 "Loading" (E4M3 in groups of 128 along K).
  *   x    device, bf16 [M,K]
  *   qx   device, out: [M,K] codes
  *   sx   device, out: f32 [M] (row schemes) or [M, K/128] (block scheme) */
@@ -119,8 +118,8 @@ ql_status qlinear_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, i
                                void* qx, float* sx, void* stream);
 
 /* M = 1 decode product, activation quantization fused: one kernel streams
- * each weight byte once.  Pages: W8A8 "Loading" ("one row in a kernel that
- * reads each byte once"); Qwen3 FP8 "Loading" (same, FP8).
+ * each weight byte once.  Pages: W8A8 "Loading" (a single token takes a
+ * kernel that touches every weight byte once); Qwen3 FP8 "Loading" (same, FP8).
  *   x    device, bf16 [1,K]
  *   wq   device, [N,K] codes from qlinear_quantize_weight (or a checkpoint)
  *   sw   device, weight scales as produced by qlinear_quantize_weight
@@ -130,9 +129,13 @@ ql_status qlinear_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, i
 ql_status qlinear_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
                        int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg, void* stream);
 
-/* 2 <= M <= 32 product on the tensor cores (tcgen05, tokens on the MMA N side,
- * weights on the 128-row side, K split across the SMs).  Pages: W8A8
- * "Loading" ("up to 32 rows on tensor cores"); Qwen3 FP8 "Loading" (same).
+/* 1 <= M <= 32 product on the tensor cores (tcgen05, tokens on the MMA N side,
+ * weights on the 128-row side, K split across the SMs).  Up to four tokens
+ * (K <= 16384 for two, K <= 8192 for three or four) run instead on the
+ * qlinear_gemv kernel, which carries them on its MMA's spare columns at the
+ * weight traffic of one token; the result is the same.  Pages: W8A8
+ * "Loading" (batches of at most 32 tokens on the tensor cores); Qwen3 FP8
+ * "Loading" (same).
  * Activation quantization runs in the same call (a short quantize pass
  * overlapped with the weight stream by programmatic dependent launch).
  *   x          device, bf16 [M,K]
@@ -154,8 +157,8 @@ ql_status qlinear_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq
  * TMEM accumulators, or kind::f8f6f4 E4M3 into f32; TMA-fed shared-memory
  * ring; the scale epilogue fused; for the block scheme each 128-wide K block
  * is promoted into f32 registers with its two scales).  Pages: W8A8 "Loading"
- * ("longer inputs rounded to int8 a row at a time and multiplied in int8 ...
- * summing in int32"); Qwen3 FP8 "Loading" (block scales).
+ * (larger batches: per-token int8 activations, int8 products, int32
+ * accumulation); Qwen3 FP8 "Loading" (block scales).
  *   qx, sx     device, from qlinear_quantize_act
  *   workspace  device, qlinear_workspace_bytes(...) bytes (may be 0 / NULL
  *              when that returns 0), same rules as qlinear_gemm_small

@@ -10,12 +10,12 @@ module only marshals numpy arrays through ctypes.  Each function names the
 page passage it follows:
 
 * "Llama 3.1 8B Instruct W8A8" model page, intro and "Loading": int8 weights
-  with one bf16 scale per output row, per-token int8 activations, int32 sums.
+  with a bf16 scale for each output row, per-token int8 activations, int32 sums.
 * "Meta-Llama-3.1-8B-Instruct-FP8-dynamic" README, "Model Optimizations" and
   the "Creation" recipe: E4M3 weights per output channel (static, symmetric),
   E4M3 activations per token (dynamic, symmetric).
-* "Qwen3 8B FP8" model page, intro and "Loading": one multiplier scale per
-  128x128 weight block, activations rounded 128 inputs at a time.
+* "Qwen3 8B FP8" model page, intro and "Loading": a multiplying scale for each
+  128x128 weight block, activations quantized in groups of 128 along K.
 
 Every function has pins in ``tests/test_oracle_*.py`` that do not go through
 the oracle's own formulas (brute force, closed forms, library routines).

@@ -14,14 +14,14 @@
  *
  * Sources (cited by page title and section):
  *  [W8A8]  "Llama 3.1 8B Instruct W8A8" model page, intro paragraph: int8
- *          weights, one bf16 scale per output row, inputs rounded to int8 a
- *          token at a time; "Loading": int8 products summed in int32.
+ *          weights, a bf16 scale for each output row, activations quantized to
+ *          int8 per token; "Loading": int8 products accumulated in int32.
  *  [FP8R]  "Meta-Llama-3.1-8B-Instruct-FP8-dynamic" README, "Model
  *          Optimizations" and the "Creation" recipe: FP8 weights, per-channel
  *          static symmetric; FP8 activations, per-token dynamic symmetric.
  *  [FP8B]  "Qwen3 8B FP8" model page, intro paragraph: E4M3 weights with one
  *          scale per 128x128 block, the scale a multiplier; widths multiples
- *          of 128; "Loading": inputs rounded to FP8 128 inputs at a time.
+ *          of 128; "Loading": activations quantized to FP8 in groups of 128.
  *  [OCP]   OCP 8-bit Floating Point Specification (E4M3: bias 7, three
  *          mantissa bits, no infinities, S.1111.111 is NaN, max 448).
  *
