@@ -98,7 +98,7 @@ __host__ __device__ inline GemvSmemLayout gemv_layout(int64_t K, int stage_bytes
   L.bars = off;  // full[stages], empty[stages], x ready
   off += 2 * kGemvMaxStages * 8 + 8;
   L.flags = off;  // abort flag, per-stage arrival counters, block reduction scratch
-  off += 16 + kGemvMaxStages * 4 + kGemvWarps * 4;
+  off += 16 + kGemvMaxStages * 4 + kGemvWarps * 4 * M;
   L.total = (off + 127) / 128 * 128;
   return L;
 }
@@ -237,24 +237,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   for (int i = tid; i < sw_cached; i += kGemvConsumers) sw_s[i] = __ldg(p.sw + sw_first + i);
 
   tc::grid_dependency_wait();  // x may be produced by the previous kernel
-  // 1. Fused activation quantization of x [1, K] into shared memory: one pass
+  // 1. Fused activation quantization of x [kM, K] into shared memory: one pass
   //    for the absmax (the first kXLoads chunks per thread loaded together),
   //    one for the codes (x is L2-resident by then).
-  for (int tok = 0; tok < kM; ++tok) {
+  if constexpr (kM == 1) {
     const int64_t nchunk8 = K / 8;  // 16-byte chunks of 8 bf16
     constexpr int kXLoads = 8;
-    const uint4* xg = reinterpret_cast<const uint4*>(p.x + tok * K);
-    uint8_t* qx_t = qx_s + tok * xstride;
-    float* sx_t = sx_s + tok * (kBlock ? KB : 1);
-    if (tok >= p.M) {
-      // a padding token (three tokens on the four-token kernel): zero codes
-      // and scales, so its products are zero; its outputs are not written
-      for (int64_t b = tid * 16; b < xstride; b += kGemvConsumers * 16)
-        *reinterpret_cast<uint4*>(qx_t + b) = make_uint4(0, 0, 0, 0);
-      for (int i = tid; i < (kBlock ? (int)KB : 1); i += kGemvConsumers) sx_t[i] = 0.0f;
-      named_bar_sync(kBarConsumers, kGemvConsumers);
-      continue;
-    }
+    const uint4* xg = reinterpret_cast<const uint4*>(p.x);
+    uint8_t* qx_t = qx_s;
+    float* sx_t = sx_s;
     if (kBlock) {
       // 16 consecutive chunks (lanes) form one 128-wide group: no CTA barrier
       for (int64_t base = 0; base < nchunk8; base += kGemvConsumers) {
@@ -312,18 +303,123 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     for (int64_t b = K + tid * 16; b < (K + 63) / 64 * 64; b += kGemvConsumers * 16)
       *reinterpret_cast<uint4*>(qx_t + b) = make_uint4(0, 0, 0, 0);
     named_bar_sync(kBarConsumers, kGemvConsumers);
+  } else {
+    // kM tokens side by side: one absmax pass and one code pass for all of
+    // them, every token's loads in flight together.  Padding tokens (past
+    // p.M) read nothing and get zero codes and scales.
+    const int nchunk8 = (int)(K / 8);  // 16-byte chunks of 8 bf16 per token
+    const uint4* xg = reinterpret_cast<const uint4*>(p.x);  // token tok at tok * nchunk8
+    if constexpr (kBlock) {
+      // flat chunk f = tok * nchunk8 + c; 16 consecutive chunks (lanes) form
+      // one 128-wide group of one token (K % 128 == 0)
+      constexpr int kB = 4;
+      const int total = kM * nchunk8;
+      for (int base = 0; base < total; base += kB * kGemvConsumers) {
+        uint4 v[kB];
+#pragma unroll
+        for (int b = 0; b < kB; ++b) {
+          const int f = base + b * kGemvConsumers + tid;
+          v[b] = f < total && f / nchunk8 < p.M ? __ldg(xg + f) : make_uint4(0, 0, 0, 0);
+        }
+        float sc[kB];
+#pragma unroll
+        for (int b = 0; b < kB; ++b) {
+          float a = absmax_chunk8(v[b]);
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+          sc[b] = a / 448.0f;
+        }
+        // one copy of the code conversion (a rolled loop picking its chunk by
+        // selects)
+#pragma unroll 1
+        for (int b = 0; b < kB; ++b) {
+          uint4 vb = v[0];
+          float sb = sc[0];
+#pragma unroll
+          for (int j = 1; j < kB; ++j)
+            if (b == j) {
+              vb = v[j];
+              sb = sc[j];
+            }
+          const int f = base + b * kGemvConsumers + tid;
+          if (f < total) {
+            const int tok = f / nchunk8, c = f - tok * nchunk8;
+            if ((lane & 15) == 0) sx_s[tok * KB + (c >> 4)] = sb;
+            reinterpret_cast<uint2*>(qx_s + tok * xstride)[c] = quant_chunk8<false>(vb, make_divisor(sb));
+          }
+        }
+      }
+    } else {
+      float amax[kM];
+#pragma unroll
+      for (int tok = 0; tok < kM; ++tok) amax[tok] = 0.0f;
+      for (int c = tid; c < nchunk8; c += 2 * kGemvConsumers) {
+        const int c2 = c + kGemvConsumers;
+        uint4 v[2 * kM];
+#pragma unroll
+        for (int tok = 0; tok < kM; ++tok) {
+          v[2 * tok] = tok < p.M ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
+          v[2 * tok + 1] = tok < p.M && c2 < nchunk8 ? __ldg(xg + tok * nchunk8 + c2) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int tok = 0; tok < kM; ++tok)
+          amax[tok] = fmaxf(amax[tok], fmaxf(absmax_chunk8(v[2 * tok]), absmax_chunk8(v[2 * tok + 1])));
+      }
+#pragma unroll
+      for (int tok = 0; tok < kM; ++tok) {
+        const float a = warp_max(amax[tok]);
+        if (lane == 0) blockred[tok * kGemvWarps + warp] = a;
+      }
+      named_bar_sync(kBarConsumers, kGemvConsumers);
+      Divisor dv[kM];
+      bool all_fast = true;
+#pragma unroll
+      for (int tok = 0; tok < kM; ++tok) {
+        float a = blockred[tok * kGemvWarps];
+#pragma unroll
+        for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, blockred[tok * kGemvWarps + w]);
+        const float sc = a / (kInt8 ? 127.0f : 448.0f);
+        if (tid == 0) sx_s[tok] = sc;
+        dv[tok] = make_divisor(sc);
+        if (tok < p.M) all_fast = all_fast && dv[tok].fast;
+      }
+      // one uniform branch for all tokens: the IEEE path gives the same codes
+      auto emit_all = [&](auto fast) {
+        constexpr bool kFast = decltype(fast)::value;
+#pragma unroll 1
+        for (int c = tid; c < nchunk8; c += kGemvConsumers) {
+          uint4 v[kM];
+#pragma unroll
+          for (int tok = 0; tok < kM; ++tok)
+            v[tok] = tok < p.M ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int tok = 0; tok < kM; ++tok)
+            reinterpret_cast<uint2*>(qx_s + tok * xstride)[c] =
+                tok < p.M ? quant_chunk8<kInt8, kFast>(v[tok], dv[tok]) : make_uint2(0, 0);
+        }
+      };
+      if (all_fast)
+        emit_all(std::true_type{});
+      else
+        emit_all(std::false_type{});
+    }
+    // zero the padding of each token's last 64-byte window so it adds nothing
+    for (int tok = 0; tok < kM; ++tok)
+      for (int64_t b = K + tid * 16; b < (K + 63) / 64 * 64; b += kGemvConsumers * 16)
+        *reinterpret_cast<uint4*>(qx_s + tok * xstride + b) = make_uint4(0, 0, 0, 0);
+    named_bar_sync(kBarConsumers, kGemvConsumers);
   }
   if (tid == 0) mbar_arrive(xready);  // the producer may fill the whole ring now
   if (blockIdx.x == 0 && (p.dbg.qx || p.dbg.sx)) {
-    for (int tok = 0; tok < p.M; ++tok) {
-      for (int64_t c = tid; c < K / 16; c += kGemvConsumers)
-        if (p.dbg.qx)
-          reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.dbg.qx) + tok * K)[c] =
-              reinterpret_cast<const uint4*>(qx_s + tok * xstride)[c];
-      const int ns = kBlock ? (int)KB : 1;
-      for (int i = tid; i < ns; i += kGemvConsumers)
-        if (p.dbg.sx) p.dbg.sx[tok * ns + i] = sx_s[tok * ns + i];
+    // [token, K] codes and [token, groups] scales; rows of K bytes (K % 16 == 0)
+    const int ns = kBlock ? (int)KB : 1;
+    for (int64_t c = tid; c < (kM == 1 ? 1 : p.M) * (K / 16); c += kGemvConsumers) {
+      const int64_t tok = kM == 1 ? 0 : c / (K / 16), cc = kM == 1 ? c : c % (K / 16);
+      if (p.dbg.qx)
+        reinterpret_cast<uint4*>(p.dbg.qx)[c] = reinterpret_cast<const uint4*>(qx_s + tok * xstride)[cc];
     }
+    for (int i = tid; i < (kM == 1 ? 1 : p.M) * ns; i += kGemvConsumers)
+      if (p.dbg.sx) p.dbg.sx[i] = sx_s[i];
   }
 
   // 2. Work split.  A stage holds 2 kRs whole rows (kRs = 1, 2 or 4) cut into
@@ -382,6 +478,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 #pragma unroll
     for (int s = 0; s < kMaxSteps; ++s) e4m3x16_to_f16(xr[s], xh[s]);
   }
+  const float sx_tok = (kBlock || kM > 1) ? 0.0f : sx_s[0];  // one token, row schemes
   float sxr[kMaxSteps / 2];  // block scheme: x scale of each pair's 128-wide group
   int64_t grp0 = 0;
   if constexpr (kBlock) {
@@ -523,7 +620,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
           } else {
             const int64_t si = n - row_begin;
             const float swn = si < sw_cached ? sw_s[si] : __ldg(p.sw + n);
-            const float sxt = sx_s[otok];
+            const float sxt = kM == 1 ? sx_tok : sx_s[otok];
             if constexpr (kInt8) {
               if (p.dbg.acc_i32) p.dbg.acc_i32[o] = vi;
               yv = __fmul_rn(__fmul_rn(__int2float_rn(vi), sxt), swn);
