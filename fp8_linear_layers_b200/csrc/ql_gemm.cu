@@ -26,6 +26,20 @@
 
 namespace ql {
 
+// 32 lanes x 16 consecutive 32-bit TMEM columns (the narrower load keeps
+// the 256-column block epilogue's 128 running sums in registers).
+namespace tc {
+QL_DEVINL void ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+}  // namespace tc
+
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 128;  // bytes of K per stage: one 128-byte swizzle row
 constexpr int kGemmEpiWarps = 8;
@@ -44,17 +58,24 @@ struct GemmParams {
   DevStatus* status;
 };
 
-template <int BN>
+// kStage: the epilogue passes its bf16 rows through a shared-memory box per
+// warp so that its global stores are row-contiguous (the block scheme, whose
+// epilogue cannot overlap the next tile's MMAs: its per-K-block promotion
+// needs the TMEM buffers back at once).
+template <int BN, bool kStaged>
 struct GemmCfg {
   static constexpr int kStageA = kGemmBM * kGemmBK;
   static constexpr int kStageB = BN * kGemmBK;
   static constexpr int kStage = kStageA + kStageB;
-  static constexpr int kStages = (kGemmSmemBudget / kStage) > 8 ? 8 : (kGemmSmemBudget / kStage);
+  static constexpr int kBudget = kStaged ? 192 * 1024 : kGemmSmemBudget;
+  static constexpr int kStages = (kBudget / kStage) > 8 ? 8 : (kBudget / kStage);
   static constexpr int kRing = kStages * kStage;
+  static constexpr int kBox = 32 * 32 * 2;                             // 32 x 32 bf16
+  static constexpr int kStaging = kStaged ? kGemmEpiWarps * kBox : 0;  // one box per warp
   static constexpr int kBufCols = BN <= 128 ? 128 : 256;  // TMEM columns per accumulator
   static constexpr int kBufs = kTmemCols / kBufCols;
   static constexpr int kHalf = BN / 2;                    // columns per epilogue warp
-  static constexpr int kSmem = kRing + 1024 + 256;
+  static constexpr int kSmem = kRing + kStaging + 1024 + 256;
   static_assert(BN % 64 == 0 && BN <= 256, "tile N");
   static_assert(kStage % 1024 == 0, "stages must stay 1024-byte aligned");
 };
@@ -88,16 +109,17 @@ template <ql_scheme S, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmParams p) {
-  using Cfg = GemmCfg<BN>;
   constexpr bool kInt8 = S == QL_W8A8_INT8_ROW;
   constexpr bool kBlock = S == QL_FP8_E4M3_BLOCK128;
+  using Cfg = GemmCfg<BN, kBlock>;
   constexpr uint32_t kIdesc = tc::idesc(kInt8, kGemmBM, BN);
   constexpr int kStages = Cfg::kStages;
   constexpr int kBufs = Cfg::kBufs;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = align1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + Cfg::kRing);
+  uint8_t* staging = ring + Cfg::kRing;  // 1024-byte aligned (stages are)
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + Cfg::kStaging);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + kBufs;
@@ -307,13 +329,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kBufs) & 1, abort_flag));
           if (!ok) break;
           tc::fence_after();
+          // 64 columns: 32-column loads; 128 columns: 16-column loads (registers)
+          constexpr int kW = Cfg::kHalf == 64 ? 32 : 16;
 #pragma unroll
-          for (int c = 0; c < Cfg::kHalf / 32; ++c) {
-            uint32_t r[32];
-            tc::ld32(tmem + lane_base + buf * Cfg::kBufCols + c0 + c * 32, r);
+          for (int c = 0; c < Cfg::kHalf / kW; ++c) {
+            uint32_t r[kW];
+            if constexpr (kW == 32)
+              tc::ld32(tmem + lane_base + buf * Cfg::kBufCols + c0 + c * kW, r);
+            else
+              tc::ld16(tmem + lane_base + buf * Cfg::kBufCols + c0 + c * kW, r);
             tc::ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(__uint_as_float(r[j]), scale, acc[c * 32 + j]);
+            for (int j = 0; j < kW; ++j) acc[c * kW + j] = fmaf(__uint_as_float(r[j]), scale, acc[c * kW + j]);
           }
           tc::fence_before();
           __syncwarp();
@@ -321,9 +348,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ++jt;
         }
         if (!ok) break;
-        if (live_m && live_n) {
+        // Each lane holds one row; stored as is, every warp store would touch
+        // 32 rows.  Per 32 columns the warp writes its 32 x 32 bf16 box to
+        // shared memory (row r's 16-byte chunk k at slot k ^ ((r / 2) % 4):
+        // one bank pass per 8 rows) and reads it back as 8 rows x 4 chunks, so
+        // that each store instruction writes 8 contiguous 64-byte row pieces.
+        uint8_t* box = staging + ew * Cfg::kBox;
+        const int mrow = m0 + q * 32;
+        if (live_n && mrow < p.M) {
 #pragma unroll
-          for (int c = 0; c < Cfg::kHalf / 32; ++c) store_row32(p.y, m, ncol + c * 32, p.N, &acc[c * 32]);
+          for (int c = 0; c < Cfg::kHalf / 32; ++c) {
+            __syncwarp();  // the previous chunk's reads are done
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              uint32_t w[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                w[j] = (uint32_t)f32_to_bf16_rn(acc[c * 32 + 8 * k + 2 * j]) |
+                       ((uint32_t)f32_to_bf16_rn(acc[c * 32 + 8 * k + 2 * j + 1]) << 16);
+              *reinterpret_cast<uint4*>(box + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
+                  make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            __syncwarp();
+            const int k = lane & 3;
+            const int n = ncol + c * 32 + k * 8;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int rr = 8 * i + (lane >> 2);
+              const uint4 v = *reinterpret_cast<const uint4*>(box + rr * 64 + ((k ^ ((rr >> 1) & 3)) << 4));
+              if (mrow + rr < p.M && n + 8 <= p.N)
+                *reinterpret_cast<uint4*>(p.y + (int64_t)(mrow + rr) * p.N + n) = v;
+            }
+          }
         }
       }
     }
@@ -346,7 +402,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 size_t gemm_workspace_bytes(ql_scheme, int64_t, int64_t, int64_t, int) { return 0; }
 
 // Tile width for this shape: fill the SMs' waves best, 128-wide tiles taxed
-// for their higher shared-memory read rate per MMA.
+// for their lower MMA rate.
 static int pick_bn(ql_scheme s, int64_t M, int64_t N, int sms) {
   const int cands_row[3] = {256, 192, 128};
   const int cands_blk[2] = {256, 128};
@@ -359,7 +415,10 @@ static int pick_bn(ql_scheme s, int64_t M, int64_t N, int sms) {
     const int64_t tiles = mt * ((N + c[i] - 1) / c[i]);
     const int64_t waves = (tiles + sms - 1) / sms;
     double eff = (double)(mt * N) / (double)(waves * sms * (int64_t)kGemmBM * c[i] / kGemmBM);
-    if (c[i] == 128) eff *= 0.85;
+    // measured: 128-wide tiles run the MMAs at ~85% of the wider tiles' rate
+    // (row schemes) and ~60% for the block scheme, whose per-K-block
+    // promotion costs the same per tile at either width
+    if (c[i] == 128) eff *= s == QL_FP8_E4M3_BLOCK128 ? 0.6 : 0.85;
     if (eff > best_eff + 1e-9) {
       best_eff = eff;
       best = c[i];
@@ -371,7 +430,7 @@ static int pick_bn(ql_scheme s, int64_t M, int64_t N, int sms) {
 template <ql_scheme S, int BN>
 static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
                                  int sms, cudaStream_t st) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, S == QL_FP8_E4M3_BLOCK128>;
   cudaError_t e = ensure_smem<gemm_kernel<S, BN>>(Cfg::kSmem);
   if (e != cudaSuccess) return e;
   const int grid = (int)std::min<int64_t>((int64_t)p.mt * p.nt, sms);
