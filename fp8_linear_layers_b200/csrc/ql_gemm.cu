@@ -76,7 +76,7 @@ struct GemmCfg {
   static constexpr int kBufs = kTmemCols / kBufCols;
   static constexpr int kHalf = BN / 2;                    // columns per epilogue warp
   static constexpr int kSmem = kRing + kStaging + 1024 + 256;
-  static_assert(BN % 64 == 0 && BN <= 256, "tile N");
+  static_assert(BN % 32 == 0 && BN <= 256, "tile N");
   static_assert(kStage % 1024 == 0, "stages must stay 1024-byte aligned");
 };
 
@@ -85,12 +85,13 @@ QL_DEVINL uint8_t* align1024(uint8_t* p) {
   return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-// Store 32 consecutive bf16 outputs of row m starting at column n.
-QL_DEVINL void store_row32(uint16_t* __restrict__ y, int64_t m, int n, int N, const float* v) {
+// Store W (16 or 32) consecutive bf16 outputs of row m starting at column n.
+template <int W>
+QL_DEVINL void store_row(uint16_t* __restrict__ y, int64_t m, int n, int N, const float* v) {
   uint16_t* dst = y + m * (int64_t)N + n;
-  if (n + 32 <= N && (N & 7) == 0) {
+  if (n + W <= N && (N & 7) == 0) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < W / 8; ++q) {
       uint32_t w[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j)
@@ -100,7 +101,7 @@ QL_DEVINL void store_row32(uint16_t* __restrict__ y, int64_t m, int n, int N, co
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
+    for (int j = 0; j < W; ++j)
       if (n + j < N) dst[j] = f32_to_bf16_rn(v[j]);
   }
 }
@@ -264,18 +265,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!ok) break;
         tc::fence_after();
         const float sxm = live_m ? __ldg(p.sx + m) : 0.0f;
-#pragma unroll 1
-        for (int c = 0; c < Cfg::kHalf / 32; ++c) {
-          const int col = c0 + c * 32;
-          uint32_t r[32];
-          tc::ld32(tmem + lane_base + buf * Cfg::kBufCols + col, r);
+        // W = 32 columns at a time; a 16-column tail for 160- and 224-wide tiles
+        auto chunk = [&](int col, auto wtag) {
+          constexpr int W = decltype(wtag)::value;
+          uint32_t r[W];
+          if constexpr (W == 32)
+            tc::ld32(tmem + lane_base + buf * Cfg::kBufCols + col, r);
+          else
+            tc::ld16(tmem + lane_base + buf * Cfg::kBufCols + col, r);
           tc::ld_wait();
           const int n = n0 + col;
           if (live_m && n < p.N) {
-            float v[32];
-            if (n + 32 <= p.N) {
+            float v[W];
+            if (n + W <= p.N) {
 #pragma unroll
-              for (int j = 0; j < 32; j += 4) {
+              for (int j = 0; j < W; j += 4) {
                 const float4 s4 = __ldg(reinterpret_cast<const float4*>(p.sw + n + j));
                 const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
@@ -286,29 +290,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
             } else {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
+              for (int j = 0; j < W; ++j) {
                 const float a = kInt8 ? __int2float_rn((int)r[j]) : __uint_as_float(r[j]);
                 v[j] = (n + j < p.N) ? __fmul_rn(__fmul_rn(a, sxm), __ldg(p.sw + n + j)) : 0.0f;
               }
             }
             if (p.acc_i32 || p.acc_f32) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
+              for (int j = 0; j < W; ++j) {
                 if (n + j < p.N) {
                   if (kInt8 && p.acc_i32) p.acc_i32[(int64_t)m * p.N + n + j] = (int)r[j];
                   if (!kInt8 && p.acc_f32) p.acc_f32[(int64_t)m * p.N + n + j] = __uint_as_float(r[j]);
                 }
               }
             }
-            store_row32(p.y, m, n, p.N, v);
+            store_row<W>(p.y, m, n, p.N, v);
           }
-        }
+        };
+#pragma unroll 1
+        for (int c = 0; c < Cfg::kHalf / 32; ++c) chunk(c0 + c * 32, std::integral_constant<int, 32>{});
+        if constexpr (Cfg::kHalf % 32 != 0)
+          chunk(c0 + Cfg::kHalf / 32 * 32, std::integral_constant<int, 16>{});
         tc::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);
         ++jt;
       } else {
         // block scheme: promote each 128-deep partial into f32 registers
+        static_assert(BN == 128 || BN == 256, "block tiles are 128 or 256 wide");
         const int ncol = n0 + c0;
         const bool live_n = ncol < p.N;
         const int nbw = ncol >> 7;  // this warp's columns lie in one 128-row weight block
@@ -404,10 +413,10 @@ size_t gemm_workspace_bytes(ql_scheme, int64_t, int64_t, int64_t, int) { return 
 // Tile width for this shape: fill the SMs' waves best, 128-wide tiles taxed
 // for their lower MMA rate.
 static int pick_bn(ql_scheme s, int64_t M, int64_t N, int sms) {
-  const int cands_row[3] = {256, 192, 128};
+  const int cands_row[5] = {256, 224, 192, 160, 128};
   const int cands_blk[2] = {256, 128};
   const int* c = s == QL_FP8_E4M3_BLOCK128 ? cands_blk : cands_row;
-  const int nc = s == QL_FP8_E4M3_BLOCK128 ? 2 : 3;
+  const int nc = s == QL_FP8_E4M3_BLOCK128 ? 2 : 5;
   const int64_t mt = (M + kGemmBM - 1) / kGemmBM;
   int best = c[0];
   double best_eff = -1.0;
@@ -419,6 +428,7 @@ static int pick_bn(ql_scheme s, int64_t M, int64_t N, int sms) {
     // (row schemes) and ~60% for the block scheme, whose per-K-block
     // promotion costs the same per tile at either width
     if (c[i] == 128) eff *= s == QL_FP8_E4M3_BLOCK128 ? 0.6 : 0.85;
+    if (c[i] == 160) eff *= 0.92;
     if (eff > best_eff + 1e-9) {
       best_eff = eff;
       best = c[i];
@@ -464,11 +474,15 @@ cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const
   switch (scheme) {
     case QL_W8A8_INT8_ROW:
       if (BN == 256) return launch_gemm_t<QL_W8A8_INT8_ROW, 256>(p, ta, tb, num_sms, st);
+      if (BN == 224) return launch_gemm_t<QL_W8A8_INT8_ROW, 224>(p, ta, tb, num_sms, st);
       if (BN == 192) return launch_gemm_t<QL_W8A8_INT8_ROW, 192>(p, ta, tb, num_sms, st);
+      if (BN == 160) return launch_gemm_t<QL_W8A8_INT8_ROW, 160>(p, ta, tb, num_sms, st);
       return launch_gemm_t<QL_W8A8_INT8_ROW, 128>(p, ta, tb, num_sms, st);
     case QL_FP8_E4M3_ROW:
       if (BN == 256) return launch_gemm_t<QL_FP8_E4M3_ROW, 256>(p, ta, tb, num_sms, st);
+      if (BN == 224) return launch_gemm_t<QL_FP8_E4M3_ROW, 224>(p, ta, tb, num_sms, st);
       if (BN == 192) return launch_gemm_t<QL_FP8_E4M3_ROW, 192>(p, ta, tb, num_sms, st);
+      if (BN == 160) return launch_gemm_t<QL_FP8_E4M3_ROW, 160>(p, ta, tb, num_sms, st);
       return launch_gemm_t<QL_FP8_E4M3_ROW, 128>(p, ta, tb, num_sms, st);
     default:
       if (BN == 256) return launch_gemm_t<QL_FP8_E4M3_BLOCK128, 256>(p, ta, tb, num_sms, st);

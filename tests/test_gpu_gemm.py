@@ -53,7 +53,9 @@ def _gpu(scheme, qx, sx, wq, sw, want_acc=True):
 
 @pytest.mark.parametrize("scheme", [ql.W8A8_INT8_ROW, ql.FP8_E4M3_ROW])
 @pytest.mark.parametrize("M,N,K", [(128, 256, 128), (128, 256, 4096), (130, 300, 272), (33, 64, 48),
-                                   (1, 1000, 1024), (257, 520, 1040), (384, 768, 2048)])
+                                   (1, 1000, 1024), (257, 520, 1040), (384, 768, 2048),
+                                   # 160- and 224-wide tiles (ragged last tile, N % 8 != 0)
+                                   (384, 6288, 512), (200, 14224, 256), (200, 14220, 256)])
 def test_gemm_small_shapes_full_compare(cuda, scheme, M, N, K):
     qx, sx, wq, sw = _inputs(scheme, M, N, K)
     gy, dbg = _gpu(scheme, qx, sx, wq, sw)
