@@ -58,20 +58,20 @@ struct GemmParams {
   DevStatus* status;
 };
 
-// kStage: the epilogue passes its bf16 rows through a shared-memory box per
-// warp so that its global stores are row-contiguous (the block scheme, whose
-// epilogue cannot overlap the next tile's MMAs: its per-K-block promotion
-// needs the TMEM buffers back at once).
-template <int BN, bool kStaged>
+
+// The epilogue passes its bf16 rows through a 32 x 32 shared-memory box per
+// warp so that its global stores are row-contiguous.  kBlock: the block
+// scheme's ring budget (its per-K-block promotion holds TMEM buffers longer).
+template <int BN, bool kBlock>
 struct GemmCfg {
   static constexpr int kStageA = kGemmBM * kGemmBK;
   static constexpr int kStageB = BN * kGemmBK;
   static constexpr int kStage = kStageA + kStageB;
-  static constexpr int kBudget = kStaged ? 192 * 1024 : kGemmSmemBudget;
+  static constexpr int kBudget = kBlock ? 192 * 1024 : kGemmSmemBudget;
   static constexpr int kStages = (kBudget / kStage) > 8 ? 8 : (kBudget / kStage);
   static constexpr int kRing = kStages * kStage;
   static constexpr int kBox = 32 * 32 * 2;                             // 32 x 32 bf16
-  static constexpr int kStaging = kStaged ? kGemmEpiWarps * kBox : 0;  // one box per warp
+  static constexpr int kStaging = kGemmEpiWarps * kBox;  // one box per warp
   static constexpr int kBufCols = BN <= 128 ? 128 : 256;  // TMEM columns per accumulator
   static constexpr int kBufs = kTmemCols / kBufCols;
   static constexpr int kHalf = BN / 2;                    // columns per epilogue warp
@@ -106,6 +106,29 @@ QL_DEVINL void store_row(uint16_t* __restrict__ y, int64_t m, int n, int N, cons
   }
 }
 
+// Each lane holds one row of 32 bf16 values (w: 16 packed pairs); stored as
+// is, every warp store would touch 32 rows.  The warp writes its 32 x 32 box
+// to shared memory (row r's 16-byte chunk k at slot k ^ ((r / 2) % 4): one
+// bank pass per 8 rows) and reads it back as 8 rows x 4 chunks, so that each
+// global store instruction writes 8 contiguous 64-byte row pieces.  Rows
+// past M are not written; the caller keeps the 32 columns inside N, N % 8 == 0.
+QL_DEVINL void store_box32(uint8_t* box, int lane, const uint32_t (&w)[16], uint16_t* __restrict__ y,
+                           int mrow, int ncol, int M, int N) {
+  __syncwarp();  // the box's previous reads are done
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    *reinterpret_cast<uint4*>(box + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
+        make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  __syncwarp();
+  const int k = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = 8 * i + (lane >> 2);
+    const uint4 v = *reinterpret_cast<const uint4*>(box + rr * 64 + ((k ^ ((rr >> 1) & 3)) << 4));
+    if (mrow + rr < M) *reinterpret_cast<uint4*>(y + (int64_t)(mrow + rr) * N + ncol + k * 8) = v;
+  }
+}
+
 template <ql_scheme S, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -130,6 +153,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = p.mt * p.nt;
+  // this CTA's tiles b, b + G, ... as (tile, K blocks [lo, hi)); fn returns
+  // false to stop
+  auto for_each_item = [&](auto&& fn) {
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x)
+      if (!fn(t, 0, p.nkb)) return;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -162,21 +191,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint64_t pol_b = l2_policy_evict_first();  // W_q: read by the few M tiles at once
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      for_each_item([&](int t, int lo, int hi) -> bool {
         const int m0 = (t % p.mt) * kGemmBM, n0 = (t / p.mt) * BN;
-        for (int kb = 0; kb < p.nkb; ++kb, ++it) {
+        for (int kb = lo; kb < hi; ++kb, ++it) {
           const int s = it % kStages;
           if (it >= (uint32_t)kStages &&
               !mbar_wait_bounded(&empty[s], ((it / kStages) - 1) & 1, abort_flag)) {
             ok = false;
-            break;
+            return false;
           }
           uint8_t* st = ring + s * Cfg::kStage;
           mbar_arrive_expect_tx(&full[s], Cfg::kStage);
           tc::tma_load_2d(st, &tmA, kb * kGemmBK, m0, &full[s], pol_a);
           tc::tma_load_2d(st + Cfg::kStageA, &tmB, kb * kGemmBK, n0, &full[s], pol_b);
         }
-      }
+        return true;
+      });
       if (!ok) {
         if (!*abort_flag) record_timeout(p.status, KID_GEMM, 1);
         *abort_flag = 1;
@@ -190,25 +220,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, jt = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      for_each_item([&](int, int lo, int hi) -> bool {
         uint32_t d = 0;
         if (!kBlock) {
           const uint32_t buf = jt % kBufs;
           if (jt >= (uint32_t)kBufs &&
               !mbar_wait_bounded(&tempty[buf], ((jt / kBufs) - 1) & 1, abort_flag)) {
             ok = false;
-            break;
+            return false;
           }
           tc::fence_after();
           d = tmem + buf * Cfg::kBufCols;
         }
-        for (int kb = 0; kb < p.nkb; ++kb, ++it) {
+        for (int kb = lo; kb < hi; ++kb, ++it) {
           if (kBlock) {
             const uint32_t buf = jt % kBufs;
             if (jt >= (uint32_t)kBufs &&
                 !mbar_wait_bounded(&tempty[buf], ((jt / kBufs) - 1) & 1, abort_flag)) {
               ok = false;
-              break;
+              return false;
             }
             tc::fence_after();
             d = tmem + buf * Cfg::kBufCols;
@@ -216,7 +246,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int s = it % kStages;
           if (!mbar_wait_bounded(&full[s], (it / kStages) & 1, abort_flag)) {
             ok = false;
-            break;
+            return false;
           }
           tc::fence_after();
           const uint32_t a_addr = smem_u32(ring + s * Cfg::kStage);
@@ -225,19 +255,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int k = 0; k < kGemmBK / 32; ++k)
             tc::mma<kInt8>(d, adesc + 2 * k, bdesc + 2 * k, kIdesc,
-                           kBlock ? (k != 0) : ((kb | k) != 0));
+                           kBlock ? (k != 0) : (kb != lo || k != 0));
           tc::commit(&empty[s]);  // the stage is free once these MMAs have read it
           if (kBlock) {
             tc::commit(&tfull[jt % kBufs]);
             ++jt;
           }
         }
-        if (!ok) break;
         if (!kBlock) {
           tc::commit(&tfull[jt % kBufs]);
           ++jt;
         }
-      }
+        return true;
+      });
       if (!ok) {
         if (!*abort_flag) record_timeout(p.status, KID_GEMM, 2);
         *abort_flag = 1;
@@ -254,19 +284,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int KB = p.K / 128;
     uint32_t jt = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+    for_each_item([&](int t, int lo, int hi) -> bool {
       const int m0 = (t % p.mt) * kGemmBM, n0 = (t / p.mt) * BN;
       const int m = m0 + q * 32 + lane;
       const bool live_m = m < p.M;
       const int c0 = h * Cfg::kHalf;  // first column of this warp inside the tile
       if constexpr (!kBlock) {
+        // The scales do not depend on the MMAs: their L2 latency overlaps the
+        // wait for the accumulator.  Lane j holds s_w of column 32 c + j of
+        // this warp's chunk c; the chunk's lanes share them by shuffles.
+        constexpr int kChunks = (Cfg::kHalf + 31) / 32;
+        const float sxm = live_m ? __ldg(p.sx + m) : 0.0f;
+        float swl[kChunks];
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          const int n = n0 + c0 + c * 32 + lane;
+          swl[c] = c * 32 + lane < Cfg::kHalf && n < p.N ? __ldg(p.sw + n) : 0.0f;
+        }
         const uint32_t buf = jt % kBufs;
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kBufs) & 1, abort_flag));
-        if (!ok) break;
+        if (!ok) return false;
         tc::fence_after();
-        const float sxm = live_m ? __ldg(p.sx + m) : 0.0f;
         // W = 32 columns at a time; a 16-column tail for 160- and 224-wide tiles
-        auto chunk = [&](int col, auto wtag) {
+        auto chunk = [&](int col, float swc, auto wtag) {
           constexpr int W = decltype(wtag)::value;
           uint32_t r[W];
           if constexpr (W == 32)
@@ -275,26 +315,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tc::ld16(tmem + lane_base + buf * Cfg::kBufCols + col, r);
           tc::ld_wait();
           const int n = n0 + col;
+          float v[W];
+#pragma unroll
+          for (int j = 0; j < W; ++j) {
+            const float a = kInt8 ? __int2float_rn((int)r[j]) : __uint_as_float(r[j]);
+            v[j] = __fmul_rn(__fmul_rn(a, sxm), __shfl_sync(0xffffffffu, swc, j));
+          }
           if (live_m && n < p.N) {
-            float v[W];
-            if (n + W <= p.N) {
-#pragma unroll
-              for (int j = 0; j < W; j += 4) {
-                const float4 s4 = __ldg(reinterpret_cast<const float4*>(p.sw + n + j));
-                const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  const float a = kInt8 ? __int2float_rn((int)r[j + u]) : __uint_as_float(r[j + u]);
-                  v[j + u] = __fmul_rn(__fmul_rn(a, sxm), sv[u]);
-                }
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < W; ++j) {
-                const float a = kInt8 ? __int2float_rn((int)r[j]) : __uint_as_float(r[j]);
-                v[j] = (n + j < p.N) ? __fmul_rn(__fmul_rn(a, sxm), __ldg(p.sw + n + j)) : 0.0f;
-              }
-            }
             if (p.acc_i32 || p.acc_f32) {
 #pragma unroll
               for (int j = 0; j < W; ++j) {
@@ -304,13 +331,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
               }
             }
+          }
+          // whole 32-column chunks inside N leave through the box (uniform per warp)
+          if (W == 32 && n + 32 <= p.N && (p.N & 7) == 0) {
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              w[j] = (uint32_t)f32_to_bf16_rn(v[2 * j]) | ((uint32_t)f32_to_bf16_rn(v[2 * j + 1]) << 16);
+            store_box32(staging + ew * Cfg::kBox, lane, w, p.y, m0 + q * 32, n, p.M, p.N);
+          } else if (live_m && n < p.N) {
             store_row<W>(p.y, m, n, p.N, v);
           }
         };
-#pragma unroll 1
-        for (int c = 0; c < Cfg::kHalf / 32; ++c) chunk(c0 + c * 32, std::integral_constant<int, 32>{});
+#pragma unroll
+        for (int c = 0; c < Cfg::kHalf / 32; ++c) chunk(c0 + c * 32, swl[c], std::integral_constant<int, 32>{});
         if constexpr (Cfg::kHalf % 32 != 0)
-          chunk(c0 + Cfg::kHalf / 32 * 32, std::integral_constant<int, 16>{});
+          chunk(c0 + Cfg::kHalf / 32 * 32, swl[kChunks - 1], std::integral_constant<int, 16>{});
         tc::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -326,17 +362,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int j = 0; j < Cfg::kHalf; ++j) acc[j] = 0.0f;
         // scales of K block kb+1 are loaded while the MMAs of block kb run
         const bool live = live_m && live_n;
-        float sx_next = live ? __ldg(p.sx + (int64_t)m * KB) : 0.0f;
-        float sw_next = live ? __ldg(p.sw + (int64_t)nbw * KB) : 0.0f;
-        for (int kb = 0; kb < p.nkb; ++kb) {
+        float sx_next = live ? __ldg(p.sx + (int64_t)m * KB + lo) : 0.0f;
+        float sw_next = live ? __ldg(p.sw + (int64_t)nbw * KB + lo) : 0.0f;
+        for (int kb = lo; kb < hi; ++kb) {
           const float scale = sx_next * sw_next;
-          if (live && kb + 1 < p.nkb) {
+          if (live && kb + 1 < hi) {
             sx_next = __ldg(p.sx + (int64_t)m * KB + kb + 1);
             sw_next = __ldg(p.sw + (int64_t)nbw * KB + kb + 1);
           }
           const uint32_t buf = jt % kBufs;
           ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kBufs) & 1, abort_flag));
-          if (!ok) break;
+          if (!ok) return false;
           tc::fence_after();
           // 64 columns: 32-column loads; 128 columns: 16-column loads (registers)
           constexpr int kW = Cfg::kHalf == 64 ? 32 : 16;
@@ -356,42 +392,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (lane == 0) mbar_arrive(&tempty[buf]);
           ++jt;
         }
-        if (!ok) break;
-        // Each lane holds one row; stored as is, every warp store would touch
-        // 32 rows.  Per 32 columns the warp writes its 32 x 32 bf16 box to
-        // shared memory (row r's 16-byte chunk k at slot k ^ ((r / 2) % 4):
-        // one bank pass per 8 rows) and reads it back as 8 rows x 4 chunks, so
-        // that each store instruction writes 8 contiguous 64-byte row pieces.
-        uint8_t* box = staging + ew * Cfg::kBox;
         const int mrow = m0 + q * 32;
         if (live_n && mrow < p.M) {
 #pragma unroll
           for (int c = 0; c < Cfg::kHalf / 32; ++c) {
-            __syncwarp();  // the previous chunk's reads are done
+            uint32_t w[16];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              uint32_t w[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                w[j] = (uint32_t)f32_to_bf16_rn(acc[c * 32 + 8 * k + 2 * j]) |
-                       ((uint32_t)f32_to_bf16_rn(acc[c * 32 + 8 * k + 2 * j + 1]) << 16);
-              *reinterpret_cast<uint4*>(box + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
-                  make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            __syncwarp();
-            const int k = lane & 3;
-            const int n = ncol + c * 32 + k * 8;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int rr = 8 * i + (lane >> 2);
-              const uint4 v = *reinterpret_cast<const uint4*>(box + rr * 64 + ((k ^ ((rr >> 1) & 3)) << 4));
-              if (mrow + rr < p.M && n + 8 <= p.N)
-                *reinterpret_cast<uint4*>(p.y + (int64_t)(mrow + rr) * p.N + n) = v;
-            }
+            for (int j = 0; j < 16; ++j)
+              w[j] = (uint32_t)f32_to_bf16_rn(acc[c * 32 + 2 * j]) |
+                     ((uint32_t)f32_to_bf16_rn(acc[c * 32 + 2 * j + 1]) << 16);
+            store_box32(staging + ew * Cfg::kBox, lane, w, p.y, mrow, ncol + c * 32, p.M, p.N);
           }
         }
       }
-    }
+      return true;
+    });
     if (!ok) {
       if (lane == 0 && !*abort_flag) record_timeout(p.status, KID_GEMM, 3);
       *abort_flag = 1;
@@ -407,8 +422,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-
-size_t gemm_workspace_bytes(ql_scheme, int64_t, int64_t, int64_t, int) { return 0; }
 
 // Tile width for this shape: fill the SMs' waves best, 128-wide tiles taxed
 // for their lower MMA rate.
@@ -436,6 +449,8 @@ static int pick_bn(ql_scheme s, int64_t M, int64_t N, int sms) {
   }
   return best;
 }
+
+size_t gemm_workspace_bytes(ql_scheme, int64_t, int64_t, int64_t, int) { return 0; }
 
 template <ql_scheme S, int BN>
 static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
