@@ -357,9 +357,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int ncol = n0 + c0;
         const bool live_n = ncol < p.N;
         const int nbw = ncol >> 7;  // this warp's columns lie in one 128-row weight block
-        float acc[Cfg::kHalf];
+        // running sums as pairs: one packed f32x2 FMA (two IEEE fmas) per pair
+        float2 acc[Cfg::kHalf / 2];
 #pragma unroll
-        for (int j = 0; j < Cfg::kHalf; ++j) acc[j] = 0.0f;
+        for (int j = 0; j < Cfg::kHalf / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
         // scales of K block kb+1 are loaded while the MMAs of block kb run
         const bool live = live_m && live_n;
         float sx_next = live ? __ldg(p.sx + (int64_t)m * KB + lo) : 0.0f;
@@ -385,7 +386,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               tc::ld16(tmem + lane_base + buf * Cfg::kBufCols + c0 + c * kW, r);
             tc::ld_wait();
 #pragma unroll
-            for (int j = 0; j < kW; ++j) acc[c * kW + j] = fmaf(__uint_as_float(r[j]), scale, acc[c * kW + j]);
+            for (int j = 0; j < kW / 2; ++j)
+              acc[(c * kW) / 2 + j] = __ffma2_rn(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])),
+                                                 make_float2(scale, scale), acc[(c * kW) / 2 + j]);
           }
           tc::fence_before();
           __syncwarp();
@@ -399,8 +402,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t w[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              w[j] = (uint32_t)f32_to_bf16_rn(acc[c * 32 + 2 * j]) |
-                     ((uint32_t)f32_to_bf16_rn(acc[c * 32 + 2 * j + 1]) << 16);
+              w[j] = (uint32_t)f32_to_bf16_rn(acc[c * 16 + j].x) | ((uint32_t)f32_to_bf16_rn(acc[c * 16 + j].y) << 16);
             store_box32(staging + ew * Cfg::kBox, lane, w, p.y, mrow, ncol + c * 32, p.M, p.N);
           }
         }
