@@ -261,14 +261,26 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         }
       }
     } else {
+      // Ring slot kEarlyStages is not written before x is quantized (the
+      // producer waits for xready there): when x fits, the absmax pass parks
+      // its chunks in that slot and the code pass reads them from shared
+      // memory instead of a second trip to L2.
+      uint4* stash = nst > kEarlyStages && (int64_t)p.stage_bytes >= nchunk8 * 16
+                         ? reinterpret_cast<uint4*>(ring + kEarlyStages * p.stage_bytes)
+                         : nullptr;
       float a_tok = 0.0f;
 #pragma unroll
       for (int i = 0; i < kXLoads; ++i) {
         const int64_t c = tid + (int64_t)i * kGemvConsumers;
-        a_tok = fmaxf(a_tok, absmax_chunk8(c < nchunk8 ? __ldg(xg + c) : make_uint4(0, 0, 0, 0)));
+        const uint4 v = c < nchunk8 ? __ldg(xg + c) : make_uint4(0, 0, 0, 0);
+        if (stash && c < nchunk8) stash[c] = v;
+        a_tok = fmaxf(a_tok, absmax_chunk8(v));
       }
-      for (int64_t c = tid + (int64_t)kXLoads * kGemvConsumers; c < nchunk8; c += kGemvConsumers)
-        a_tok = fmaxf(a_tok, absmax_chunk8(__ldg(xg + c)));
+      for (int64_t c = tid + (int64_t)kXLoads * kGemvConsumers; c < nchunk8; c += kGemvConsumers) {
+        const uint4 v = __ldg(xg + c);
+        if (stash) stash[c] = v;
+        a_tok = fmaxf(a_tok, absmax_chunk8(v));
+      }
       a_tok = warp_max(a_tok);
       if (lane == 0) blockred[warp] = a_tok;
       named_bar_sync(kBarConsumers, kGemvConsumers);
@@ -281,15 +293,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       // one uniform branch: the eight values of every chunk run side by side
       auto emit_all = [&](auto fast) {
         constexpr bool kFast = decltype(fast)::value;
-        // a rolled loop re-reading x (L2-resident): the straight-line form
-        // measured slower inside a step, where its instructions are fetched
-        // while the weight stream congests L2
+        // a rolled loop re-reading x (parked in shared memory, else
+        // L2-resident): the straight-line form measured slower inside a step,
+        // where its instructions are fetched while the weight stream congests L2
         uint2* q2 = reinterpret_cast<uint2*>(qx_t);
 #pragma unroll 1
         for (int64_t c = tid; c < nchunk8; c += 2 * kGemvConsumers) {
           const int64_t c2 = c + kGemvConsumers;
-          const uint4 v0 = __ldg(xg + c);
-          const uint4 v1 = c2 < nchunk8 ? __ldg(xg + c2) : make_uint4(0, 0, 0, 0);
+          const uint4 v0 = stash ? stash[c] : __ldg(xg + c);
+          const uint4 v1 = c2 < nchunk8 ? (stash ? stash[c2] : __ldg(xg + c2)) : make_uint4(0, 0, 0, 0);
           q2[c] = quant_chunk8<kInt8, kFast>(v0, dv);
           if (c2 < nchunk8) q2[c2] = quant_chunk8<kInt8, kFast>(v1, dv);
         }
@@ -298,6 +310,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         emit_all(std::true_type{});
       else
         emit_all(std::false_type{});
+      // the slot's next writer is the producer's bulk copy (the async proxy)
+      if (stash) fence_proxy_async_smem();
     }
     // zero the padding of the last 64-byte window so it adds nothing
     for (int64_t b = K + tid * 16; b < (K + 63) / 64 * 64; b += kGemvConsumers * 16)
