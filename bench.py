@@ -8,6 +8,7 @@ per-row: 14 GEMV launches (activation quantization fused) per step.  Metric:
 HBM GB/s of algorithmic bytes (weights + scales + x + y) per second, whole job.
 
 Other workloads (``--workload``), same JSON line:
+  decode-fused  the decode layer with q|k|v and gate|up side by side along N: 8 GEMVs
   prefill       W8A8, M in {512, 1024} x gate/up/down/fused-qkv: TOPS
   small         M in {2, 8, 16, 32} x the 7 Llama shapes x {W8A8, FP8 row}: GB/s
   kproj         W8A8, M = 8, N = 1024, K = 4096 (8 outlier channels): GB/s
@@ -104,6 +105,11 @@ def workloads():
         "decode", "decode GEMV M=1: one Llama-3.1-8B layer's 7 projections (q,k,v,o,gate,up,down) "
         "in W8A8 int8 and in FP8 E4M3 per-row, per-token dynamic activation quantization fused", "GB/s",
         [Product(n, s, 1, N, K, oc(K)) for n, N, K in S.LLAMA31_8B for s in (INT8, FP8R)])
+    w["decode-fused"] = Workload(
+        "decode-fused", "decode GEMV M=1: one Llama-3.1-8B layer with q|k|v and gate|up stored side by "
+        "side along N (qkv 6144x4096, o 4096x4096, gate_up 28672x4096, down 4096x14336) in W8A8 int8 and "
+        "in FP8 E4M3 per-row, per-token dynamic activation quantization fused", "GB/s",
+        [Product(n, s, 1, N, K, oc(K)) for n, N, K in S.LLAMA31_8B_FUSED for s in (INT8, FP8R)])
     w["prefill"] = Workload(
         "prefill", "prefill W8A8 int8 GEMM: M in {512, 1024} x Llama-3.1-8B gate/up 14336x4096, "
         "down 4096x14336, fused qkv 6144x4096; per-token quantization + tcgen05 kind::i8", "TOPS",
@@ -135,7 +141,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["qlinear", "reference"], default="qlinear")
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "prefill", "small", "kproj", "qwen-decode", "qwen-small", "qwen-prefill"])
+                    choices=["decode", "decode-fused", "prefill", "small", "kproj", "qwen-decode",
+                             "qwen-small", "qwen-prefill"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -296,6 +303,8 @@ class Runner:
             item = dict(p=p, wqs=wqs, xs=xs, ys=ys, ws=ws, amount=wl.amount(p))
             if p.M > 32:  # pre-quantized activations for the dominant-kernel timing
                 item["q"] = [ql.quantize_act(p.scheme, x) for x in xs]
+                gws = ql.workspace_bytes(p.scheme, p.M, p.N, p.K)  # the K split's sums (block scheme)
+                item["ws_gemm"] = ql.new_workspace(gws) if gws else None
             self.items.append(item)
         del weights
         torch.cuda.synchronize()
@@ -323,7 +332,7 @@ class Runner:
                 ql.gemm_small(p.scheme, i["xs"][t], wq, sw, i["ws"], y=i["ys"][t])
             else:
                 qx, sx = i["q"][t]
-                ql.gemm(p.scheme, qx, sx, wq, sw, y=i["ys"][t])
+                ql.gemm(p.scheme, qx, sx, wq, sw, workspace=i["ws_gemm"], y=i["ys"][t])
 
     def capture(self, fn, stream):
         torch = self.torch

@@ -207,11 +207,14 @@ ql_status qlinear_gemm(ql_scheme scheme, const void* qx, const float* sx, const 
   QL_TRY(check_debug(dbg));
   DeviceInfo d;
   QL_TRY(current_device(&d));
+  // The workspace is optional here: with it, block-scheme shapes that fill
+  // less than one wave of tiles split K over more CTAs; without it, whole tiles.
   const size_t need_ws = ql::gemm_workspace_bytes(scheme, M, N, K, d.sms);
-  if (need_ws && (!workspace || ws_bytes < need_ws)) return QL_ERR_WORKSPACE;
-  if (need_ws && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return QL_ERR_MISALIGNED;
-  cudaError_t e = ql::launch_gemm(scheme, qx, sx, wq, sw, M, N, K, y, workspace, ws_bytes, dbg,
-                                  d.sms, d.status, static_cast<cudaStream_t>(stream));
+  const bool use_ws = need_ws && workspace && ws_bytes >= need_ws;
+  if (use_ws && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return QL_ERR_MISALIGNED;
+  cudaError_t e = ql::launch_gemm(scheme, qx, sx, wq, sw, M, N, K, y, use_ws ? workspace : nullptr,
+                                  use_ws ? ws_bytes : 0, dbg, d.sms, d.status,
+                                  static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm");
 }
 

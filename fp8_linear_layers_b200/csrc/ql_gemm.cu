@@ -53,10 +53,30 @@ struct GemmParams {
   uint16_t* y;
   int M, N, K;
   int mt, nt, nkb;  // tiles along M and N, K blocks of 128
+  int split;        // block scheme: K halves per tile (1 = whole tiles, or 2)
+  float* parts;     // split = 2: f32 partial sums, [half][tile][warp][column / 4][lane][4]
+  uint32_t* counters;  // split = 2: [mt * nt] arrivals per tile, zero between calls
   int32_t* acc_i32;
   float* acc_f32;
   DevStatus* status;
 };
+
+constexpr uint32_t kGemmEpiBar = 1;  // named barrier of the epilogue warps
+
+// OR vote over the epilogue warps that doubles as their barrier.
+QL_DEVINL bool gemm_epi_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(kGemmEpiBar), "r"(kGemmEpiWarps * 32)
+      : "memory");
+  return r != 0;
+}
+
 
 
 // The epilogue passes its bf16 rows through a 32 x 32 shared-memory box per
@@ -150,14 +170,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* mma_done = tempty + kBufs;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* last_flag = abort_flag + 1;  // split tiles: this CTA adds the last part
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = p.mt * p.nt;
-  // this CTA's tiles b, b + G, ... as (tile, K blocks [lo, hi)); fn returns
-  // false to stop
+  // this CTA's work items b, b + G, ... as (tile, K blocks [lo, hi)): item i
+  // is K range i % split of tile i / split; fn returns false to stop
+  const int nitems = ntiles * p.split;
   auto for_each_item = [&](auto&& fn) {
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x)
-      if (!fn(t, 0, p.nkb)) return;
+    for (int i = blockIdx.x; i < nitems; i += gridDim.x) {
+      const int t = i / p.split, r = i - t * p.split;
+      if (!fn(t, (int)(((int64_t)r * p.nkb) / p.split), (int)(((int64_t)(r + 1) * p.nkb) / p.split))) return;
+    }
   };
 
   if (threadIdx.x == 0) {
@@ -373,7 +397,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const uint32_t buf = jt % kBufs;
           ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kBufs) & 1, abort_flag));
-          if (!ok) return false;
+          if (!ok) break;
           tc::fence_after();
           // 64 columns: 32-column loads; 128 columns: 16-column loads (registers)
           constexpr int kW = Cfg::kHalf == 64 ? 32 : 16;
@@ -394,6 +418,60 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[buf]);
           ++jt;
+        }
+        if (p.split == 1) {
+          if (!ok) return false;
+        } else {
+          // Split tile: every epilogue warp reaches the votes and barriers
+          // below, so they leave together if any of them gave up a wait.
+          if (gemm_epi_any(!ok)) return false;
+          // Each K half parks its sums in its own slab, laid out the way the
+          // warps hold them (lane-minor, so each warp store writes 512
+          // contiguous bytes; stored as [M, N] rows, every store touched 32
+          // rows), and the CTA that arrives second reads the other half's and
+          // adds the two (f32 addition commutes: the same bits in either order
+          // of arrival) and writes y.  (Adding the halves with L2 reductions
+          // measured slower than the work saved.)
+          const int half = hi == p.nkb ? 1 : 0;  // the second half ends at the last K block
+          constexpr int kV = Cfg::kHalf / 4;     // float4 per thread
+          auto slot = [&](int hf) {
+            return reinterpret_cast<float4*>(p.parts) +
+                   ((int64_t)(hf * ntiles + t) * kGemmEpiWarps + ew) * kV * 32 + lane;
+          };
+          {
+            float4* mine = slot(half);
+#pragma unroll
+            for (int j = 0; j < kV; ++j)
+              __stcg(mine + j * 32, make_float4(acc[2 * j].x, acc[2 * j].y, acc[2 * j + 1].x, acc[2 * j + 1].y));
+          }
+          __threadfence();
+          named_bar_sync(kGemmEpiBar, kGemmEpiWarps * 32);
+          if (ew == 0 && lane == 0) {
+            const unsigned old = atomicAdd(p.counters + t, 1u);
+            *last_flag = old == (unsigned)(p.split - 1);
+          }
+          named_bar_sync(kGemmEpiBar, kGemmEpiWarps * 32);
+          if (!*last_flag) return true;
+          __threadfence();
+          {
+            const float4* other = slot(1 - half);
+            // eight 16-byte loads in flight at a time (the 128 running sums
+            // leave no registers for more)
+#pragma unroll
+            for (int j0 = 0; j0 < kV; j0 += 8) {
+              float4 v[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) v[j] = __ldcg(other + (j0 + j) * 32);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                acc[2 * (j0 + j)] = make_float2(acc[2 * (j0 + j)].x + v[j].x, acc[2 * (j0 + j)].y + v[j].y);
+                acc[2 * (j0 + j) + 1] =
+                    make_float2(acc[2 * (j0 + j) + 1].x + v[j].z, acc[2 * (j0 + j) + 1].y + v[j].w);
+              }
+              asm volatile("" ::: "memory");
+            }
+          }
+          if (ew == 0 && lane == 0) p.counters[t] = 0u;  // both halves have arrived
         }
         const int mrow = m0 + q * 32;
         if (live_n && mrow < p.M) {
@@ -452,7 +530,38 @@ static int pick_bn(ql_scheme s, int64_t M, int64_t N, int sms) {
   return best;
 }
 
-size_t gemm_workspace_bytes(ql_scheme, int64_t, int64_t, int64_t, int) { return 0; }
+// Block scheme with at most half a wave of 256-wide tiles and a long K
+// (M = 512 with N = 4096, K >= 8192: down_proj): each tile's K blocks are
+// split in two halves run by two CTAs, which meet in an f32 workspace.
+// Measured per K block, 256-wide tiles promote at ~1.6x the 128-wide rate, so
+// a split 256-wide tile beats a whole 128-wide one once K is long enough to
+// repay parking and re-reading the f32 halves (Qwen3-8B down_proj at M = 512:
+// 47 -> 36 us; at K = 4096 the split measured 2% slower than whole 128-wide
+// tiles).  Otherwise (and for the row schemes) whole tiles.
+struct GemmPlan {
+  int bn, split;
+};
+
+static GemmPlan plan_gemm(ql_scheme s, int64_t M, int64_t N, int64_t K, int sms) {
+  GemmPlan pl{pick_bn(s, M, N, sms), 1};
+  if (s != QL_FP8_E4M3_BLOCK128) return pl;
+  const int64_t tiles = ((M + kGemmBM - 1) / kGemmBM) * ((N + 255) / 256);
+  const int64_t nkb = (K + kGemmBK - 1) / kGemmBK;
+  if (2 * tiles <= sms && nkb >= 64) pl = GemmPlan{256, 2};
+  return pl;
+}
+
+static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+// Two slabs of one 128 x 256 f32 tile per tile.
+static size_t split_parts_bytes(int64_t tiles) { return (size_t)2 * tiles * kGemmBM * 256 * 4; }
+
+size_t gemm_workspace_bytes(ql_scheme s, int64_t M, int64_t N, int64_t K, int sms) {
+  const GemmPlan pl = plan_gemm(s, M, N, K, sms);
+  if (pl.split == 1) return 0;
+  const int64_t tiles = ((M + kGemmBM - 1) / kGemmBM) * ((N + pl.bn - 1) / pl.bn);
+  return align256(split_parts_bytes(tiles)) + align256((size_t)tiles * 4);
+}
 
 template <ql_scheme S, int BN>
 static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
@@ -460,16 +569,20 @@ static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, cons
   using Cfg = GemmCfg<BN, S == QL_FP8_E4M3_BLOCK128>;
   cudaError_t e = ensure_smem<gemm_kernel<S, BN>>(Cfg::kSmem);
   if (e != cudaSuccess) return e;
-  const int grid = (int)std::min<int64_t>((int64_t)p.mt * p.nt, sms);
+  const int grid = (int)std::min<int64_t>((int64_t)p.mt * p.nt * p.split, sms);
   gemm_kernel<S, BN><<<grid, kGemmThreads, Cfg::kSmem, st>>>(a, b, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
-                        const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y, void*,
-                        size_t, const ql_debug* dbg, int num_sms, DevStatus* status,
+                        const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
+                        size_t ws_bytes, const ql_debug* dbg, int num_sms, DevStatus* status,
                         cudaStream_t st) {
-  const int BN = pick_bn(scheme, M, N, num_sms);
+  // the K split needs its workspace; without one, whole tiles
+  GemmPlan pl = plan_gemm(scheme, M, N, K, num_sms);
+  const size_t need = gemm_workspace_bytes(scheme, M, N, K, num_sms);
+  if (pl.split > 1 && (workspace == nullptr || ws_bytes < need)) pl = GemmPlan{pick_bn(scheme, M, N, num_sms), 1};
+  const int BN = pl.bn;
   GemmParams p;
   p.sx = sx;
   p.sw = sw;
@@ -480,6 +593,11 @@ cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const
   p.mt = (int)((M + kGemmBM - 1) / kGemmBM);
   p.nt = (int)((N + BN - 1) / BN);
   p.nkb = (int)((K + kGemmBK - 1) / kGemmBK);
+  p.split = pl.split;
+  p.parts = pl.split > 1 ? static_cast<float*>(workspace) : nullptr;
+  p.counters = pl.split > 1 ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) +
+                                                          align256(split_parts_bytes((int64_t)p.mt * p.nt)))
+                            : nullptr;
   p.acc_i32 = dbg ? dbg->acc_i32 : nullptr;
   p.acc_f32 = dbg ? dbg->acc_f32 : nullptr;
   p.status = status;

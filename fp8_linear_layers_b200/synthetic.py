@@ -51,6 +51,14 @@ LLAMA31_8B_PREFILL = (
     ("down_proj", 4096, 14336),
     ("qkv_proj", 6144, 4096),
 )
+# The same layer with the projections that read one input stored side by side
+# along N (q|k|v and gate|up, the serving layout): four products instead of seven.
+LLAMA31_8B_FUSED = (
+    ("qkv_proj", 6144, 4096),
+    ("o_proj", 4096, 4096),
+    ("gate_up_proj", 28672, 4096),
+    ("down_proj", 4096, 14336),
+)
 
 
 def outlier_count(K: int, fraction: float = 0.01) -> int:

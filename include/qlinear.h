@@ -160,8 +160,20 @@ ql_status qlinear_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq
  * (larger batches: per-token int8 activations, int8 products, int32
  * accumulation); Qwen3 FP8 "Loading" (block scales).
  *   qx, sx     device, from qlinear_quantize_act
- *   workspace  device, qlinear_workspace_bytes(...) bytes (may be 0 / NULL
- *              when that returns 0), same rules as qlinear_gemm_small
+ *   workspace  optional (NULL / 0 bytes: whole tiles).  Block scheme only:
+ *              when the 128x256 output tiles fill at most half the SMs (e.g.
+ *              M = 512 with N = 4096, or N = 1024) and K >= 8192, a
+ *              workspace of at least qlinear_workspace_bytes(...) bytes
+ *              (256-byte aligned, ZERO-FILLED before its first use) lets the
+ *              call split each tile's K blocks in two halves run by two CTAs
+ *              that park their f32 partial sums in it (two 128x256 f32
+ *              tiles per output tile, then one arrival counter per tile);
+ *              the second to arrive adds the two (the same bits in either
+ *              order).  A completed call leaves the
+ *              counters zero again, for any next shape; zero the workspace
+ *              again after a QL_ERR_TIMEOUT.  Two calls in flight at the same
+ *              time must not share it.  Row schemes: qlinear_workspace_bytes
+ *              returns 0.
  *   dbg        optional (NULL): acc_i32 (int8) / acc_f32 (E4M3 row) [M,N] */
 ql_status qlinear_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
                        const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,

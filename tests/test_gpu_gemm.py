@@ -111,6 +111,44 @@ def test_gemm_qwen_block_m512_full_size(cuda, name, N, K):
     _sampled_compare(ql.FP8_E4M3_BLOCK128, 512, N, K, nsamp=1500)
 
 
+@pytest.mark.parametrize("M,N,K", [(200, 384, 8192), (512, 1024, 8192), (512, 4096, 12288)])
+def test_gemm_block_split_k(cuda, M, N, K):
+    """Block scheme with at most half a wave of 256-wide tiles and K >= 8192: with a
+    workspace each tile's K blocks are split in two halves run by two CTAs
+    that meet in f32 partial sums; the outputs stay within the tolerance of
+    the oracle, two calls in a row agree bit for bit (f32 addition commutes,
+    so the order of arrival does not matter), the arrival counters are zero
+    again afterwards, and without a workspace the call runs whole tiles."""
+    scheme = ql.FP8_E4M3_BLOCK128
+    ws_n = ql.workspace_bytes(scheme, M, N, K)
+    tiles = -(-M // 128) * -(-N // 256)
+    slabs = 2 * tiles * 128 * 256 * 4  # two f32 partial tiles per 128 x 256 tile, then the counters
+    assert ws_n > slabs
+    qx, sx, wq, sw = _inputs(scheme, M, N, K, outliers=3)
+    args = (u8_dev(qx), f32_dev(sx), u8_dev(wq), f32_dev(sw))
+    ws = ql.new_workspace(ws_n)
+    y1 = ql.gemm(scheme, *args, workspace=ws)
+    y2 = ql.gemm(scheme, *args, workspace=ws)
+    y0 = ql.gemm(scheme, *args)
+    st, detail = ql.device_status()
+    assert st == 0, detail
+    assert torch.count_nonzero(ws[slabs:]) == 0, "the arrival counters must be left zero"
+    rng = np.random.default_rng(7)
+    pm = np.concatenate([rng.integers(0, M, 2000), np.arange(M), np.full(N, M - 1)])
+    pn = np.concatenate([rng.integers(0, N, 2000), np.full(M, N - 1), np.arange(N)])
+    ry, _, _ = oracle.linear_sampled(scheme, qx, sx, wq, sw, pm, pn, want_acc=True)
+    for tag, y in (("whole tiles", y0), ("split, first call", y1), ("split, second call", y2)):
+        assert_y_close(bits(y)[pm, pn], ry, f"gemm block {M}x{N}x{K} {tag}")
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    # the same through qlinear_forward, whose workspace holds q_x, s_x and then the sums
+    x = synthetic.make_x(M, K, seed=0, tag="gemm-x", outliers=3)
+    wsf = ql.new_workspace(ql.forward_workspace_bytes(scheme, M, N, K))
+    yf = ql.forward(scheme, torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16), args[2], args[3],
+                    workspace=wsf)
+    assert ql.device_status()[0] == 0
+    assert_y_close(bits(yf)[pm, pn], ry, f"forward block {M}x{N}x{K}")
+
+
 def test_forward_dispatches_large_m_through_quant_and_gemm(cuda):
     """qlinear_forward with M > 32: fused per-token quantization into the
     workspace, then the GEMM; compared with the oracle's whole method."""

@@ -95,3 +95,23 @@ def test_gemv_zero_token(cuda):
         y = ql.gemv(scheme, torch.zeros((1, K), dtype=torch.bfloat16, device="cuda"), u8_dev(wq),
                     f32_dev(sw))
         assert torch.count_nonzero(y.float()) == 0
+
+
+@pytest.mark.parametrize("scheme", [ql.W8A8_INT8_ROW, ql.FP8_E4M3_ROW, ql.FP8_E4M3_BLOCK128])
+def test_gemv_side_by_side_weights_equal_separate(cuda, scheme):
+    """Every output row depends only on its own weight row and scale, so the
+    q|k|v weights stored side by side along N give, in one launch, exactly
+    the bits of the three separate products on the same token."""
+    K = 4096
+    parts = [(4096, "q"), (1024, "k"), (1024, "v")]
+    x = bf16_dev(synthetic.make_x(1, K, seed=5, tag="fused-x", outliers=synthetic.outlier_count(K)))
+    wqs, sws, ys = [], [], []
+    for N, tag in parts:
+        w = synthetic.make_w_device(N, K, seed=5, tag="fused-" + tag)
+        wq, sw = ql.quantize_weight(scheme, w)
+        wqs.append(wq)
+        sws.append(sw)
+        ys.append(ql.gemv(scheme, x, wq, sw))
+    y_fused = ql.gemv(scheme, x, torch.cat(wqs, 0).contiguous(), torch.cat(sws, 0).contiguous())
+    assert ql.device_status()[0] == 0
+    assert torch.equal(y_fused.view(torch.int16), torch.cat(ys, 1).view(torch.int16))
