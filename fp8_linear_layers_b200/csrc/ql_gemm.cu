@@ -19,6 +19,9 @@
 //   warps 2..9  epilogue: tcgen05.ld from TMEM, scales, bf16, global stores;
 //               two TMEM accumulators (or per-K-block buffers) let the
 //               epilogue of one tile overlap the MMAs of the next
+// Launched with programmatic dependent launch: the W tiles of the first two
+// stages are requested before the grid dependency wait (they do not depend on
+// the preceding kernel), q_x, s_x and y only after it.
 // Every mbarrier wait is bounded; on a timeout the kernel records it, drains
 // its own copies and MMAs, frees TMEM and returns.
 #include "ql_tc.cuh"
@@ -46,6 +49,7 @@ constexpr int kGemmEpiWarps = 8;
 constexpr int kGemmThreads = 64 + kGemmEpiWarps * 32;
 constexpr int kTmemCols = 512;
 constexpr int kGemmSmemBudget = 200 * 1024;
+constexpr int kGemmEarlyStages = 2;  // W tiles requested before the grid dependency wait
 
 struct GemmParams {
   const float* sx;
@@ -185,6 +189,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   };
 
   if (threadIdx.x == 0) {
+    tc::launch_dependents();  // the next kernel's CTAs may start as SMs free up
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -213,12 +218,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       const uint64_t pol_a = l2_policy_evict_last();   // q_x: re-read by every N tile
       const uint64_t pol_b = l2_policy_evict_first();  // W_q: read by the few M tiles at once
+      // The kernel is launched with programmatic dependent launch.  The W
+      // tiles of the first stages do not depend on the preceding kernel (the
+      // quantization that writes q_x and s_x): they are requested before the
+      // grid dependency wait, the q_x tiles that complete those stages after
+      // it.  Only two stages go out early: more would queue the preceding
+      // kernel's own loads behind this kernel's weight reads.
+      uint32_t pre = 0;
+      for_each_item([&](int t, int lo, int hi) -> bool {
+        const int n0 = (t / p.mt) * BN;
+        for (int kb = lo; kb < hi && pre < (uint32_t)kGemmEarlyStages; ++kb, ++pre) {
+          mbar_arrive_expect_tx(&full[pre], Cfg::kStage);
+          tc::tma_load_2d(ring + pre * Cfg::kStage + Cfg::kStageA, &tmB, kb * kGemmBK, n0, &full[pre], pol_b);
+        }
+        return pre < (uint32_t)kGemmEarlyStages;
+      });
+      tc::grid_dependency_wait();
       uint32_t it = 0;
       bool ok = true;
       for_each_item([&](int t, int lo, int hi) -> bool {
         const int m0 = (t % p.mt) * kGemmBM, n0 = (t / p.mt) * BN;
         for (int kb = lo; kb < hi; ++kb, ++it) {
           const int s = it % kStages;
+          if (it < pre) {  // its W tile is on the way: the q_x tile completes the stage
+            tc::tma_load_2d(ring + s * Cfg::kStage, &tmA, kb * kGemmBK, m0, &full[s], pol_a);
+            continue;
+          }
           if (it >= (uint32_t)kStages &&
               !mbar_wait_bounded(&empty[s], ((it / kStages) - 1) & 1, abort_flag)) {
             ok = false;
@@ -306,6 +331,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int h = ew >> 2;    // which half of the tile's columns
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const int KB = p.K / 128;
+    tc::grid_dependency_wait();  // s_x (and y's previous readers) belong to the preceding kernels
     uint32_t jt = 0;
     bool ok = true;
     for_each_item([&](int t, int lo, int hi) -> bool {
@@ -570,8 +596,17 @@ static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, cons
   cudaError_t e = ensure_smem<gemm_kernel<S, BN>>(Cfg::kSmem);
   if (e != cudaSuccess) return e;
   const int grid = (int)std::min<int64_t>((int64_t)p.mt * p.nt * p.split, sms);
-  gemm_kernel<S, BN><<<grid, kGemmThreads, Cfg::kSmem, st>>>(a, b, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<S, BN>, a, b, p);
 }
 
 cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,

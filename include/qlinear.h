@@ -52,6 +52,12 @@
  *     block scheme, K <= 133144 for int8 (int32 range of K * 127^2) and
  *     K < 131072 for E4M3; M >= 1 with no upper limit except int32 indexing
  *     (M * K and M * N below 2^31).
+ *   - The products and the activation quantization are launched with
+ *     programmatic dependent launch: a call's kernel may start while the
+ *     previous kernel on the stream is finishing.  It reads W_q (and, in the
+ *     GEMV, s_w) before it waits for that kernel, and everything else after.
+ *     So W_q and s_w must not be written by work still in flight on the same
+ *     stream (weights are written once, before the projections run).
  *   - Kernels that wait on a barrier wait a bounded time; if a wait gives up
  *     the kernel records QL_ERR_TIMEOUT in a device status word and returns
  *     without finishing its output.  qlinear_get_device_status reads it.
