@@ -17,7 +17,8 @@
 //  * activation quantization runs first as its own short kernel writing q_x
 //    and s_x into the workspace; this kernel is launched with programmatic
 //    dependent launch, starts its weight loads at once and waits for the
-//    quantized tokens only before loading them.
+//    quantized tokens only before loading them; it releases the next kernel
+//    on the stream as soon as its own CTAs have started.
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2..5
 // epilogue (one TMEM lane = one weight row per thread).  Every mbarrier wait is
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   const int nkb = p.nkb;
 
   if (threadIdx.x == 0) {
+    tc::launch_dependents();  // the next kernel's CTAs may start as SMs free up
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
