@@ -432,6 +432,23 @@ def _oracle_items(wl: Workload, rows_cap: int):
     return items
 
 
+def sample_rows_text(wl: Workload, rows_cap: int) -> str:
+    """The output rows the oracle sample covers: the first rows_cap of each
+    product, capped at the product's N (whole 128-row blocks for the block scheme)."""
+    counts = []
+    for p in wl.products:
+        rows = min(p.N, rows_cap)
+        if p.scheme == FP8B:
+            rows = max(128, rows // 128 * 128)
+        counts.append(rows)
+    if len(counts) == 1:
+        return f"first {counts[0]} output rows of the workload's one product"
+    if len(set(counts)) == 1:
+        return f"first {counts[0]} output rows of each of the {len(counts)} products"
+    return (f"first min(N, {rows_cap}) output rows of each of the {len(counts)} products "
+            f"({sum(counts)} rows in all)")
+
+
 def oracle_sample(wl: Workload, budget_s: float, rows_cap: int):
     """The CPU oracle (whole method from bf16 X) on the first rows_cap output
     rows of every product of the workload, repeated for about budget_s.
@@ -484,7 +501,7 @@ def run_reference(args):
     scale = 1e9 if wl.unit == "GB/s" else 1e12
     value = step_amount * args.steps / dt / scale
     full = sum(wl.amount(p) for p in wl.products)
-    sample = (f"first {rows} output rows of each of the workload's {len(items)} products, "
+    sample = (f"{sample_rows_text(wl, rows)}, "
               f"{100 * step_amount / full:.3g}% of a full step, per step; single thread")
     line = base_line(wl, args, args.gpus)
     line.update({"value": value, "impl": "reference", "ms_per_step": dt / args.steps * 1e3,
@@ -599,7 +616,7 @@ def main():
         rows = pick_rows(wl, min(args.cpu_seconds, 4.0))
         v, secs, passes, per_pass = oracle_sample(wl, args.cpu_seconds, rows)
         cpu = {"value": round(v, 6), "unit": wl.unit, "cores": 1, "kind": "oracle",
-               "sample": f"first {rows} output rows of each of the {len(wl.products)} products "
+               "sample": f"{sample_rows_text(wl, rows)} "
                          f"({100 * per_pass / run.step_amount:.3g}% of a step) x {passes} passes, "
                          f"{secs:.1f} s, single thread"}
 
