@@ -16,6 +16,8 @@ page passage it follows:
   E4M3 activations per token (dynamic, symmetric).
 * "Qwen3 8B FP8" model page, intro and "Loading": a multiplying scale for each
   128x128 weight block, activations quantized in groups of 128 along K.
+* The same pages' "Against bf16" sections: a loader option that never rounds
+  the input (weight-only products, ``linear_weight_only``).
 
 Every function has pins in ``tests/test_oracle_*.py`` that do not go through
 the oracle's own formulas (brute force, closed forms, library routines).
@@ -72,13 +74,15 @@ def lib() -> ctypes.CDLL:
                                             i64p, i64p, i64, u16p, i32p, f64p]
         L.oracle_linear_rows.argtypes = [ctypes.c_int, u8p, f32p, u8p, f32p, i64, i64, i64, i64,
                                          i64, u16p, i32p, f64p]
+        L.oracle_linear_wo_rows.argtypes = [ctypes.c_int, u16p, u8p, f32p, i64, i64, i64, i64,
+                                            i64, u16p, f64p]
         L.oracle_e4m3_encode_n.argtypes = [f32p, i64, u8p]
         L.oracle_f32_to_bf16_n.argtypes = [f32p, i64, u16p]
         L.oracle_int8_round_n.argtypes = [f32p, i64, i32p]
         L.oracle_f64_to_bf16_n.argtypes = [f64p, i64, u16p]
         L.oracle_rounding_is_nearest.restype = ctypes.c_int
         for name in ("oracle_quantize_weight", "oracle_quantize_act", "oracle_linear",
-                     "oracle_linear_sampled", "oracle_linear_rows"):
+                     "oracle_linear_sampled", "oracle_linear_rows", "oracle_linear_wo_rows"):
             getattr(L, name).restype = ctypes.c_int
         if not L.oracle_rounding_is_nearest():
             raise RuntimeError("oracle: FPU is not rounding to nearest")
@@ -248,6 +252,30 @@ def linear_rows(scheme: int, qx, sx, wq, sw, n0: int, n1: int):
                                 _p(y, ctypes.c_uint16), None, None):
         raise ValueError("oracle_linear_rows: bad shape")
     return y
+
+
+def linear_weight_only(scheme: int, x_bf16, wq, sw, n0: int = 0, n1: int | None = None,
+                       want_acc: bool = False):
+    """Weight-only ("equivalent" numerics, W8A16 / FP8 weight-only) product:
+    X stays bf16, each weight is its code times its row or block scale, the
+    sum is taken in f64 and rounded once -> y [M, n1-n0] bf16 bits.  The
+    loader option that never rounds the input ("Llama 3.1 8B Instruct W8A8",
+    "Against bf16"; "Qwen3 8B FP8", "Against bf16") and the W8A16 contrast in
+    the W8A8 model page's "Context".  With want_acc also returns the f64 value
+    before the final rounding."""
+    x = _u16(x_bf16)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    sw = np.ascontiguousarray(sw, np.float32)
+    M, K = x.shape
+    N = wq.shape[0]
+    n1 = N if n1 is None else n1
+    y = np.empty((M, n1 - n0), np.uint16)
+    acc = np.empty((M, n1 - n0), np.float64) if want_acc else None
+    if lib().oracle_linear_wo_rows(scheme, _p(x, ctypes.c_uint16), _p(wq, ctypes.c_uint8),
+                                   _p(sw, ctypes.c_float), M, N, K, n0, n1,
+                                   _p(y, ctypes.c_uint16), _p(acc, ctypes.c_double)):
+        raise ValueError("oracle_linear_wo_rows: bad shape")
+    return (y, acc) if want_acc else y
 
 
 def forward(scheme: int, x_bf16, wq, sw):

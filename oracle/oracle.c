@@ -35,6 +35,11 @@
  *  - row-scheme epilogue: y = bf16( ((float)acc * s_x[m]) * s_w[n] ), f32
  *    left to right; block scheme: y = bf16( sum_kb P_kb * s_x[m,kb] *
  *    s_w[n/128,kb] ) with P_kb exact and the sum in f64, rounded once.
+ *  - weight-only ("equivalent") product: the activations are not rounded at
+ *    all; each weight is dequantized (code x its row or block scale, exact in
+ *    f64), multiplied by the bf16 activation (exact in f64), summed in f64 and
+ *    rounded once to bf16.  Only that f64 sum rounds: its error is at most
+ *    (K-1) 2^-53 sum_k |x w|.
  */
 #include <fenv.h>
 #include <math.h>
@@ -358,6 +363,59 @@ int oracle_forward(int scheme, const uint16_t* x, const uint8_t* wq, const float
                    int64_t N, int64_t K, uint8_t* qx, float* sx, uint16_t* y) {
   if (oracle_quantize_act(scheme, x, M, K, qx, sx)) return -1;
   return oracle_linear(scheme, qx, sx, wq, sw, M, N, K, y, 0, 0);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Weight-only products ("equivalent" numerics)                             */
+/* ------------------------------------------------------------------------ */
+
+/* The pages' loader option numerics="equivalent" never rounds the input
+ * ("Llama 3.1 8B Instruct W8A8", "Against bf16"; "Qwen3 8B FP8", "Against
+ * bf16"), and the W8A8 model page's "Context" contrasts W8A8 with W8A16,
+ * which quantizes only the weights and keeps computing in bf16.  So here X
+ * stays bf16 and only W is quantized:
+ *   y[m,n] = bf16( sum_k x[m,k] * (q_w[n,k] * s_w) ),
+ * s_w = s_w[n] (row schemes) or s_w[n/128, k/128] (block scheme).
+ * The dequantized weight needs at most 24 + 4 significant bits (int8 codes
+ * have 7, E4M3 4, scales 24) and its product with a bf16 (8 bits) is exact in
+ * f64; the sum over k is the one f64 rounding, then one rounding to bf16. */
+static double weight_value(int scheme, const uint8_t* wq, const float* sw, int64_t N, int64_t K,
+                           int64_t n, int64_t k) {
+  uint8_t c = wq[n * K + k];
+  double code = (scheme == ORACLE_INT8_ROW) ? (double)(int8_t)c : oracle_e4m3_decode(c);
+  double s;
+  if (scheme == ORACLE_FP8_BLOCK)
+    s = MUTANT(14) ? (double)sw[(k / 128) * (N / 128) + n / 128] : (double)sw[(n / 128) * (K / 128) + k / 128];
+  else
+    s = (double)sw[n];
+  return MUTANT(13) ? code : code * s;
+}
+
+static uint16_t linear_wo_one(int scheme, const uint16_t* x, const uint8_t* wq, const float* sw,
+                              int64_t N, int64_t K, int64_t m, int64_t n, double* acc_f64) {
+  double y = 0.0;
+  for (int64_t k = MUTANT(15) ? 1 : 0; k < K; ++k)
+    y += (double)oracle_bf16_to_f32(x[m * K + k]) * weight_value(scheme, wq, sw, N, K, n, k);
+  if (acc_f64) *acc_f64 = y;
+  return oracle_f64_to_bf16(y);
+}
+
+/* Output columns [n0, n1) of the weight-only product: x bf16 [M,K], wq [N,K],
+ * sw as for the quantized product; y and acc_f64 (the f64 value before the
+ * final rounding, may be NULL) are [M, n1-n0]. */
+int oracle_linear_wo_rows(int scheme, const uint16_t* x, const uint8_t* wq, const float* sw,
+                          int64_t M, int64_t N, int64_t K, int64_t n0, int64_t n1, uint16_t* y,
+                          double* acc_f64) {
+  if (M < 0 || N <= 0 || K <= 0 || scheme < 0 || scheme > 2) return -1;
+  if (scheme == ORACLE_FP8_BLOCK && (N % 128 || K % 128)) return -1;
+  if (n0 < 0 || n1 > N || n0 > n1) return -1;
+  int64_t W = n1 - n0;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = n0; n < n1; ++n) {
+      int64_t o = m * W + (n - n0);
+      y[o] = linear_wo_one(scheme, x, wq, sw, N, K, m, n, acc_f64 ? acc_f64 + o : 0);
+    }
+  return 0;
 }
 
 /* Bulk forms of the codecs, for sweeps over many values. */

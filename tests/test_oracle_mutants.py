@@ -14,7 +14,8 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
-PINS = ["tests/test_oracle_codecs.py", "tests/test_oracle_quant.py", "tests/test_oracle_linear.py"]
+PINS = ["tests/test_oracle_codecs.py", "tests/test_oracle_quant.py", "tests/test_oracle_linear.py",
+        "tests/test_oracle_weight_only.py"]
 
 MUTANTS = {
     1: "f32->bf16 truncates instead of rounding",
@@ -29,6 +30,9 @@ MUTANTS = {
     10: "block weight-scale index transposed",
     11: "block weight scale from one element, not the block max",
     12: "E4M3 row product drops the last input channel",
+    13: "weight-only product drops the weight scale",
+    14: "weight-only block weight-scale index transposed",
+    15: "weight-only product drops the first input channel",
 }
 
 
