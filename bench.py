@@ -15,6 +15,8 @@ Other workloads (``--workload``), same JSON line:
   qwen-decode   FP8 128x128 block, M = 1 x the 7 Qwen3-8B shapes: GB/s
   qwen-small    FP8 block, M = 32 x the Qwen shapes: GB/s
   qwen-prefill  FP8 block, M = 512 x the Qwen shapes: TOPS
+  decode-wo     the decode layer as weight-only products (x not rounded; int8
+                and FP8 per-row weights): 14 weight-only GEMVs, GB/s
 
 Legs of the line:
   value     device time of K steps, each one CUDA-graph replay of the step's
@@ -66,6 +68,7 @@ class Product:
     N: int
     K: int
     outliers: int
+    wo: bool = False  # weight-only product (activations not rounded)
 
 
 @dataclass
@@ -81,6 +84,8 @@ class Workload:
 
     @property
     def kernel(self):
+        if self.products[0].wo:
+            return "ql::gemv_kernel (weight-only)"
         M = self.products[0].M
         return "ql::gemv_kernel" if M == 1 else ("ql::gemm_small_kernel" if M <= 32 else "ql::gemm_kernel")
 
@@ -122,6 +127,10 @@ def workloads():
     w["kproj"] = Workload(
         "kproj", "W8A8 int8 k_proj shape: X [8, 4096] with 8 outlier channels, W [1024, 4096]",
         "GB/s", [Product("k_proj", INT8, 8, 1024, 4096, 8)])
+    w["decode-wo"] = Workload(
+        "decode-wo", "weight-only decode GEMV M=1 (activations kept bf16, \"equivalent\" numerics): one "
+        "Llama-3.1-8B layer's 7 projections with int8 and with FP8 E4M3 per-row weights", "GB/s",
+        [Product(n, s, 1, N, K, oc(K), wo=True) for n, N, K in S.LLAMA31_8B for s in (INT8, FP8R)])
     w["qwen-decode"] = Workload(
         "qwen-decode", "Qwen3-8B FP8 128x128-block projections at M=1 (7 shapes)", "GB/s",
         [Product(n, FP8B, 1, N, K, 0) for n, N, K in S.QWEN3_8B])
@@ -142,7 +151,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["qlinear", "reference"], default="qlinear")
     ap.add_argument("--workload", default="decode",
                     choices=["decode", "decode-fused", "prefill", "small", "kproj", "qwen-decode",
-                             "qwen-small", "qwen-prefill"])
+                             "qwen-small", "qwen-prefill", "decode-wo"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -248,10 +257,12 @@ L2_BYTES = 126e6
 # DRAM bytes per launch of the dominant kernel from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum), with the hash of the kernel sources it was taken on: when the
 # sources differ the figure no longer describes the kernel and the line reports null.
-KERNEL_SOURCES = {"ql::gemv_kernel": ["ql_gemv.cu", "ql_common.cuh", "ql_tc.cuh", "ql_internal.h"]}
+_GEMV_SOURCES = ["ql_gemv.cu", "ql_common.cuh", "ql_tc.cuh", "ql_internal.h"]
+KERNEL_SOURCES = {"ql::gemv_kernel": _GEMV_SOURCES, "ql::gemv_kernel (weight-only)": _GEMV_SOURCES}
 TRAFFIC = {
     # workload: (bytes per launch, kernel source hash, summary file)
-    "decode": (31237029, "a3bcad88a4eafd29", "profiles/gemv_decode_dram.md"),
+    "decode": (31236974, "233ea157dd920e9f", "profiles/gemv_decode_dram.md"),
+    "decode-wo": (31224887, "233ea157dd920e9f", "profiles/gemv_decode_weight_only_dram.md"),
 }
 
 
@@ -314,11 +325,17 @@ class Runner:
     def _w(self, i, t):
         return i["wqs"][t % len(i["wqs"])]
 
+    def _forward(self, i, x, wq, sw, y):
+        p = i["p"]
+        if p.wo:
+            self.ql.gemv_weight_only(p.scheme, x, wq, sw, y=y)
+        else:
+            self.ql.forward(p.scheme, x, wq, sw, workspace=i["ws"], y=y)
+
     def step(self, t):
-        ql = self.ql
         for i in self.items:
             wq, sw = self._w(i, t)
-            ql.forward(i["p"].scheme, i["xs"][t], wq, sw, workspace=i["ws"], y=i["ys"][t])
+            self._forward(i, i["xs"][t], wq, sw, i["ys"][t])
 
     def dominant(self, t):
         """Launches of the dominant kernel alone (the product on quantized inputs)."""
@@ -326,7 +343,9 @@ class Runner:
         for i in self.items:
             p = i["p"]
             wq, sw = self._w(i, t)
-            if p.M == 1:
+            if p.wo:
+                ql.gemv_weight_only(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
+            elif p.M == 1:
                 ql.gemv(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
             elif p.M <= 32:
                 ql.gemm_small(p.scheme, i["xs"][t], wq, sw, i["ws"], y=i["ys"][t])
@@ -368,7 +387,7 @@ class Runner:
         def body(c):
             for i, xv, yv in views:
                 wq, sw = self._w(i, c)
-                ql.forward(i["p"].scheme, xv, wq, sw, workspace=i["ws"], y=yv)
+                self._forward(i, xv, wq, sw, yv)
 
         with torch.cuda.stream(stream):
             body(0)
@@ -428,8 +447,14 @@ def _oracle_items(wl: Workload, rows_cap: int):
         w = synthetic.make_w(rows, p.K, seed=0, tag=f"oracle.{p.name}")
         x = synthetic.make_x(p.M, p.K, seed=0, tag=f"oracle.{p.name}.x", outliers=p.outliers)
         wq, sw = oracle.quantize_weight(p.scheme, w)
-        items.append((p.scheme, x, wq, sw, wl.amount(Product(p.name, p.scheme, p.M, rows, p.K, 0))))
+        items.append((p.scheme, x, wq, sw, wl.amount(Product(p.name, p.scheme, p.M, rows, p.K, 0)),
+                      p.wo))
     return items
+
+
+def _oracle_run(scheme, x, wq, sw, wo):
+    import oracle
+    return oracle.linear_weight_only(scheme, x, wq, sw) if wo else oracle.forward(scheme, x, wq, sw)
 
 
 def sample_rows_text(wl: Workload, rows_cap: int) -> str:
@@ -459,8 +484,8 @@ def oracle_sample(wl: Workload, budget_s: float, rows_cap: int):
     done, t_used, passes = 0.0, 0.0, 0
     while t_used < budget_s or passes == 0:
         t0 = time.perf_counter()
-        for scheme, x, wq, sw, amt in items:
-            oracle.forward(scheme, x, wq, sw)
+        for scheme, x, wq, sw, amt, wo in items:
+            _oracle_run(scheme, x, wq, sw, wo)
             done += amt
         t_used += time.perf_counter() - t0
         passes += 1
@@ -477,7 +502,8 @@ def pick_rows(wl: Workload, seconds: float) -> int:
 def base_line(wl, args, world):
     return {"metric": METRIC, "unit": wl.unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "s8*s8->s32 (W8A8), e4m3*e4m3->f32 (FP8)",
+            "dtype": ("bf16 x (int8|e4m3 weights as f16) -> f32 (weight-only)" if wl.products[0].wo
+                      else "s8*s8->s32 (W8A8), e4m3*e4m3->f32 (FP8)"),
             "data": "synthetic (seeded N(0,1) activations with outlier channels x20; N(0,0.02) weights)"}
 
 
@@ -491,12 +517,12 @@ def run_reference(args):
     items = _oracle_items(wl, rows)
     step_amount = sum(i[4] for i in items)
     for _ in range(args.warmup):
-        for scheme, x, wq, sw, _ in items:
-            oracle.forward(scheme, x, wq, sw)
+        for scheme, x, wq, sw, _, wo in items:
+            _oracle_run(scheme, x, wq, sw, wo)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        for scheme, x, wq, sw, _ in items:
-            oracle.forward(scheme, x, wq, sw)
+        for scheme, x, wq, sw, _, wo in items:
+            _oracle_run(scheme, x, wq, sw, wo)
     dt = time.perf_counter() - t0
     scale = 1e9 if wl.unit == "GB/s" else 1e12
     value = step_amount * args.steps / dt / scale
@@ -505,7 +531,8 @@ def run_reference(args):
               f"{100 * step_amount / full:.3g}% of a full step, per step; single thread")
     line = base_line(wl, args, args.gpus)
     line.update({"value": value, "impl": "reference", "ms_per_step": dt / args.steps * 1e3,
-                 "dtype": "s8*s8->s32 (int8), e4m3*e4m3 exact (int64 fixed point)",
+                 "dtype": ("f64 sums of exact bf16 x dequantized-weight products" if wl.products[0].wo
+                           else "s8*s8->s32 (int8), e4m3*e4m3 exact (int64 fixed point)"),
                  "config": {**workload_config(wl), "parallelism": f"replicas x{args.gpus}",
                             "note": "CPU oracle, the plain definition, on a row sample per step"},
                  "cpu_baseline": {"value": value, "unit": wl.unit, "cores": 1, "kind": "oracle",

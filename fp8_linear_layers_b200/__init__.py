@@ -39,7 +39,7 @@ STATUS = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED_SHAPE", 3:
 EXPORTS = ("qlinear_quantize_weight", "qlinear_quantize_act", "qlinear_gemv", "qlinear_gemm_small",
            "qlinear_gemm", "qlinear_forward", "qlinear_workspace_bytes",
            "qlinear_forward_workspace_bytes", "qlinear_get_device_status", "qlinear_status_string",
-           "qlinear_last_cuda_error", "qlinear_gemm_small_noalloc")
+           "qlinear_last_cuda_error", "qlinear_gemm_small_noalloc", "qlinear_gemv_weight_only")
 
 
 class QLinearError(RuntimeError):
@@ -84,6 +84,7 @@ def lib() -> ctypes.CDLL:
         L.qlinear_quantize_weight.argtypes = [i32, vp, i64, i64, vp, vp, vp]
         L.qlinear_quantize_act.argtypes = [i32, vp, i64, i64, vp, vp, vp]
         L.qlinear_gemv.argtypes = [i32, vp, vp, vp, i64, i64, vp, vp, vp]
+        L.qlinear_gemv_weight_only.argtypes = [i32, vp, vp, vp, i64, i64, vp, vp]
         L.qlinear_gemm_small.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp, vp]
         L.qlinear_gemm.argtypes = [i32, vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp, vp]
         L.qlinear_forward.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]
@@ -98,7 +99,8 @@ def lib() -> ctypes.CDLL:
         L.qlinear_last_cuda_error.restype = ctypes.c_char_p
         for name in ("qlinear_quantize_weight", "qlinear_quantize_act", "qlinear_gemv",
                      "qlinear_gemm_small", "qlinear_gemm", "qlinear_forward",
-                     "qlinear_get_device_status", "qlinear_gemm_small_noalloc"):
+                     "qlinear_get_device_status", "qlinear_gemm_small_noalloc",
+                     "qlinear_gemv_weight_only"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -171,6 +173,23 @@ def gemv(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor, y=Non
     _check(lib().qlinear_gemv(scheme, _dev(x, torch.bfloat16, "x"), _dev(wq, torch.uint8, "wq"),
                               _dev(sw, torch.float32, "sw"), N, K, _dev(y, torch.bfloat16, "y"),
                               debug._c() if debug else None, _stream(stream)), "qlinear_gemv")
+    return y
+
+
+def gemv_weight_only(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor, y=None,
+                     stream=None) -> torch.Tensor:
+    """M = 1 weight-only product ("equivalent" numerics, W8A16 / FP8 weight-only):
+    x bf16 [1,K] (or [K]) is not rounded -> y bf16 [1,N]."""
+    K = x.shape[-1]
+    N = wq.shape[0]
+    if x.numel() != K:
+        raise ValueError("gemv_weight_only takes a single token")
+    if y is None:
+        y = torch.empty((1, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().qlinear_gemv_weight_only(scheme, _dev(x, torch.bfloat16, "x"),
+                                          _dev(wq, torch.uint8, "wq"), _dev(sw, torch.float32, "sw"),
+                                          N, K, _dev(y, torch.bfloat16, "y"), _stream(stream)),
+           "qlinear_gemv_weight_only")
     return y
 
 

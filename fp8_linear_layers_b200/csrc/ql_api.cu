@@ -167,6 +167,24 @@ ql_status qlinear_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, cons
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemv");
 }
 
+ql_status qlinear_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const void* wq,
+                                   const float* sw, int64_t N, int64_t K, uint16_t* y,
+                                   void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_n(scheme, N, K));
+  if (K > ql::gemv_weight_only_max_k()) return QL_ERR_UNSUPPORTED_SHAPE;
+  QL_TRY(need(x));
+  QL_TRY(need(wq));
+  QL_TRY(need(sw));
+  QL_TRY(need(y));
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  cudaError_t e = ql::launch_gemv_weight_only(scheme, x, wq, sw, N, K, y, d.sms, d.status,
+                                              static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemv_weight_only");
+}
+
 ql_status qlinear_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
                              int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
                              size_t ws_bytes, const ql_debug* dbg, void* stream) {

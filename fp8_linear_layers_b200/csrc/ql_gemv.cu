@@ -39,6 +39,10 @@
 //    fixed order, applies the scales, writes y and releases the stage.
 //  * Every wait is bounded; a warp that gives up raises a CTA abort flag that
 //    every other wait checks, so all roles leave without further barriers.
+//  * Weight-only variant (kWO, the pages' "equivalent" numerics that never
+//    round the input): the same weight stream and MMA mapping with x staged
+//    as f16 (scaled by an exact power of two) instead of codes, and int8
+//    weights converted exactly to f16 for the f16 MMAs; sums in f32.
 #include <type_traits>
 
 #include "ql_common.cuh"
@@ -57,6 +61,7 @@ constexpr int kGemvSmemBudget = 200 * 1024;     // one CTA per SM
 constexpr int kGemvMaxK = 32768;
 constexpr int64_t kGemvMaxK2 = 16384;           // two tokens: units of at most 64 windows
 constexpr int64_t kGemvMaxK4 = 8192;            // three or four tokens: stages of 8 rows
+constexpr int64_t kGemvMaxKWO = 16384;          // weight-only: 2K bytes of staged x beside the ring
 constexpr int kGemvUnits = 16;                  // units per stage (the MMA's 16 A rows)
 constexpr int kGemvSwCache = 2048;              // row scales kept in shared memory
 constexpr uint32_t kBarConsumers = 1;           // named barrier of the consumer warps
@@ -80,15 +85,16 @@ struct GemvSmemLayout {
   int ring, qx, sx, swc, part, bars, flags, total;
 };
 
-// Shared-memory carve-up; `sw_floats` is the number of weight scales cached.
+// Shared-memory carve-up; `sw_floats` is the number of weight scales cached,
+// `xelem` the bytes per staged x element (1: codes; 2: f16 for weight-only).
 __host__ __device__ inline GemvSmemLayout gemv_layout(int64_t K, int stage_bytes, int stages,
-                                                      int sw_floats, int M = 1) {
+                                                      int sw_floats, int M = 1, int xelem = 1) {
   GemvSmemLayout L;
   int off = 0;
   L.ring = off;
   off += stages * stage_bytes;
-  L.qx = off;  // M rows of K codes, each padded to whole 128-byte blocks
-  off += M * (int)((K + 127) / 128) * 128;
+  L.qx = off;  // M rows of K codes (or f16 values), each padded to whole 128-element blocks
+  off += M * (int)((K + 127) / 128) * 128 * xelem;
   L.sx = off;
   off += (int)((M * (K / 128 + 1) + 31) / 32) * 128;
   L.swc = off;
@@ -138,12 +144,43 @@ QL_DEVINL void e4m3x16_to_f16(const uint4& v, uint32_t (&h)[8]) {
   }
 }
 
-template <ql_scheme kScheme, int kRs, int kMaxSteps, int kM>
+// a - b on f16x2 (exact for the integers below 2048 used here).
+QL_DEVINL uint32_t sub_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Eight f16x2 registers from 16 int8 codes (byte order kept), exact.  With
+// its sign bit flipped, code c reads as the unsigned byte c + 128; placed
+// under the f16 exponent of 1024 (unit spacing there) it is the f16 value
+// 1024 + c + 128, and subtracting 1152 leaves c.
+QL_DEVINL void s8x16_to_f16(const uint4& v, uint32_t (&h)[8]) {
+  const uint32_t w[4] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u, v.z ^ 0x80808080u,
+                         v.w ^ 0x80808080u};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    h[2 * q] = sub_f16x2(__byte_perm(w[q], 0x64646464u, 0x4140), 0x64806480u);
+    h[2 * q + 1] = sub_f16x2(__byte_perm(w[q], 0x64646464u, 0x4342), 0x64806480u);
+  }
+}
+
+// Two f32 -> f16x2 (lo in bits [15:0]), round to nearest even.
+QL_DEVINL uint32_t f32x2_to_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// kWO: weight-only product (x is not quantized; see the weight-only prologue).
+template <ql_scheme kScheme, int kRs, int kMaxSteps, int kM, bool kWO = false>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams p) {
   // kM tokens x kQ = 8 / kRs segment classes must fit the 8 B columns
   static_assert(kM == 1 || (kM * (8 / kRs) <= 8 && kRs >= 2), "tokens do not fit the B columns");
+  static_assert(!kWO || kM == 1, "the weight-only product takes one token");
   constexpr bool kInt8 = kScheme == QL_W8A8_INT8_ROW;
   constexpr bool kBlock = kScheme == QL_FP8_E4M3_BLOCK128;
+  constexpr bool kIntAcc = kInt8 && !kWO;  // exact int32 sums on s8 MMAs
 
   extern __shared__ __align__(1024) uint8_t smem[];
   const int64_t N = p.N, K = p.K;
@@ -156,7 +193,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   const int64_t sw_count = kBlock ? (((row_end - 1) >> 7) - (row_begin >> 7) + 1) * KB : row_end - row_begin;
   const int sw_cached = (int)min(sw_count, (int64_t)kGemvSwCache);
   const int nst = p.stages;
-  const GemvSmemLayout L = gemv_layout(K, p.stage_bytes, nst, kGemvSwCache, kM);
+  const GemvSmemLayout L = gemv_layout(K, p.stage_bytes, nst, kGemvSwCache, kM, kWO ? 2 : 1);
   const int64_t xstride = (K + 127) / 128 * 128;  // bytes between the tokens' codes
   uint8_t* ring = smem + L.ring;
   uint8_t* qx_s = smem + L.qx;
@@ -240,7 +277,61 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   // 1. Fused activation quantization of x [kM, K] into shared memory: one pass
   //    for the absmax (the first kXLoads chunks per thread loaded together),
   //    one for the codes (x is L2-resident by then).
-  if constexpr (kM == 1) {
+  if constexpr (kWO) {
+    // Weight-only: x is not quantized.  The MMAs run on f16, so x is staged
+    // as x * 2^e in f16, e the power of two that puts the token's absmax in
+    // [2^14, 2^15): a bf16 significand (8 bits) fits f16's 11, so every element
+    // within a factor 2^31 of the absmax is carried exactly (smaller ones round
+    // to f16's subnormal spacing).  The products with the f16 weight values
+    // are exact in f32; the epilogue multiplies the sums by 2^-e (exact).
+    const int64_t nchunk8 = K / 8;  // 16-byte chunks of 8 bf16
+    constexpr int kXLoads = 8;
+    const uint4* xg = reinterpret_cast<const uint4*>(p.x);
+    uint4* stash = nst > kEarlyStages && (int64_t)p.stage_bytes >= nchunk8 * 16
+                       ? reinterpret_cast<uint4*>(ring + kEarlyStages * p.stage_bytes)
+                       : nullptr;
+    float a_tok = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kXLoads; ++i) {
+      const int64_t c = tid + (int64_t)i * kGemvConsumers;
+      const uint4 v = c < nchunk8 ? __ldg(xg + c) : make_uint4(0, 0, 0, 0);
+      if (stash && c < nchunk8) stash[c] = v;
+      a_tok = fmaxf(a_tok, absmax_chunk8(v));
+    }
+    for (int64_t c = tid + (int64_t)kXLoads * kGemvConsumers; c < nchunk8; c += kGemvConsumers) {
+      const uint4 v = __ldg(xg + c);
+      if (stash) stash[c] = v;
+      a_tok = fmaxf(a_tok, absmax_chunk8(v));
+    }
+    a_tok = warp_max(a_tok);
+    if (lane == 0) blockred[warp] = a_tok;
+    named_bar_sync(kBarConsumers, kGemvConsumers);
+    float a = blockred[0];
+#pragma unroll
+    for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, blockred[w]);
+    // e = 14 - exponent(a), kept within [-113, 126] so that 2^e and 2^-e are
+    // normal f32 (a zero or subnormal absmax takes e = 126)
+    int e2 = 126;
+    const int ea = (int)((__float_as_uint(a) >> 23) & 0xFFu);
+    if (ea != 0) e2 = min(126, 14 - (ea - 127));
+    const float up = __uint_as_float((uint32_t)(127 + e2) << 23);
+    const float down = __uint_as_float((uint32_t)(127 - e2) << 23);
+    for (int i = tid; i < (kBlock ? (int)KB : 1); i += kGemvConsumers) sx_s[i] = down;
+    uint4* xs4 = reinterpret_cast<uint4*>(qx_s);
+#pragma unroll 1
+    for (int64_t c = tid; c < nchunk8; c += kGemvConsumers) {
+      const uint4 v = stash ? stash[c] : __ldg(xg + c);
+      xs4[c] = make_uint4(f32x2_to_f16x2(bf16_lo(v.x) * up, bf16_hi(v.x) * up),
+                          f32x2_to_f16x2(bf16_lo(v.y) * up, bf16_hi(v.y) * up),
+                          f32x2_to_f16x2(bf16_lo(v.z) * up, bf16_hi(v.z) * up),
+                          f32x2_to_f16x2(bf16_lo(v.w) * up, bf16_hi(v.w) * up));
+    }
+    if (stash) fence_proxy_async_smem();
+    // zero the padding of the last 64-element window so it adds nothing
+    for (int64_t b = 2 * K + tid * 16; b < 2 * ((K + 63) / 64 * 64); b += kGemvConsumers * 16)
+      *reinterpret_cast<uint4*>(qx_s + b) = make_uint4(0, 0, 0, 0);
+    named_bar_sync(kBarConsumers, kGemvConsumers);
+  } else if constexpr (kM == 1) {
     const int64_t nchunk8 = K / 8;  // 16-byte chunks of 8 bf16
     constexpr int kXLoads = 8;
     const uint4* xg = reinterpret_cast<const uint4*>(p.x);
@@ -424,7 +515,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     named_bar_sync(kBarConsumers, kGemvConsumers);
   }
   if (tid == 0) mbar_arrive(xready);  // the producer may fill the whole ring now
-  if (blockIdx.x == 0 && (p.dbg.qx || p.dbg.sx)) {
+  if (!kWO && blockIdx.x == 0 && (p.dbg.qx || p.dbg.sx)) {
     // [token, K] codes and [token, groups] scales; rows of K bytes (K % 16 == 0)
     const int ns = kBlock ? (int)KB : 1;
     for (int64_t c = tid; c < (kM == 1 ? 1 : p.M) * (K / 16); c += kGemvConsumers) {
@@ -480,15 +571,30 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   const int64_t ulen = min(seg, K - (int64_t)uq * seg);  // unit bytes inside K
   uint4 xr[kMaxSteps];
   uint32_t vmask = 0;  // steps whose 16 bytes of this lane lie inside the unit
+  if constexpr (!kWO) {
 #pragma unroll
-  for (int s = 0; s < kMaxSteps; ++s) {
-    const int64_t off = (int64_t)((st0 + s) ^ flip) * 64 + t * 16;
-    const bool v = s < nsteps && off < ulen;
-    xr[s] = v ? ld_s128(qx_s + xtok * xstride + (int64_t)uq * seg + off) : make_uint4(0, 0, 0, 0);
-    vmask |= (uint32_t)v << s;
+    for (int s = 0; s < kMaxSteps; ++s) {
+      const int64_t off = (int64_t)((st0 + s) ^ flip) * 64 + t * 16;
+      const bool v = s < nsteps && off < ulen;
+      xr[s] = v ? ld_s128(qx_s + xtok * xstride + (int64_t)uq * seg + off) : make_uint4(0, 0, 0, 0);
+      vmask |= (uint32_t)v << s;
+    }
   }
-  uint32_t xh[kInt8 ? 1 : kMaxSteps][8];  // E4M3 schemes: x fragments as f16
-  if constexpr (!kInt8) {
+  uint32_t xh[kIntAcc ? 1 : kMaxSteps][8];  // f16 MMA schemes: x fragments as f16
+  if constexpr (kWO) {
+    // the lane's 16 staged f16 values at the same K positions (32 bytes)
+#pragma unroll
+    for (int s = 0; s < kMaxSteps; ++s) {
+      const int64_t off = (int64_t)((st0 + s) ^ flip) * 64 + t * 16;
+      const bool v = s < nsteps && off < ulen;
+      const uint8_t* src = qx_s + 2 * ((int64_t)uq * seg + off);
+      const uint4 lo = v ? ld_s128(src) : make_uint4(0, 0, 0, 0);
+      const uint4 hi = v ? ld_s128(src + 16) : make_uint4(0, 0, 0, 0);
+      xh[s][0] = lo.x, xh[s][1] = lo.y, xh[s][2] = lo.z, xh[s][3] = lo.w;
+      xh[s][4] = hi.x, xh[s][5] = hi.y, xh[s][6] = hi.z, xh[s][7] = hi.w;
+      vmask |= (uint32_t)v << s;
+    }
+  } else if constexpr (!kInt8) {
 #pragma unroll
     for (int s = 0; s < kMaxSteps; ++s) e4m3x16_to_f16(xr[s], xh[s]);
   }
@@ -508,13 +614,18 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     const int off = ((st0 + s) ^ flip) * 64;
     const uint4 w0 = (vm0 >> s) & 1u ? ld_s128(wb + off) : make_uint4(0, 0, 0, 0);
     const uint4 w1 = (vm1 >> s) & 1u ? ld_s128(wb + w_half + off) : make_uint4(0, 0, 0, 0);
-    if constexpr (kInt8) {
+    if constexpr (kIntAcc) {
       mma_s8(dd[0], w0.x, w1.x, w0.y, w1.y, xr[s].x, xr[s].y);
       mma_s8(dd[1], w0.z, w1.z, w0.w, w1.w, xr[s].z, xr[s].w);
     } else {
       uint32_t h0[8], h1[8];
-      e4m3x16_to_f16(w0, h0);
-      e4m3x16_to_f16(w1, h1);
+      if constexpr (kInt8) {  // weight-only int8: codes to f16 (exact)
+        s8x16_to_f16(w0, h0);
+        s8x16_to_f16(w1, h1);
+      } else {
+        e4m3x16_to_f16(w0, h0);
+        e4m3x16_to_f16(w1, h1);
+      }
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         mma_f16(dd[q & 1], h0[2 * q], h1[2 * q], h0[2 * q + 1], h1[2 * q + 1], xh[s][2 * q], xh[s][2 * q + 1]);
@@ -548,7 +659,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         k0[a] = e ? d[a >> 1][a & 1][1] : d[a >> 1][a & 1][0];
         k1[a] = e ? d[a >> 1][a & 1][3] : d[a >> 1][a & 1][2];
       }
-      if constexpr (kInt8) {  // carried bit-for-bit through the float slot, summed as int32
+      if constexpr (kIntAcc) {  // carried bit-for-bit through the float slot, summed as int32
         kept0 = __int_as_float((int)(k0[0] + k0[1] + k0[2] + k0[3]));
         kept1 = __int_as_float((int)(k1[0] + k1[1] + k1[2] + k1[3]));
       } else {
@@ -611,12 +722,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 #pragma unroll
         for (int w = (kM == 1 ? wg : 0); w < kGemvWarps; w += (kM == 1 ? 2 : 1)) {
           const float pv = ps[(otok * kGemvWarps + w) * kGemvUnits + u];
-          if constexpr (kInt8)
+          if constexpr (kIntAcc)
             vi += __float_as_int(pv);
           else
             vf += pv;
         }
-        if constexpr (kInt8) {
+        if constexpr (kIntAcc) {
           if (kM == 1) vi += __shfl_xor_sync(0xffffffffu, vi, 16);
 #pragma unroll
           for (int o = 1; o < kQ; o <<= 1) vi += __shfl_xor_sync(0xffffffffu, vi, o);
@@ -635,7 +746,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
             const int64_t si = n - row_begin;
             const float swn = si < sw_cached ? sw_s[si] : __ldg(p.sw + n);
             const float sxt = kM == 1 ? sx_tok : sx_s[otok];
-            if constexpr (kInt8) {
+            if constexpr (kIntAcc) {
               if (p.dbg.acc_i32) p.dbg.acc_i32[o] = vi;
               yv = __fmul_rn(__fmul_rn(__int2float_rn(vi), sxt), swn);
             } else {
@@ -656,10 +767,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 }
 
 int gemv_max_k() { return kGemvMaxK; }
+int gemv_weight_only_max_k() { return (int)kGemvMaxKWO; }
 
-template <ql_scheme S, int kRs, int kSteps, int kM>
+template <ql_scheme S, int kRs, int kSteps, int kM, bool kWO = false>
 static cudaError_t launch_gemv_r(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
-  cudaError_t e = ensure_smem<gemv_kernel<S, kRs, kSteps, kM>>((int)smem);
+  cudaError_t e = ensure_smem<gemv_kernel<S, kRs, kSteps, kM, kWO>>((int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -671,7 +783,7 @@ static cudaError_t launch_gemv_r(const GemvParams& p, int grid, size_t smem, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<S, kRs, kSteps, kM>, p);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<S, kRs, kSteps, kM, kWO>, p);
 }
 
 // Steps per warp: 4 when a unit has at most 32 windows of 64 bytes, else 8.
@@ -694,19 +806,28 @@ static cudaError_t launch_gemv_t(const GemvParams& p, int grid, size_t smem, cud
   }
 }
 
+// Weight-only: one token, the same stage shapes (K <= 16384: at most 32
+// windows per unit, so 4 steps per warp).
+template <ql_scheme S>
+static cudaError_t launch_gemv_wo_t(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
+  if (p.seg_len > 32 * 64) return cudaErrorInvalidValue;
+  switch (p.rows_per_stage / 2) {
+    case 1: return launch_gemv_r<S, 1, 4, 1, true>(p, grid, smem, st);
+    case 2: return launch_gemv_r<S, 2, 4, 1, true>(p, grid, smem, st);
+    case 4: return launch_gemv_r<S, 4, 4, 1, true>(p, grid, smem, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 int gemv_max_k_tokens(int64_t M) {
   return M == 1 ? (int)kGemvMaxK : M == 2 ? (int)kGemvMaxK2 : M <= 4 ? (int)kGemvMaxK4 : 0;
 }
 
-cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
-                        int64_t M, int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg,
-                        int num_sms, DevStatus* status, cudaStream_t st) {
-  if (M < 1 || M > 4 || K > gemv_max_k_tokens(M)) return cudaErrorInvalidValue;
-  GemvParams p;
-  p.x = x;
-  p.wq = static_cast<const uint8_t*>(wq);
-  p.sw = sw;
-  p.y = y;
+// Stage shape, ring depth and grid for M tokens (xelem: bytes per staged x
+// element).  Returns cudaErrorInvalidValue / InvalidConfiguration for shapes
+// the kernel does not take.
+static cudaError_t gemv_setup(GemvParams& p, int64_t M, int64_t N, int64_t K, int xelem,
+                              int num_sms, int* grid, size_t* smem) {
   p.N = N;
   p.K = K;
   p.M = (int)M;
@@ -721,22 +842,60 @@ cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, con
   const int km = M <= 2 ? (int)M : 4;  // the kernel's token count (three tokens pad to four)
   p.rows_per_stage = 2 * rs;
   p.stage_bytes = (int)(((int64_t)p.rows_per_stage * K + 127) / 128 * 128);
-  const int fixed = gemv_layout(K, p.stage_bytes, 0, kGemvSwCache, km).total;
+  const int fixed = gemv_layout(K, p.stage_bytes, 0, kGemvSwCache, km, xelem).total;
   p.stages = (int)std::min<int64_t>(kGemvMaxStages, (kGemvSmemBudget - fixed) / p.stage_bytes);
   if (p.stages < 2) return cudaErrorInvalidConfiguration;
   const int q = 8 / rs;
   p.seg_len = ((K + q - 1) / q + 127) / 128 * 128;
   // the kernel keeps at most 64 windows of 64 bytes per unit
   if (p.seg_len > 64 * 64) return cudaErrorInvalidValue;
+  const int64_t stage_rows_total = (N + p.rows_per_stage - 1) / p.rows_per_stage;
+  *grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms, stage_rows_total));
+  *smem = gemv_layout(K, p.stage_bytes, p.stages, kGemvSwCache, km, xelem).total;
+  return cudaSuccess;
+}
+
+cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
+                        int64_t M, int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg,
+                        int num_sms, DevStatus* status, cudaStream_t st) {
+  if (M < 1 || M > 4 || K > gemv_max_k_tokens(M)) return cudaErrorInvalidValue;
+  GemvParams p;
+  p.x = x;
+  p.wq = static_cast<const uint8_t*>(wq);
+  p.sw = sw;
+  p.y = y;
+  int grid = 0;
+  size_t smem = 0;
+  cudaError_t e = gemv_setup(p, M, N, K, 1, num_sms, &grid, &smem);
+  if (e != cudaSuccess) return e;
   p.dbg = dbg ? *dbg : ql_debug{nullptr, nullptr, nullptr, nullptr};
   p.status = status;
-  const int64_t stage_rows_total = (N + p.rows_per_stage - 1) / p.rows_per_stage;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms, stage_rows_total));
-  const size_t smem = gemv_layout(K, p.stage_bytes, p.stages, kGemvSwCache, km).total;
   switch (scheme) {
     case QL_W8A8_INT8_ROW: return launch_gemv_t<QL_W8A8_INT8_ROW>(p, grid, smem, st);
     case QL_FP8_E4M3_ROW: return launch_gemv_t<QL_FP8_E4M3_ROW>(p, grid, smem, st);
     default: return launch_gemv_t<QL_FP8_E4M3_BLOCK128>(p, grid, smem, st);
+  }
+}
+
+cudaError_t launch_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const void* wq,
+                                    const float* sw, int64_t N, int64_t K, uint16_t* y,
+                                    int num_sms, DevStatus* status, cudaStream_t st) {
+  if (K > kGemvMaxKWO) return cudaErrorInvalidValue;
+  GemvParams p;
+  p.x = x;
+  p.wq = static_cast<const uint8_t*>(wq);
+  p.sw = sw;
+  p.y = y;
+  int grid = 0;
+  size_t smem = 0;
+  cudaError_t e = gemv_setup(p, 1, N, K, 2, num_sms, &grid, &smem);
+  if (e != cudaSuccess) return e;
+  p.dbg = ql_debug{nullptr, nullptr, nullptr, nullptr};
+  p.status = status;
+  switch (scheme) {
+    case QL_W8A8_INT8_ROW: return launch_gemv_wo_t<QL_W8A8_INT8_ROW>(p, grid, smem, st);
+    case QL_FP8_E4M3_ROW: return launch_gemv_wo_t<QL_FP8_E4M3_ROW>(p, grid, smem, st);
+    default: return launch_gemv_wo_t<QL_FP8_E4M3_BLOCK128>(p, grid, smem, st);
   }
 }
 

@@ -48,6 +48,12 @@ int gemv_max_k_tokens(int64_t M);  // largest K the GEMV takes for M tokens (0: 
 cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
                         int64_t M, int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg,
                         int num_sms, DevStatus* status, cudaStream_t st);
+// M = 1 weight-only product: x stays bf16 (staged as exactly scaled f16), W codes
+// dequantized to f16 in registers, f32 sums; K <= gemv_weight_only_max_k().
+int gemv_weight_only_max_k();
+cudaError_t launch_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const void* wq,
+                                    const float* sw, int64_t N, int64_t K, uint16_t* y,
+                                    int num_sms, DevStatus* status, cudaStream_t st);
 
 // Large-M tcgen05 GEMM on pre-quantized activations.
 size_t gemm_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);

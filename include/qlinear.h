@@ -135,6 +135,29 @@ ql_status qlinear_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, i
 ql_status qlinear_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
                        int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg, void* stream);
 
+/* M = 1 weight-only product ("equivalent" numerics: W8A16 / FP8 weight-only):
+ * the activations are not rounded, only the weights are quantized,
+ *   y[n] = bf16_rne( sum_k x[k] * (q_w[n,k] * s_w) ),
+ * s_w = s_w[n] (row schemes) or s_w[n/128, k/128] (block scheme).  Pages: the
+ * W8A8 and Qwen3 FP8 model pages, "Against bf16" (a loader option that never
+ * rounds the input); the W8A8 page's "Context" (W8A16 quantizes only the
+ * weights and keeps computing in bf16).  One kernel streams each weight byte
+ * once, as qlinear_gemv does.
+ *   x    device, bf16 [1,K]
+ *   wq   device, [N,K] codes from qlinear_quantize_weight (or a checkpoint)
+ *   sw   device, the matching weight scales
+ *   y    device, out: bf16 [1,N]
+ * Arithmetic: x is staged as x * 2^e in f16 (e the power of two that puts the
+ * token's absmax in [2^14, 2^15); every element within 2^31 of the absmax is
+ * carried exactly), the codes convert exactly to f16, the products are exact
+ * and summed in f32 on the tensor cores, then scaled by 2^-e and s_w in f32.
+ * Tolerance against the exact value: |y - y_exact| <= 2^-7 |y_exact| + 1e-3.
+ * Errors: argument checks as above; K <= 16384 (else QL_ERR_UNSUPPORTED_SHAPE:
+ * the staged f16 x takes 2K bytes of shared memory beside the weight ring). */
+ql_status qlinear_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const void* wq,
+                                   const float* sw, int64_t N, int64_t K, uint16_t* y,
+                                   void* stream);
+
 /* 1 <= M <= 32 product on the tensor cores (tcgen05, tokens on the MMA N side,
  * weights on the 128-row side, K split across the SMs).  Up to four tokens
  * (K <= 16384 for two, K <= 8192 for three or four) run instead on the

@@ -62,6 +62,14 @@ def test_host_validation_rejects_before_launch(L):
     assert L.qlinear_quantize_act(0, ALIGNED, -1, 64, ALIGNED, ALIGNED, None) == INV
     assert L.qlinear_gemm_small(0, ALIGNED, ALIGNED, ALIGNED, 33, 64, 64, ALIGNED, ALIGNED, 1 << 20,
                                 None, None) == SHAPE
+    # the weight-only GEMV: the same argument rules, and K at most 16384
+    WO = L.qlinear_gemv_weight_only
+    assert WO(7, ALIGNED, ALIGNED, ALIGNED, 64, 64, ALIGNED, None) == INV
+    assert WO(1, None, ALIGNED, ALIGNED, 64, 64, ALIGNED, None) == INV
+    assert WO(1, ALIGNED, ALIGNED + 8, ALIGNED, 64, 64, ALIGNED, None) == MIS
+    assert WO(0, ALIGNED, ALIGNED, ALIGNED, 64, 40, ALIGNED, None) == SHAPE
+    assert WO(2, ALIGNED, ALIGNED, ALIGNED, 100, 256, ALIGNED, None) == SHAPE
+    assert WO(0, ALIGNED, ALIGNED, ALIGNED, 16, 16400, ALIGNED, None) == SHAPE
     # M = 0 is a no-op that succeeds without a device
     assert L.qlinear_quantize_act(0, None, 0, 64, None, None, None) == 0
     assert L.qlinear_forward(0, None, None, None, 0, 64, 64, None, None, 0, None) == 0
