@@ -1,0 +1,95 @@
+"""Host-side logic of bench.py (CPU only): the workloads' algorithmic amounts
+against the shape totals, the oracle sample's description, and the rule that a
+DRAM-traffic figure is reported only for the kernel sources it was taken on."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+LLAMA_WEIGHT_BYTES = 218_103_808  # q/o 4096x4096, k/v 1024x4096, gate/up/down 14336x4096
+QWEN_WEIGHT_BYTES = 192_937_984   # gate/up/down 12288x4096
+
+
+def _weights(wl):
+    return sum(p.N * p.K for p in wl.products)
+
+
+def test_decode_layer_bytes():
+    w = bench.workloads()
+    dec = w["decode"]
+    assert _weights(dec) == 2 * LLAMA_WEIGHT_BYTES  # int8 and FP8 per-row copies
+    # weights + 4N scales + 2K x + 2N y per product
+    extra = sum(4 * p.N + 2 * p.K + 2 * p.N for p in dec.products)
+    assert sum(dec.amount(p) for p in dec.products) == 2 * LLAMA_WEIGHT_BYTES + extra == 436_879_360
+    # the weight-only layer moves the same bytes through the same 14 products
+    wo = w["decode-wo"]
+    assert all(p.wo for p in wo.products) and not any(p.wo for p in dec.products)
+    assert [(p.name, p.scheme, p.N, p.K) for p in wo.products] == \
+        [(p.name, p.scheme, p.N, p.K) for p in dec.products]
+    assert sum(wo.amount(p) for p in wo.products) == 436_879_360
+    # side by side along N: the same weight bytes in 8 products
+    assert _weights(w["decode-fused"]) == 2 * LLAMA_WEIGHT_BYTES
+    assert len(w["decode-fused"].products) == 8
+
+
+def test_qwen_block_layer_bytes_and_scales():
+    w = bench.workloads()
+    q = w["qwen-decode"]
+    assert _weights(q) == QWEN_WEIGHT_BYTES
+    for p in q.products:  # one f32 scale per 128x128 block
+        assert q.amount(p) == p.N * p.K + 4 * (p.N // 128) * (p.K // 128) + 2 * p.K + 2 * p.N
+
+
+def test_prefill_ops():
+    pre = bench.workloads()["prefill"]
+    assert pre.unit == "TOPS" and pre.bound == "tensor"
+    ops = {(p.M, p.name): pre.amount(p) for p in pre.products}
+    assert ops[(512, "gate_proj")] == 2 * 512 * 14336 * 4096  # 60.13 G
+    assert ops[(1024, "down_proj")] == 2 * 1024 * 4096 * 14336
+
+
+def test_workload_kernels_and_bounds():
+    w = bench.workloads()
+    assert w["decode"].kernel == "ql::gemv_kernel" and w["decode"].bound == "hbm"
+    assert w["decode-wo"].kernel == "ql::gemv_kernel (weight-only)"
+    assert w["small"].kernel == "ql::gemm_small_kernel"
+    assert w["qwen-prefill"].kernel == "ql::gemm_kernel"
+
+
+def test_sample_description_caps_rows_at_n():
+    w = bench.workloads()
+    assert bench.sample_rows_text(w["kproj"], 10 ** 6) == \
+        "first 1024 output rows of the workload's one product"
+    assert bench.sample_rows_text(w["decode"], 300) == \
+        "first 300 output rows of each of the 14 products"
+    t = bench.sample_rows_text(w["decode"], 5000)
+    assert t.startswith("first min(N, 5000)") and f"({2 * (4096 + 1024 + 1024 + 4096 + 4096) + 4 * 5000} rows" in t
+    # block scheme: whole 128-row blocks
+    assert bench.sample_rows_text(w["qwen-decode"], 300) == \
+        "first 256 output rows of each of the 7 products"
+
+
+def test_traffic_is_tied_to_kernel_sources(monkeypatch):
+    wl = bench.workloads()["decode"]
+    h = bench.kernel_source_hash(wl.kernel)
+    assert h is not None and len(h) == 16
+    monkeypatch.setitem(bench.TRAFFIC, "decode", (123, h, "profiles/x.md"))
+    assert bench.measured_traffic(wl) == (123, "profiles/x.md")
+    monkeypatch.setitem(bench.TRAFFIC, "decode", (123, "0" * 16, "profiles/x.md"))
+    assert bench.measured_traffic(wl) == (None, None)
+    # a workload without a capture reports null
+    assert bench.measured_traffic(bench.workloads()["small"]) == (None, None)
+
+
+def test_committed_traffic_summaries_exist():
+    for key, (bytes_per_launch, _, path) in bench.TRAFFIC.items():
+        assert os.path.exists(os.path.join(ROOT, path)), path
+        wl = bench.workloads()[key]
+        per_launch = sum(wl.amount(p) for p in wl.products) / len(wl.products)
+        # the recorded DRAM traffic is within 1% of the algorithmic bytes (no re-reads)
+        assert bytes_per_launch == pytest.approx(per_launch, rel=0.01)
