@@ -436,6 +436,45 @@ def timed(torch, stream, graphs, steps):
 
 
 # ------------------------------------------------------------------ CPU oracle
+def _host_bits(torch, t):
+    """bf16 tensor -> uint16 bit patterns on the host."""
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view("uint16")
+
+
+def parity_sample(run, torch, rows: int = 8):
+    """The step's outputs (input copy 0) against the CPU oracle on the first
+    `rows` output rows of every product: the largest absolute and relative
+    error and whether every sampled output is within 2^-7 |y| + 1e-3.  A
+    report beside the throughput; the parity tests are the gate."""
+    import numpy as np
+    import oracle
+    max_abs, max_rel, ok, count = 0.0, 0.0, True, 0
+    for i in run.items:
+        p = i["p"]
+        wq, sw = run._w(i, 0)
+        r = min(rows, p.N)
+        sub = 128 if p.scheme == FP8B else r  # block scales cover 128-row blocks
+        x = _host_bits(torch, i["xs"][0])
+        wq_h = np.ascontiguousarray(wq[:sub].cpu().numpy())
+        sw_h = np.ascontiguousarray((sw[:1] if p.scheme == FP8B else sw[:sub]).cpu().numpy())
+        if p.wo:
+            ref = oracle.linear_weight_only(p.scheme, x, wq_h, sw_h, 0, r)
+        else:
+            qx, sx = oracle.quantize_act(p.scheme, x)
+            ref = oracle.linear_rows(p.scheme, qx, sx, wq_h, sw_h, 0, r)
+        got = _host_bits(torch, i["ys"][0])[:, :r]
+        g, e = oracle.bf16_bits_to_f64(got), oracle.bf16_bits_to_f64(ref)
+        err = np.abs(g - e)
+        max_abs = max(max_abs, float(err.max()))
+        nz = np.abs(e) > 0
+        if nz.any():
+            max_rel = max(max_rel, float((err[nz] / np.abs(e[nz])).max()))
+        ok = ok and bool(np.all(err <= 2.0 ** -7 * np.abs(e) + 1e-3))
+        count += got.size
+    return {"outputs": count, "rows_per_product": rows, "max_abs_err": max_abs,
+            "max_rel_err": max_rel, "within_tolerance": ok, "tolerance": "2^-7 |y_oracle| + 1e-3"}
+
+
 def _oracle_items(wl: Workload, rows_cap: int):
     import oracle
     from fp8_linear_layers_b200 import synthetic
@@ -638,6 +677,17 @@ def main():
     e2e_value = whole_job_value(world, run.step_amount, e2e_steps, e2e_ms, scale)
     del g_e2e
 
+    # ---- the outputs against the oracle on a row sample (rank 0; never fatal)
+    parity = None
+    if rank == 0:
+        try:
+            with torch.cuda.stream(stream):
+                run.step(0)
+            stream.synchronize()
+            parity = parity_sample(run, torch)
+        except Exception as exc:  # the report must not cost the bench line
+            parity = {"error": f"{type(exc).__name__}: {exc}"}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = pick_rows(wl, min(args.cpu_seconds, 4.0))
@@ -661,6 +711,7 @@ def main():
                               f"touched per cycle ({weight_bytes / 1e6:.0f} MB of weights per step); no flush"),
                        "timing": "one CUDA graph replay per step, CUDA events on the launch stream"},
             "roofline": roofline,
+            "parity": parity,
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 1), "unit": wl.unit, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,

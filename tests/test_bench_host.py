@@ -93,3 +93,40 @@ def test_committed_traffic_summaries_exist():
         per_launch = sum(wl.amount(p) for p in wl.products) / len(wl.products)
         # the recorded DRAM traffic is within 1% of the algorithmic bytes (no re-reads)
         assert bytes_per_launch == pytest.approx(per_launch, rel=0.01)
+
+
+class _FakeRun:
+    """CPU stand-in for bench.Runner: items whose outputs come from the oracle."""
+
+    def __init__(self, items):
+        self.items = items
+
+    def _w(self, i, t):
+        return i["wqs"][t % len(i["wqs"])]
+
+
+def _fake_item(scheme, M, N, K, wo):
+    import numpy as np
+    import torch
+    import oracle
+    from fp8_linear_layers_b200 import synthetic
+    x = synthetic.make_x(M, K, seed=2, tag=f"fake.{scheme}.{wo}", outliers=2)
+    w = synthetic.make_w(N, K, seed=2, tag=f"fake.w.{scheme}")
+    wq, sw = oracle.quantize_weight(scheme, w)
+    y = oracle.linear_weight_only(scheme, x, wq, sw) if wo else oracle.forward(scheme, x, wq, sw)
+    t16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    p = bench.Product("fake", scheme, M, N, K, 2, wo=wo)
+    return dict(p=p, xs=[t16(x)], ys=[t16(y)],
+                wqs=[(torch.from_numpy(wq), torch.from_numpy(np.ascontiguousarray(sw)))])
+
+
+def test_parity_sample_against_oracle_outputs():
+    import torch
+    items = [_fake_item(s, M, 256, 256, wo) for s in (0, 1, 2) for M, wo in ((1, False), (3, False), (1, True))]
+    rep = bench.parity_sample(_FakeRun(items), torch, rows=8)
+    assert rep["within_tolerance"] and rep["max_abs_err"] == 0.0
+    assert rep["outputs"] == sum(i["p"].M * 8 for i in items)
+    # a wrong output is reported
+    items[4]["ys"][0][0, 3] = items[4]["ys"][0][0, 3] * 1.5 + 1.0
+    rep = bench.parity_sample(_FakeRun(items), torch, rows=8)
+    assert not rep["within_tolerance"] and rep["max_abs_err"] > 0.5
