@@ -1,6 +1,5 @@
 """The C ABI library: it loads without a GPU, exports every function the header
 declares, and rejects bad arguments on the host before touching a device."""
-import ctypes
 import os
 import re
 

@@ -13,7 +13,7 @@ import torch
 import fp8_linear_layers_b200 as ql
 import oracle
 from fp8_linear_layers_b200 import synthetic
-from tests._util import bf16_dev, bits
+from tests._util import bf16_dev
 
 pytestmark = pytest.mark.gpu
 

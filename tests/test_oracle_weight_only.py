@@ -17,7 +17,6 @@ from fractions import Fraction
 
 import numpy as np
 import pytest
-import torch
 
 import oracle
 from fp8_linear_layers_b200 import synthetic
