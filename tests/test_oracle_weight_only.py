@@ -11,7 +11,9 @@ model page's "Context": X stays bf16, only W is quantized.
 * numpy's f64 matmul of X and the dequantized weights (a library routine);
 * the W8A8 result on inputs that per-token quantization reproduces exactly;
 * agreement with the unquantized X . W^T within the weight-rounding bound;
-* sign symmetry and argument checks.
+* sign symmetry and argument checks;
+* the hand-worked example in ``tests/golden/weight_only_worked_example.txt``
+  (two ties rounded to even).
 """
 from fractions import Fraction
 
@@ -162,3 +164,17 @@ def test_weight_only_rejects_bad_shapes():
     with pytest.raises(ValueError):
         oracle.linear_weight_only(INT8, x, np.zeros((4, 128), np.uint8), np.ones(4, np.float32),
                                   n0=2, n1=5)
+
+
+def test_weight_only_worked_example_golden():
+    import os
+    from test_oracle_linear import GOLDEN, _read_worked
+    d = _read_worked(os.path.join(GOLDEN, "weight_only_worked_example.txt"))
+    x = _bf16(np.array([[float(v) for v in d["x"]]]))
+    w = np.array([[float(v) for v in d[f"w{i}"]] for i in range(3)]) * 2.0 ** int(d["w_exp"][0])
+    wq, sw = oracle.quantize_weight(INT8, _bf16(w))
+    assert np.all(sw == np.float32(2.0 ** int(d["w_exp"][0])))
+    y, acc = oracle.linear_weight_only(INT8, x, wq, sw, want_acc=True)
+    scale = 2.0 ** int(d["w_exp"][0])
+    assert (acc[0] / scale).tolist() == [float(v) for v in d["sum"]]
+    assert oracle.bf16_bits_to_f64(y)[0].tolist() == [float(v) for v in d["y"]]
