@@ -172,7 +172,7 @@ static int64_t e4m3_units(uint8_t c) {
 /* ------------------------------------------------------------------------ */
 
 static uint8_t quantize_one(int scheme, float x, float s) {
-  float t = (s > 0.0f) ? x / s : 0.0f;
+  float t = (s > 0.0f) ? (MUTANT(16) ? x * (1.0f / s) : x / s) : 0.0f;
   if (scheme == ORACLE_INT8_ROW) return (uint8_t)(int8_t)oracle_int8_round(t);
   return oracle_e4m3_encode(t);
 }
@@ -196,7 +196,7 @@ int oracle_quantize_weight(int scheme, const uint16_t* w, int64_t N, int64_t K, 
           for (int64_t k = kb * 128; k < kb * 128 + 128; ++k)
             a = fmaxf(a, fabsf(oracle_bf16_to_f32(w[n * K + k])));
         if (MUTANT(11)) a = fabsf(oracle_bf16_to_f32(w[nb * 128 * K + kb * 128]));
-        float s = a / 448.0f;
+        float s = MUTANT(18) ? a * (1.0f / 448.0f) : a / 448.0f;
         sw[nb * KB + kb] = s;
         for (int64_t n = nb * 128; n < nb * 128 + 128; ++n)
           for (int64_t k = kb * 128; k < kb * 128 + 128; ++k)
@@ -212,7 +212,7 @@ int oracle_quantize_weight(int scheme, const uint16_t* w, int64_t N, int64_t K, 
     if (scheme == ORACLE_INT8_ROW)
       s = MUTANT(5) ? a / 127.0f : oracle_bf16_to_f32(oracle_f32_to_bf16(a / 127.0f));
     else
-      s = a / 448.0f;
+      s = MUTANT(18) ? a * (1.0f / 448.0f) : a / 448.0f;
     sw[n] = s;
     for (int64_t k = 0; k < K; ++k)
       wq[n * K + k] = quantize_one(scheme, oracle_bf16_to_f32(w[n * K + k]), s);
@@ -240,7 +240,7 @@ int oracle_quantize_act(int scheme, const uint16_t* x, int64_t M, int64_t K, uin
       for (int64_t k = 0; k < width; ++k) a = fmaxf(a, fabsf(oracle_bf16_to_f32(xs[k])));
       if (MUTANT(7)) /* per-token absmax where a per-group one is due */
         for (int64_t k = 0; k < K; ++k) a = fmaxf(a, fabsf(oracle_bf16_to_f32(x[m * K + k])));
-      float s = a / qmax;
+      float s = MUTANT(17) ? a * (1.0f / qmax) : a / qmax;
       sx[m * G + g] = s;
       for (int64_t k = 0; k < width; ++k)
         qx[m * K + g * width + k] = quantize_one(scheme, oracle_bf16_to_f32(xs[k]), s);

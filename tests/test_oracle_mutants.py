@@ -14,7 +14,7 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_codecs.py", "tests/test_oracle_quant.py", "tests/test_oracle_linear.py",
-        "tests/test_oracle_weight_only.py"]
+        "tests/test_oracle_weight_only.py", "tests/test_oracle_division.py"]
 
 MUTANTS = {
     1: "f32->bf16 truncates instead of rounding",
@@ -32,6 +32,9 @@ MUTANTS = {
     13: "weight-only product drops the weight scale",
     14: "weight-only block weight-scale index transposed",
     15: "weight-only product drops the first input channel",
+    16: "quotient x * (1 / s) instead of the division x / s",
+    17: "activation scale absmax * (1 / qmax) instead of absmax / qmax",
+    18: "E4M3 weight scale absmax * (1 / 448) instead of absmax / 448",
 }
 
 
