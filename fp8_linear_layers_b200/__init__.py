@@ -39,7 +39,10 @@ STATUS = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED_SHAPE", 3:
 EXPORTS = ("qlinear_quantize_weight", "qlinear_quantize_act", "qlinear_gemv", "qlinear_gemm_small",
            "qlinear_gemm", "qlinear_forward", "qlinear_workspace_bytes",
            "qlinear_forward_workspace_bytes", "qlinear_get_device_status", "qlinear_status_string",
-           "qlinear_last_cuda_error", "qlinear_gemm_small_noalloc", "qlinear_gemv_weight_only")
+           "qlinear_last_cuda_error", "qlinear_gemm_small_noalloc", "qlinear_gemv_weight_only",
+           "qlinear_debug_gemv_stalled", "qlinear_forward_weight_only", "qlinear_gemv_grouped",
+           "qlinear_gemv_prequant", "qlinear_gemm_small_prequant",
+           "qlinear_gemm_quant_out", "qlinear_weight_only_workspace_bytes")
 
 
 class QLinearError(RuntimeError):
@@ -85,6 +88,14 @@ def lib() -> ctypes.CDLL:
         L.qlinear_quantize_act.argtypes = [i32, vp, i64, i64, vp, vp, vp]
         L.qlinear_gemv.argtypes = [i32, vp, vp, vp, i64, i64, vp, vp, vp]
         L.qlinear_gemv_weight_only.argtypes = [i32, vp, vp, vp, i64, i64, vp, vp]
+        L.qlinear_debug_gemv_stalled.argtypes = [i32, vp, vp, vp, i64, i64, vp, vp]
+        L.qlinear_forward_weight_only.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]
+        L.qlinear_weight_only_workspace_bytes.argtypes = [i32, i64, i64, i64]
+        L.qlinear_weight_only_workspace_bytes.restype = sz
+        L.qlinear_gemv_grouped.argtypes = [i32, vp, i32, i64, vp]
+        L.qlinear_gemv_prequant.argtypes = [i32, vp, vp, vp, vp, i64, i64, vp, vp]
+        L.qlinear_gemm_small_prequant.argtypes = [i32, vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]
+        L.qlinear_gemm_quant_out.argtypes = [i32, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp, sz, vp]
         L.qlinear_gemm_small.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp, vp]
         L.qlinear_gemm.argtypes = [i32, vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp, vp]
         L.qlinear_forward.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]
@@ -100,7 +111,10 @@ def lib() -> ctypes.CDLL:
         for name in ("qlinear_quantize_weight", "qlinear_quantize_act", "qlinear_gemv",
                      "qlinear_gemm_small", "qlinear_gemm", "qlinear_forward",
                      "qlinear_get_device_status", "qlinear_gemm_small_noalloc",
-                     "qlinear_gemv_weight_only"):
+                     "qlinear_gemv_weight_only", "qlinear_debug_gemv_stalled",
+                     "qlinear_forward_weight_only", "qlinear_gemv_grouped",
+                     "qlinear_gemv_prequant", "qlinear_gemm_small_prequant",
+                     "qlinear_gemm_quant_out"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -176,6 +190,61 @@ def gemv(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor, y=Non
     return y
 
 
+GEMV_MAX_GROUP = 8  # QL_GEMV_MAX_GROUP
+
+
+class _GemvProblem(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("qx", ctypes.c_void_p), ("sx", ctypes.c_void_p),
+                ("wq", ctypes.c_void_p), ("sw", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("N", ctypes.c_int64)]
+
+
+def gemv_grouped(scheme: int, problems, stream=None) -> list:
+    """Several M = 1 products of one K in one launch.  `problems` is a list of
+    (x, wq [N,K], sw, y or None) tuples, x a bf16 [1,K] tensor or a pair
+    (q_x [1,K] uint8, s_x f32) already quantized; returns the outputs [1,N]."""
+    if not 1 <= len(problems) <= GEMV_MAX_GROUP:
+        raise ValueError(f"1 to {GEMV_MAX_GROUP} products per grouped launch")
+    K = problems[0][1].shape[1]
+    table = (_GemvProblem * len(problems))()
+    ys = []
+    for j, (x, wq, sw, y) in enumerate(problems):
+        qx, sx = (x if isinstance(x, tuple) else (None, None))
+        xin = qx if qx is not None else x
+        if xin.numel() != K or xin.shape[-1] != K or wq.shape[1] != K:
+            raise ValueError("every product of a grouped launch takes one token of the same K")
+        N = wq.shape[0]
+        if y is None:
+            y = torch.empty((1, N), dtype=torch.bfloat16, device=xin.device)
+        if qx is None:
+            table[j] = _GemvProblem(_dev(x, torch.bfloat16, "x"), None, None, _dev(wq, torch.uint8, "wq"),
+                                    _dev(sw, torch.float32, "sw"), _dev(y, torch.bfloat16, "y"), N)
+        else:
+            table[j] = _GemvProblem(None, _dev(qx, torch.uint8, "qx"), _dev(sx, torch.float32, "sx"),
+                                    _dev(wq, torch.uint8, "wq"), _dev(sw, torch.float32, "sw"),
+                                    _dev(y, torch.bfloat16, "y"), N)
+        ys.append(y)
+    _check(lib().qlinear_gemv_grouped(scheme, ctypes.cast(table, ctypes.c_void_p), len(problems), K,
+                                      _stream(stream)), "qlinear_gemv_grouped")
+    return ys
+
+
+def gemv_prequant(scheme: int, qx: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
+                  y=None, stream=None) -> torch.Tensor:
+    """M = 1 on an input already quantized: q_x uint8 [1,K], s_x f32 -> y bf16 [1,N]."""
+    K = qx.shape[-1]
+    N = wq.shape[0]
+    if qx.numel() != K:
+        raise ValueError("gemv_prequant takes a single token")
+    if y is None:
+        y = torch.empty((1, N), dtype=torch.bfloat16, device=qx.device)
+    _check(lib().qlinear_gemv_prequant(scheme, _dev(qx, torch.uint8, "qx"), _dev(sx, torch.float32, "sx"),
+                                       _dev(wq, torch.uint8, "wq"), _dev(sw, torch.float32, "sw"), N, K,
+                                       _dev(y, torch.bfloat16, "y"), _stream(stream)),
+           "qlinear_gemv_prequant")
+    return y
+
+
 def gemv_weight_only(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor, y=None,
                      stream=None) -> torch.Tensor:
     """M = 1 weight-only product ("equivalent" numerics, W8A16 / FP8 weight-only):
@@ -191,6 +260,45 @@ def gemv_weight_only(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.T
                                           N, K, _dev(y, torch.bfloat16, "y"), _stream(stream)),
            "qlinear_gemv_weight_only")
     return y
+
+
+def debug_gemv_stalled(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor, y=None,
+                       stream=None) -> torch.Tensor:
+    """Test hook: gemv with its weight copies held back, so its bounded waits run
+    out (about 2 s) and the kernel records QL_ERR_TIMEOUT in the status word."""
+    K = x.shape[-1]
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((1, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().qlinear_debug_gemv_stalled(scheme, _dev(x, torch.bfloat16, "x"),
+                                            _dev(wq, torch.uint8, "wq"), _dev(sw, torch.float32, "sw"),
+                                            N, K, _dev(y, torch.bfloat16, "y"), _stream(stream)),
+           "qlinear_debug_gemv_stalled")
+    return y
+
+
+def forward_weight_only(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor, y=None,
+                        workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """1 <= M <= 32 weight-only product: x bf16 [M,K] is not rounded -> y bf16 [M,N].
+    A zero-filled workspace of weight_only_workspace_bytes(...) is made if none is given."""
+    M, K = x.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        nb = weight_only_workspace_bytes(scheme, M, N, K)
+        workspace = new_workspace(nb) if nb else None
+    wp, wn = _ws(workspace)
+    _check(lib().qlinear_forward_weight_only(scheme, _dev(x, torch.bfloat16, "x"),
+                                             _dev(wq, torch.uint8, "wq"),
+                                             _dev(sw, torch.float32, "sw"), M, N, K,
+                                             _dev(y, torch.bfloat16, "y"), wp, wn, _stream(stream)),
+           "qlinear_forward_weight_only")
+    return y
+
+
+def weight_only_workspace_bytes(scheme: int, M: int, N: int, K: int) -> int:
+    return int(lib().qlinear_weight_only_workspace_bytes(scheme, M, N, K))
 
 
 def workspace_bytes(scheme: int, M: int, N: int, K: int) -> int:
@@ -228,6 +336,21 @@ def gemm_small(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
     return y
 
 
+def gemm_small_prequant(scheme: int, qx: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor,
+                        sw: torch.Tensor, workspace: torch.Tensor, y=None, stream=None):
+    """1 <= M <= 32 on an input already quantized: q_x uint8 [M,K], s_x f32 -> y bf16 [M,N]."""
+    M, K = qx.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device)
+    wp, wn = _ws(workspace)
+    _check(lib().qlinear_gemm_small_prequant(scheme, _dev(qx, torch.uint8, "qx"), _dev(sx, torch.float32, "sx"),
+                                             _dev(wq, torch.uint8, "wq"), _dev(sw, torch.float32, "sw"),
+                                             M, N, K, _dev(y, torch.bfloat16, "y"), wp, wn, _stream(stream)),
+           "qlinear_gemm_small_prequant")
+    return y
+
+
 def gemm_small_noalloc(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor, y=None,
                        stream=None):
     """Same as ``gemm_small`` with the library's fixed device scratch instead of a
@@ -259,6 +382,28 @@ def gemm(scheme: int, qx: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: 
                               _dev(y, torch.bfloat16, "y"), wp, wn, debug._c() if debug else None,
                               _stream(stream)), "qlinear_gemm")
     return y
+
+
+def gemm_quant_out(scheme: int, qx: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
+                   workspace: torch.Tensor | None = None, y=None, want_y: bool = True, qy=None, sy=None,
+                   stream=None):
+    """Block scheme, large M: q_x, s_x -> (y bf16 [M,N] or None, q_y uint8 [M,N], s_y f32 [M,N/128]),
+    the output quantized in the same kernel for the product that reads it next."""
+    M, K = qx.shape
+    N = wq.shape[0]
+    if want_y and y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device)
+    if qy is None:
+        qy = torch.empty((M, N), dtype=torch.uint8, device=qx.device)
+    if sy is None:
+        sy = torch.empty((M, N // 128), dtype=torch.float32, device=qx.device)
+    wp, wn = _ws(workspace)
+    _check(lib().qlinear_gemm_quant_out(scheme, _dev(qx, torch.uint8, "qx"), _dev(sx, torch.float32, "sx"),
+                                        _dev(wq, torch.uint8, "wq"), _dev(sw, torch.float32, "sw"), M, N, K,
+                                        _dev(y, torch.bfloat16, "y") if y is not None else None,
+                                        _dev(qy, torch.uint8, "qy"), _dev(sy, torch.float32, "sy"), wp, wn,
+                                        _stream(stream)), "qlinear_gemm_quant_out")
+    return y, qy, sy
 
 
 def forward(scheme: int, x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,

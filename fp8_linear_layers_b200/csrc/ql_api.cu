@@ -167,6 +167,57 @@ ql_status qlinear_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, cons
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemv");
 }
 
+ql_status qlinear_gemv_grouped(ql_scheme scheme, const ql_gemv_problem* problems, int count,
+                               int64_t K, void* stream) {
+  if (!valid_scheme(scheme) || !problems) return QL_ERR_INVALID_ARG;
+  if (count < 1 || count > QL_GEMV_MAX_GROUP) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  if (K > ql::gemv_max_k()) return QL_ERR_UNSUPPORTED_SHAPE;
+  for (int j = 0; j < count; ++j) {
+    const ql_gemv_problem& pr = problems[j];
+    QL_TRY(check_n(scheme, pr.N, K));
+    if (pr.x) {
+      QL_TRY(need(pr.x));
+    } else {
+      QL_TRY(need(pr.qx));
+      QL_TRY(need(pr.sx));
+    }
+    QL_TRY(need(pr.wq));
+    QL_TRY(need(pr.sw));
+    QL_TRY(need(pr.y));
+  }
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  cudaError_t e = ql::launch_gemv_grouped(scheme, problems, count, K, d.sms, d.status,
+                                          static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemv_grouped");
+}
+
+ql_status qlinear_gemv_prequant(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
+                                const float* sw, int64_t N, int64_t K, uint16_t* y, void* stream) {
+  if (!qx || !sx) return QL_ERR_INVALID_ARG;
+  const ql_gemv_problem one{nullptr, qx, sx, wq, sw, y, N};
+  return qlinear_gemv_grouped(scheme, &one, 1, K, stream);
+}
+
+ql_status qlinear_debug_gemv_stalled(ql_scheme scheme, const uint16_t* x, const void* wq,
+                                    const float* sw, int64_t N, int64_t K, uint16_t* y,
+                                    void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_n(scheme, N, K));
+  if (K > ql::gemv_max_k()) return QL_ERR_UNSUPPORTED_SHAPE;
+  QL_TRY(need(x));
+  QL_TRY(need(wq));
+  QL_TRY(need(sw));
+  QL_TRY(need(y));
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  cudaError_t e = ql::launch_gemv(scheme, x, wq, sw, 1, N, K, y, nullptr, d.sms, d.status,
+                                  static_cast<cudaStream_t>(stream), true);
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_debug_gemv_stalled");
+}
+
 ql_status qlinear_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const void* wq,
                                    const float* sw, int64_t N, int64_t K, uint16_t* y,
                                    void* stream) {
@@ -180,9 +231,37 @@ ql_status qlinear_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const vo
   QL_TRY(need(y));
   DeviceInfo d;
   QL_TRY(current_device(&d));
-  cudaError_t e = ql::launch_gemv_weight_only(scheme, x, wq, sw, N, K, y, d.sms, d.status,
+  cudaError_t e = ql::launch_gemv_weight_only(scheme, x, wq, sw, 1, N, K, y, d.sms, d.status,
                                               static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemv_weight_only");
+}
+
+ql_status qlinear_forward_weight_only(ql_scheme scheme, const uint16_t* x, const void* wq,
+                                      const float* sw, int64_t M, int64_t N, int64_t K,
+                                      uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_n(scheme, N, K));
+  QL_TRY(check_m(M, N, K));
+  if (M == 0) return QL_OK;
+  if (M > 32) return QL_ERR_UNSUPPORTED_SHAPE;
+  QL_TRY(need(x));
+  QL_TRY(need(wq));
+  QL_TRY(need(sw));
+  QL_TRY(need(y));
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  const size_t need_ws = ql::gemm_small_wo_workspace_bytes(scheme, M, N, K);
+  if (need_ws && (!workspace || ws_bytes < need_ws)) return QL_ERR_WORKSPACE;
+  if (need_ws && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return QL_ERR_MISALIGNED;
+  cudaError_t e = ql::launch_gemm_small_wo(scheme, x, wq, sw, M, N, K, y, workspace, ws_bytes, d.sms,
+                                           d.status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_forward_weight_only");
+}
+
+size_t qlinear_weight_only_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K) {
+  if (!valid_scheme(scheme) || M <= 0 || M > 32 || N <= 0 || K <= 0) return 0;
+  return ql::gemm_small_wo_workspace_bytes(scheme, M, N, K);
 }
 
 ql_status qlinear_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
@@ -207,6 +286,32 @@ ql_status qlinear_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq
   cudaError_t e = ql::launch_gemm_small(scheme, x, wq, sw, M, N, K, y, workspace, ws_bytes, dbg,
                                         d.sms, d.status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm_small");
+}
+
+ql_status qlinear_gemm_small_prequant(ql_scheme scheme, const void* qx, const float* sx,
+                                      const void* wq, const float* sw, int64_t M, int64_t N,
+                                      int64_t K, uint16_t* y, void* workspace, size_t ws_bytes,
+                                      void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_n(scheme, N, K));
+  QL_TRY(check_m(M, N, K));
+  if (M == 0) return QL_OK;
+  if (M > 32) return QL_ERR_UNSUPPORTED_SHAPE;
+  QL_TRY(need(qx));
+  QL_TRY(need(sx));
+  QL_TRY(need(wq));
+  QL_TRY(need(sw));
+  QL_TRY(need(y));
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  const size_t need_ws = ql::gemm_small_workspace_bytes(scheme, M, N, K, d.sms);
+  if (!workspace || ws_bytes < need_ws) return QL_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return QL_ERR_MISALIGNED;
+  cudaError_t e = ql::launch_gemm_small(scheme, nullptr, wq, sw, M, N, K, y, workspace, ws_bytes,
+                                        nullptr, d.sms, d.status, static_cast<cudaStream_t>(stream),
+                                        static_cast<const uint8_t*>(qx), sx);
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm_small_prequant");
 }
 
 ql_status qlinear_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
@@ -234,6 +339,34 @@ ql_status qlinear_gemm(ql_scheme scheme, const void* qx, const float* sx, const 
                                   use_ws ? ws_bytes : 0, dbg, d.sms, d.status,
                                   static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm");
+}
+
+ql_status qlinear_gemm_quant_out(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
+                                 const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                 void* qy, float* sy, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  if (scheme != QL_FP8_E4M3_BLOCK128) return QL_ERR_UNSUPPORTED_SHAPE;
+  QL_TRY(check_k(scheme, K));
+  QL_TRY(check_n(scheme, N, K));
+  QL_TRY(check_m(M, N, K));
+  if (M == 0) return QL_OK;
+  QL_TRY(need(qx));
+  QL_TRY(need(sx));
+  QL_TRY(need(wq));
+  QL_TRY(need(sw));
+  QL_TRY(need(qy));
+  QL_TRY(need(sy));
+  if (y) QL_TRY(need(y));
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  const size_t need_ws = ql::gemm_workspace_bytes(scheme, M, N, K, d.sms);
+  const bool use_ws = need_ws && workspace && ws_bytes >= need_ws;
+  if (use_ws && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return QL_ERR_MISALIGNED;
+  cudaError_t e = ql::launch_gemm(scheme, qx, sx, wq, sw, M, N, K, y, use_ws ? workspace : nullptr,
+                                  use_ws ? ws_bytes : 0, nullptr, d.sms, d.status,
+                                  static_cast<cudaStream_t>(stream), static_cast<uint8_t*>(qy), sy);
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm_quant_out");
 }
 
 size_t qlinear_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K) {
@@ -370,11 +503,13 @@ extern "C" ql_status qlinear_gemm_small_noalloc(ql_scheme scheme, const uint16_t
   void* scratch = nullptr;
   QL_TRY(noalloc_scratch(&scratch));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // The split-tile sums and arrival counters must start at zero; the scratch
-  // keeps whatever the previous call left, so clear them (no allocation).
+  // The arrival counters and the atomic-sum slots must start at zero; the
+  // scratch keeps whatever the previous call left, so clear them (no
+  // allocation).  Nothing to clear when the shape runs on the GEMV kernel.
   const size_t zeroed = ql::gemm_small_zeroed_bytes(scheme, M, N, K, d.sms);
-  cudaError_t e = cudaMemsetAsync(scratch, 0, zeroed, st);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scratch sums and counters)");
+  cudaError_t e = cudaSuccess;
+  if (zeroed && (e = cudaMemsetAsync(scratch, 0, zeroed, st)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemsetAsync(scratch sums and counters)");
   e = ql::launch_gemm_small(scheme, x, wq, sw, M, N, K, y, scratch, kNoAllocScratchBytes, nullptr,
                             d.sms, d.status, st);
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm_small_noalloc");

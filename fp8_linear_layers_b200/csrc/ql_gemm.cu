@@ -62,6 +62,8 @@ struct GemmParams {
   uint32_t* counters;  // split = 2: [mt * nt] arrivals per tile, zero between calls
   int32_t* acc_i32;
   float* acc_f32;
+  uint8_t* qy;      // block scheme: E4M3 codes of y [M,N] for the next product, or null
+  float* sy;        // and their scales [M, N/128]
   DevStatus* status;
 };
 
@@ -99,7 +101,8 @@ struct GemmCfg {
   static constexpr int kBufCols = BN <= 128 ? 128 : 256;  // TMEM columns per accumulator
   static constexpr int kBufs = kTmemCols / kBufCols;
   static constexpr int kHalf = BN / 2;                    // columns per epilogue warp
-  static constexpr int kSmem = kRing + kStaging + 1024 + 256;
+  static constexpr int kRed = kGemmEpiWarps * 32 * 4;  // per-lane group maxima (output quantization)
+  static constexpr int kSmem = kRing + kStaging + kRed + 1024 + 256;
   static_assert(BN % 32 == 0 && BN <= 256, "tile N");
   static_assert(kStage % 1024 == 0, "stages must stay 1024-byte aligned");
 };
@@ -153,7 +156,8 @@ QL_DEVINL void store_box32(uint8_t* box, int lane, const uint32_t (&w)[16], uint
   }
 }
 
-template <ql_scheme S, int BN>
+// kQ (block scheme only): the epilogue also writes y's E4M3 codes and scales.
+template <ql_scheme S, int BN, bool kQ = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmParams p) {
@@ -167,7 +171,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = align1024(smem_raw);
   uint8_t* staging = ring + Cfg::kRing;  // 1024-byte aligned (stages are)
-  uint64_t* full = reinterpret_cast<uint64_t*>(staging + Cfg::kStaging);
+  float* red = reinterpret_cast<float*>(staging + Cfg::kStaging);
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + Cfg::kStaging + Cfg::kRed);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + kBufs;
@@ -446,7 +451,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ++jt;
         }
         if (p.split == 1) {
-          if (!ok) return false;
+          // the output quantization of 128-wide tiles meets the partner warp
+          // at a barrier: every warp votes first, so that all leave together
+          if (kQ && Cfg::kHalf < 128) {
+            if (gemm_epi_any(!ok)) return false;
+          } else if (!ok) {
+            return false;
+          }
         } else {
           // Split tile: every epilogue warp reaches the votes and barriers
           // below, so they leave together if any of them gave up a wait.
@@ -500,7 +511,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (ew == 0 && lane == 0) p.counters[t] = 0u;  // both halves have arrived
         }
         const int mrow = m0 + q * 32;
-        if (live_n && mrow < p.M) {
+        if constexpr (kQ) {
+          // The output's own quantization for the product that reads it next
+          // (E4M3, one scale per token per 128 outputs: the group of 128
+          // columns is this thread's row here, split over the warps of the
+          // two column halves on 128-wide tiles).  The codes are those of the
+          // bf16 y: s = absmax / 448 (one IEEE division), code = E4M3(y / s).
+          // Rounding to bf16 is monotonic in |v|, so the largest |bf16(v)| of
+          // the group is bf16(max |v|).
+          float a = 0.0f;
+#pragma unroll
+          for (int j = 0; j < Cfg::kHalf / 2; ++j) a = fmaxf(a, fmaxf(fabsf(acc[j].x), fabsf(acc[j].y)));
+          a = bf16_lo(f32_to_bf16_rn(a));
+          if constexpr (Cfg::kHalf < 128) {
+            red[ew * 32 + lane] = a;
+            named_bar_sync(kGemmEpiBar, kGemmEpiWarps * 32);
+            a = fmaxf(a, red[(ew ^ 4) * 32 + lane]);
+            named_bar_sync(kGemmEpiBar, kGemmEpiWarps * 32);  // red is free again
+          }
+          auto pack = [&](int j) {
+            return (uint32_t)f32_to_bf16_rn(acc[j].x) | ((uint32_t)f32_to_bf16_rn(acc[j].y) << 16);
+          };
+          if (p.y && live_n && mrow < p.M) {
+#pragma unroll
+            for (int c = 0; c < Cfg::kHalf / 32; ++c) {
+              uint32_t w[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) w[j] = pack(c * 16 + j);
+              store_box32(staging + ew * Cfg::kBox, lane, w, p.y, mrow, ncol + c * 32, p.M, p.N);
+            }
+          }
+          const float sc = a / 448.0f;
+          const Divisor dv = make_divisor(sc);
+          if (live_n && live_m) {
+            uint8_t* qrow = p.qy + (int64_t)m * p.N + ncol;
+#pragma unroll
+            for (int c = 0; c < Cfg::kHalf / 16; ++c) {
+              const uint2 q0 = quant_chunk8<false>(make_uint4(pack(8 * c), pack(8 * c + 1), pack(8 * c + 2), pack(8 * c + 3)), dv);
+              const uint2 q1 = quant_chunk8<false>(make_uint4(pack(8 * c + 4), pack(8 * c + 5), pack(8 * c + 6), pack(8 * c + 7)), dv);
+              *reinterpret_cast<uint4*>(qrow + c * 16) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+            }
+            if ((ncol & 127) == 0) p.sy[(int64_t)m * (p.N / 128) + (ncol >> 7)] = sc;
+          }
+        } else if (live_n && mrow < p.M) {
 #pragma unroll
           for (int c = 0; c < Cfg::kHalf / 32; ++c) {
             uint32_t w[16];
@@ -589,11 +642,11 @@ size_t gemm_workspace_bytes(ql_scheme s, int64_t M, int64_t N, int64_t K, int sm
   return align256(split_parts_bytes(tiles)) + align256((size_t)tiles * 4);
 }
 
-template <ql_scheme S, int BN>
+template <ql_scheme S, int BN, bool kQ = false>
 static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
                                  int sms, cudaStream_t st) {
   using Cfg = GemmCfg<BN, S == QL_FP8_E4M3_BLOCK128>;
-  cudaError_t e = ensure_smem<gemm_kernel<S, BN>>(Cfg::kSmem);
+  cudaError_t e = ensure_smem<gemm_kernel<S, BN, kQ>>(Cfg::kSmem);
   if (e != cudaSuccess) return e;
   const int grid = (int)std::min<int64_t>((int64_t)p.mt * p.nt * p.split, sms);
   cudaLaunchConfig_t cfg = {};
@@ -606,13 +659,15 @@ static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_kernel<S, BN>, a, b, p);
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<S, BN, kQ>, a, b, p);
 }
 
 cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
                         const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
                         size_t ws_bytes, const ql_debug* dbg, int num_sms, DevStatus* status,
-                        cudaStream_t st) {
+                        cudaStream_t st, uint8_t* qy, float* sy) {
+  if ((qy != nullptr) != (sy != nullptr) || (qy && scheme != QL_FP8_E4M3_BLOCK128))
+    return cudaErrorInvalidValue;
   // the K split needs its workspace; without one, whole tiles
   GemmPlan pl = plan_gemm(scheme, M, N, K, num_sms);
   const size_t need = gemm_workspace_bytes(scheme, M, N, K, num_sms);
@@ -635,6 +690,8 @@ cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const
                             : nullptr;
   p.acc_i32 = dbg ? dbg->acc_i32 : nullptr;
   p.acc_f32 = dbg ? dbg->acc_f32 : nullptr;
+  p.qy = qy;
+  p.sy = sy;
   p.status = status;
   CUtensorMap ta, tb;
   cudaError_t e = make_tmap_u8_sw128(&ta, qx, (uint64_t)K, (uint64_t)M, (uint64_t)K, kGemmBK, kGemmBM);
@@ -655,6 +712,10 @@ cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const
       if (BN == 160) return launch_gemm_t<QL_FP8_E4M3_ROW, 160>(p, ta, tb, num_sms, st);
       return launch_gemm_t<QL_FP8_E4M3_ROW, 128>(p, ta, tb, num_sms, st);
     default:
+      if (qy) {
+        if (BN == 256) return launch_gemm_t<QL_FP8_E4M3_BLOCK128, 256, true>(p, ta, tb, num_sms, st);
+        return launch_gemm_t<QL_FP8_E4M3_BLOCK128, 128, true>(p, ta, tb, num_sms, st);
+      }
       if (BN == 256) return launch_gemm_t<QL_FP8_E4M3_BLOCK128, 256>(p, ta, tb, num_sms, st);
       return launch_gemm_t<QL_FP8_E4M3_BLOCK128, 128>(p, ta, tb, num_sms, st);
   }

@@ -56,7 +56,8 @@ struct SmallParams {
   int ntn;          // 128-row tiles of W_q
   int nkb;          // 128-byte K blocks
   int units;        // ntn * nkb
-  void* accum;         // [ntn][kSmallSlots][NTOK][128] int32 or f32: parked partials, or atomic sums (zero between calls)
+  void* accum;         // [kSmallSlots][ntn][NTOK][128] int32 or f32: parked partials, or atomic
+                       // sums in slot 0 (slot 0 zero between calls; slot 1 written before read)
   unsigned* counters;  // [ntn], zero between calls
   int32_t* acc_i32;
   float* acc_f32;
@@ -313,9 +314,11 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         const int c_last = unit_owner((t + 1) * nkb - 1, p.units, G);
         const int ncon = c_last - c_first + 1;
         const bool few = ncon <= kSmallSlots;
-        Acc* tacc = reinterpret_cast<Acc*>(p.accum) + (int64_t)t * kSmallSlots * NTOK * 128;
+        // slot k of tile t; slot 0 is also the atomic-sum slot
+        Acc* tacc = reinterpret_cast<Acc*>(p.accum) + (int64_t)t * NTOK * 128;
+        const int64_t slot_stride = (int64_t)p.ntn * NTOK * 128;
         if (few) {
-          Acc* slot = tacc + (c - c_first) * NTOK * 128;
+          Acc* slot = tacc + (c - c_first) * slot_stride;
 #pragma unroll
           for (int m = 0; m < NTOK; ++m)
             if (m < p.M) slot[m * 128 + et] = acc[m];
@@ -340,7 +343,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
               Acc v = 0;
               if (m < p.M) {
                 // fixed order: the first contributor's part, then the second's
-                v = __ldcg(tacc + m * 128 + et) + __ldcg(tacc + NTOK * 128 + m * 128 + et);
+                v = __ldcg(tacc + m * 128 + et) + __ldcg(tacc + slot_stride + m * 128 + et);
               }
               acc[m] = v;
             }
@@ -393,18 +396,22 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
 
 namespace {
 struct SmallLayout {
-  size_t qx, sx, accum, counters, total;
+  size_t qx, sx, accum, counters, zeroed, total;
 };
 
 SmallLayout small_layout(ql_scheme s, int64_t M, int64_t N, int64_t K, int sms) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
   const int ntok = M <= 16 ? 16 : 32;
   (void)sms;
-  // the region that must be zero when a call starts comes first
+  // The region that must be zero when a call starts comes first: the arrival
+  // counters, then partial-sum slot 0 of every tile (the atomic-sum slot);
+  // slot 1 (parked partials, always written before they are read) follows.
+  const size_t slot_bytes = (size_t)((N + 127) / 128) * ntok * 128 * 4;
   SmallLayout L;
   L.counters = 0;
   L.accum = up((size_t)((N + 127) / 128) * 4);
-  L.qx = L.accum + up((size_t)((N + 127) / 128) * kSmallSlots * ntok * 128 * 4);
+  L.zeroed = L.accum + slot_bytes;
+  L.qx = L.accum + up(kSmallSlots * slot_bytes);
   L.sx = L.qx + up((size_t)(M * K));
   L.total = L.sx + up((size_t)M * (s == QL_FP8_E4M3_BLOCK128 ? K / 128 : 1) * 4);
   return L;
@@ -416,7 +423,9 @@ size_t gemm_small_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_
 }
 
 size_t gemm_small_zeroed_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms) {
-  return small_layout(scheme, M, N, K, num_sms).qx;
+  // the GEMV route (up to four tokens) does not touch the workspace
+  if (K <= gemv_max_k_tokens(M)) return 0;
+  return small_layout(scheme, M, N, K, num_sms).zeroed;
 }
 
 template <ql_scheme S, int NTOK>
@@ -441,19 +450,26 @@ static cudaError_t launch_small_t(const SmallParams& p, const CUtensorMap& tw, c
 cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq,
                               const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
                               void* workspace, size_t ws_bytes, const ql_debug* dbg, int num_sms,
-                              DevStatus* status, cudaStream_t st) {
+                              DevStatus* status, cudaStream_t st, const uint8_t* pre_qx,
+                              const float* pre_sx) {
   const SmallLayout L = small_layout(scheme, M, N, K, num_sms);
   if (ws_bytes < L.total) return cudaErrorInvalidValue;
-  // Up to four tokens: the GEMV kernel carries them on its MMA's B columns
-  // with the activation quantization fused, at the weight traffic of one
-  // token and without the split-K reduction (the workspace is not used).
-  if (K <= gemv_max_k_tokens(M))
-    return launch_gemv(scheme, x, wq, sw, M, N, K, y, dbg, num_sms, status, st);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint8_t* qx = ws + L.qx;
-  float* sx = reinterpret_cast<float*>(ws + L.sx);
-  cudaError_t e = launch_quantize_act(scheme, x, M, K, qx, sx, st);
-  if (e != cudaSuccess) return e;
+  const uint8_t* qx = pre_qx;
+  const float* sx = pre_sx;
+  cudaError_t e = cudaSuccess;
+  if (!pre_qx) {
+    // Up to four tokens: the GEMV kernel carries them on its MMA's B columns
+    // with the activation quantization fused, at the weight traffic of one
+    // token and without the split-K reduction (the workspace is not used).
+    if (K <= gemv_max_k_tokens(M))
+      return launch_gemv(scheme, x, wq, sw, M, N, K, y, dbg, num_sms, status, st);
+    uint8_t* wqx = ws + L.qx;
+    float* wsx = reinterpret_cast<float*>(ws + L.sx);
+    if ((e = launch_quantize_act(scheme, x, M, K, wqx, wsx, st)) != cudaSuccess) return e;
+    qx = wqx;
+    sx = wsx;
+  }
 
   SmallParams p;
   p.sx = sx;
@@ -492,7 +508,7 @@ cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* w
                      : launch_small_t<QL_FP8_E4M3_BLOCK128, 32>(p, tw, tx, grid, st);
   }
   if (e != cudaSuccess) return e;
-  if (dbg && (dbg->qx || dbg->sx)) {
+  if (dbg && !pre_qx && (dbg->qx || dbg->sx)) {
     // debug capture of the quantized tokens (stream-ordered device copies)
     if (dbg->qx && (e = cudaMemcpyAsync(dbg->qx, qx, (size_t)(M * K), cudaMemcpyDeviceToDevice, st)) != cudaSuccess)
       return e;

@@ -65,13 +65,24 @@ constexpr int64_t kGemvMaxKWO = 16384;          // weight-only: 2K bytes of stag
 constexpr int kGemvUnits = 16;                  // units per stage (the MMA's 16 A rows)
 constexpr int kGemvSwCache = 2048;              // row scales kept in shared memory
 constexpr uint32_t kBarConsumers = 1;           // named barrier of the consumer warps
+constexpr int kGemvMaxGroup = QL_GEMV_MAX_GROUP;  // products of one grouped launch
 
-struct GemvParams {
-  const uint16_t* x;
+// One product of a launch.  A grouped launch runs up to kGemvMaxGroup
+// products of the same K side by side, each on its own set of CTAs.
+struct GemvProblem {
+  const uint16_t* x;   // bf16 input, or (when sx is set) its codes as the producer of x wrote them
+  const float* sx;     // pre-quantized input: its scales ([1] or [K/128]); null: quantize x here
   const uint8_t* wq;
   const float* sw;
   uint16_t* y;
-  int64_t N, K;
+  int64_t N;
+};
+
+struct GemvParams {
+  GemvProblem prob[kGemvMaxGroup];
+  int cta0[kGemvMaxGroup + 1];  // CTAs [cta0[j], cta0[j+1]) run product j
+  int nprob;
+  int64_t K;
   int M;               // tokens: 1 to 4 (extra tokens ride on the MMA's B columns)
   int rows_per_stage;  // 2 kRs whole rows per ring stage (kRs = 1, 2 or 4: the kernel's template)
   int stage_bytes;     // R_s * K rounded up to 128
@@ -79,6 +90,7 @@ struct GemvParams {
   int64_t seg_len;     // bytes per unit segment: ceil(K R_s / 8) rounded up to 128
   ql_debug dbg;
   DevStatus* status;
+  int stall;  // test hook: the producer issues no copies, so every consumer wait runs out
 };
 
 struct GemvSmemLayout {
@@ -177,16 +189,41 @@ template <ql_scheme kScheme, int kRs, int kMaxSteps, int kM, bool kWO = false>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams p) {
   // kM tokens x kQ = 8 / kRs segment classes must fit the 8 B columns
   static_assert(kM == 1 || (kM * (8 / kRs) <= 8 && kRs >= 2), "tokens do not fit the B columns");
-  static_assert(!kWO || kM == 1, "the weight-only product takes one token");
   constexpr bool kInt8 = kScheme == QL_W8A8_INT8_ROW;
   constexpr bool kBlock = kScheme == QL_FP8_E4M3_BLOCK128;
   constexpr bool kIntAcc = kInt8 && !kWO;  // exact int32 sums on s8 MMAs
 
   extern __shared__ __align__(1024) uint8_t smem[];
-  const int64_t N = p.N, K = p.K;
-  const int G = gridDim.x;
-  const int64_t row_begin = ((int64_t)blockIdx.x * N) / G;
-  const int64_t row_end = ((int64_t)(blockIdx.x + 1) * N) / G;
+  // The product this CTA runs and its place among that product's CTAs
+  // (constant-index parameter reads and selects: no local copy of the table).
+  int pj = 0;
+#pragma unroll
+  for (int j = 1; j < kGemvMaxGroup; ++j)
+    if (j < p.nprob && (int)blockIdx.x >= p.cta0[j]) pj = j;
+  const uint16_t* px = p.prob[0].x;
+  const float* psx = p.prob[0].sx;
+  const uint8_t* pwq = p.prob[0].wq;
+  const float* psw = p.prob[0].sw;
+  uint16_t* py = p.prob[0].y;
+  int64_t N = p.prob[0].N;
+  int cta_lo = p.cta0[0], cta_hi = p.cta0[1];
+#pragma unroll
+  for (int j = 1; j < kGemvMaxGroup; ++j)
+    if (j == pj) {
+      px = p.prob[j].x;
+      psx = p.prob[j].sx;
+      pwq = p.prob[j].wq;
+      psw = p.prob[j].sw;
+      py = p.prob[j].y;
+      N = p.prob[j].N;
+      cta_lo = p.cta0[j];
+      cta_hi = p.cta0[j + 1];
+    }
+  const int64_t K = p.K;
+  const int G = cta_hi - cta_lo;               // this product's CTAs
+  const int bid = (int)blockIdx.x - cta_lo;    // this CTA among them
+  const int64_t row_begin = ((int64_t)bid * N) / G;
+  const int64_t row_end = ((int64_t)(bid + 1) * N) / G;
   const int64_t KB = K / 128;
   // weight scales this CTA needs: its rows (row schemes) or its 128-row blocks
   const int64_t sw_first = kBlock ? (row_begin >> 7) * KB : row_begin;
@@ -235,7 +272,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 
   if (warp == kGemvWarps) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && !p.stall) {
       const uint64_t policy = l2_policy_evict_first();
       int issued = 0;
       for (int i = 0; i < nstages; ++i) {
@@ -257,7 +294,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         const int64_t nr = stage_rows(i);
         const uint32_t bytes = (uint32_t)(nr * K);
         mbar_arrive_expect_tx(&full[slot], bytes);
-        bulk_g2s(ring + slot * p.stage_bytes, p.wq + r0 * K, bytes, &full[slot], policy);
+        bulk_g2s(ring + slot * p.stage_bytes, pwq + r0 * K, bytes, &full[slot], policy);
         issued = i + 1;
       }
       // Drain: no copy may still be writing this CTA's shared memory when it
@@ -271,13 +308,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 
   // -------------------------------------------------------------- consumers
   // 0. The CTA's weight scales into shared memory (immutable inputs: no wait).
-  for (int i = tid; i < sw_cached; i += kGemvConsumers) sw_s[i] = __ldg(p.sw + sw_first + i);
+  for (int i = tid; i < sw_cached; i += kGemvConsumers) sw_s[i] = __ldg(psw + sw_first + i);
 
   tc::grid_dependency_wait();  // x may be produced by the previous kernel
   // 1. Fused activation quantization of x [kM, K] into shared memory: one pass
   //    for the absmax (the first kXLoads chunks per thread loaded together),
   //    one for the codes (x is L2-resident by then).
-  if constexpr (kWO) {
+  if constexpr (kWO && kM == 1) {
     // Weight-only: x is not quantized.  The MMAs run on f16, so x is staged
     // as x * 2^e in f16, e the power of two that puts the token's absmax in
     // [2^14, 2^15): a bf16 significand (8 bits) fits f16's 11, so every element
@@ -286,7 +323,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     // are exact in f32; the epilogue multiplies the sums by 2^-e (exact).
     const int64_t nchunk8 = K / 8;  // 16-byte chunks of 8 bf16
     constexpr int kXLoads = 8;
-    const uint4* xg = reinterpret_cast<const uint4*>(p.x);
+    const uint4* xg = reinterpret_cast<const uint4*>(px);
     uint4* stash = nst > kEarlyStages && (int64_t)p.stage_bytes >= nchunk8 * 16
                        ? reinterpret_cast<uint4*>(ring + kEarlyStages * p.stage_bytes)
                        : nullptr;
@@ -331,13 +368,74 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     for (int64_t b = 2 * K + tid * 16; b < 2 * ((K + 63) / 64 * 64); b += kGemvConsumers * 16)
       *reinterpret_cast<uint4*>(qx_s + b) = make_uint4(0, 0, 0, 0);
     named_bar_sync(kBarConsumers, kGemvConsumers);
+  } else if constexpr (kWO) {
+    // Weight-only, kM tokens side by side: one absmax pass and one staging
+    // pass for all of them, each token with its own power of two.  Padding
+    // tokens (past p.M) read nothing and stage zeros.
+    const int nchunk8 = (int)(K / 8);
+    const uint4* xg = reinterpret_cast<const uint4*>(px);  // token tok at tok * nchunk8
+    const int64_t xs2 = 2 * xstride;                        // bytes between staged tokens
+    float amax[kM];
+#pragma unroll
+    for (int tok = 0; tok < kM; ++tok) amax[tok] = 0.0f;
+    for (int c = tid; c < nchunk8; c += kGemvConsumers) {
+#pragma unroll
+      for (int tok = 0; tok < kM; ++tok) {
+        const uint4 v = tok < p.M ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
+        amax[tok] = fmaxf(amax[tok], absmax_chunk8(v));
+      }
+    }
+#pragma unroll
+    for (int tok = 0; tok < kM; ++tok) {
+      const float a = warp_max(amax[tok]);
+      if (lane == 0) blockred[tok * kGemvWarps + warp] = a;
+    }
+    named_bar_sync(kBarConsumers, kGemvConsumers);
+    float up[kM];
+    const int sx_per_tok = kBlock ? (int)KB : 1;  // block scheme: one scale per group
+#pragma unroll
+    for (int tok = 0; tok < kM; ++tok) {
+      float a = blockred[tok * kGemvWarps];
+#pragma unroll
+      for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, blockred[tok * kGemvWarps + w]);
+      int e2 = 126;
+      const int ea = (int)((__float_as_uint(a) >> 23) & 0xFFu);
+      if (ea != 0) e2 = min(126, 14 - (ea - 127));
+      up[tok] = __uint_as_float((uint32_t)(127 + e2) << 23);
+      const float down = __uint_as_float((uint32_t)(127 - e2) << 23);
+      for (int i = tid; i < sx_per_tok; i += kGemvConsumers) sx_s[tok * sx_per_tok + i] = down;
+    }
+#pragma unroll 1
+    for (int c = tid; c < nchunk8; c += kGemvConsumers) {
+#pragma unroll
+      for (int tok = 0; tok < kM; ++tok) {
+        const uint4 v = tok < p.M ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
+        const float u = up[tok];
+        reinterpret_cast<uint4*>(qx_s + tok * xs2)[c] =
+            make_uint4(f32x2_to_f16x2(bf16_lo(v.x) * u, bf16_hi(v.x) * u),
+                       f32x2_to_f16x2(bf16_lo(v.y) * u, bf16_hi(v.y) * u),
+                       f32x2_to_f16x2(bf16_lo(v.z) * u, bf16_hi(v.z) * u),
+                       f32x2_to_f16x2(bf16_lo(v.w) * u, bf16_hi(v.w) * u));
+      }
+    }
+    // zero the padding of each token's last 64-element window
+    for (int tok = 0; tok < kM; ++tok)
+      for (int64_t b = 2 * K + tid * 16; b < 2 * ((K + 63) / 64 * 64); b += kGemvConsumers * 16)
+        *reinterpret_cast<uint4*>(qx_s + tok * xs2 + b) = make_uint4(0, 0, 0, 0);
+    named_bar_sync(kBarConsumers, kGemvConsumers);
   } else if constexpr (kM == 1) {
     const int64_t nchunk8 = K / 8;  // 16-byte chunks of 8 bf16
     constexpr int kXLoads = 8;
-    const uint4* xg = reinterpret_cast<const uint4*>(p.x);
+    const uint4* xg = reinterpret_cast<const uint4*>(px);
     uint8_t* qx_t = qx_s;
     float* sx_t = sx_s;
-    if (kBlock) {
+    if (psx) {
+      // Pre-quantized input (the producer of x wrote its codes and scales):
+      // the codes go to shared memory as they are.
+      const uint4* qg = reinterpret_cast<const uint4*>(px);
+      for (int64_t c = tid; c < K / 16; c += kGemvConsumers) reinterpret_cast<uint4*>(qx_t)[c] = __ldg(qg + c);
+      for (int i = tid; i < (kBlock ? (int)KB : 1); i += kGemvConsumers) sx_t[i] = __ldg(psx + i);
+    } else if (kBlock) {
       // 16 consecutive chunks (lanes) form one 128-wide group: no CTA barrier
       for (int64_t base = 0; base < nchunk8; base += kGemvConsumers) {
         const int64_t c = base + tid;
@@ -413,7 +511,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     // them, every token's loads in flight together.  Padding tokens (past
     // p.M) read nothing and get zero codes and scales.
     const int nchunk8 = (int)(K / 8);  // 16-byte chunks of 8 bf16 per token
-    const uint4* xg = reinterpret_cast<const uint4*>(p.x);  // token tok at tok * nchunk8
+    const uint4* xg = reinterpret_cast<const uint4*>(px);  // token tok at tok * nchunk8
     if constexpr (kBlock) {
       // flat chunk f = tok * nchunk8 + c; 16 consecutive chunks (lanes) form
       // one 128-wide group of one token (K % 128 == 0)
@@ -515,7 +613,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     named_bar_sync(kBarConsumers, kGemvConsumers);
   }
   if (tid == 0) mbar_arrive(xready);  // the producer may fill the whole ring now
-  if (!kWO && blockIdx.x == 0 && (p.dbg.qx || p.dbg.sx)) {
+  if (!kWO && blockIdx.x == 0 && (p.dbg.qx || p.dbg.sx)) {  // product 0's first CTA
     // [token, K] codes and [token, groups] scales; rows of K bytes (K % 16 == 0)
     const int ns = kBlock ? (int)KB : 1;
     for (int64_t c = tid; c < (kM == 1 ? 1 : p.M) * (K / 16); c += kGemvConsumers) {
@@ -587,7 +685,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     for (int s = 0; s < kMaxSteps; ++s) {
       const int64_t off = (int64_t)((st0 + s) ^ flip) * 64 + t * 16;
       const bool v = s < nsteps && off < ulen;
-      const uint8_t* src = qx_s + 2 * ((int64_t)uq * seg + off);
+      const uint8_t* src = qx_s + 2 * (xtok * xstride + (int64_t)uq * seg + off);
       const uint4 lo = v ? ld_s128(src) : make_uint4(0, 0, 0, 0);
       const uint4 hi = v ? ld_s128(src + 16) : make_uint4(0, 0, 0, 0);
       xh[s][0] = lo.x, xh[s][1] = lo.y, xh[s][2] = lo.z, xh[s][3] = lo.w;
@@ -683,8 +781,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         const float p0 = __uint_as_float(e ? d[0][1] : d[0][0]) + __uint_as_float(e ? d[1][1] : d[1][0]);
         const float p1 = __uint_as_float(e ? d[0][3] : d[0][2]) + __uint_as_float(e ? d[1][3] : d[1][2]);
         const int64_t grp = min(grp0 + m, KB - 1);
-        const float sw0 = blk0 + grp < sw_cached ? sw_s[blk0 + grp] : __ldg(p.sw + sw_first + blk0 + grp);
-        const float sw1 = blk1 + grp < sw_cached ? sw_s[blk1 + grp] : __ldg(p.sw + sw_first + blk1 + grp);
+        const float sw0 = blk0 + grp < sw_cached ? sw_s[blk0 + grp] : __ldg(psw + sw_first + blk0 + grp);
+        const float sw1 = blk1 + grp < sw_cached ? sw_s[blk1 + grp] : __ldg(psw + sw_first + blk1 + grp);
         res0 = fmaf(p0, sxr[m] * sw0, res0);
         res1 = fmaf(p1, sxr[m] * sw1, res1);
       }
@@ -744,7 +842,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
             yv = vf;
           } else {
             const int64_t si = n - row_begin;
-            const float swn = si < sw_cached ? sw_s[si] : __ldg(p.sw + n);
+            const float swn = si < sw_cached ? sw_s[si] : __ldg(psw + n);
             const float sxt = kM == 1 ? sx_tok : sx_s[otok];
             if constexpr (kIntAcc) {
               if (p.dbg.acc_i32) p.dbg.acc_i32[o] = vi;
@@ -754,7 +852,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
               yv = __fmul_rn(__fmul_rn(vf, sxt), swn);
             }
           }
-          p.y[o] = f32_to_bf16_rn(yv);
+          py[o] = f32_to_bf16_rn(yv);
         }
       }
       __syncwarp();
@@ -806,11 +904,21 @@ static cudaError_t launch_gemv_t(const GemvParams& p, int grid, size_t smem, cud
   }
 }
 
-// Weight-only: one token, the same stage shapes (K <= 16384: at most 32
-// windows per unit, so 4 steps per warp).
+// Weight-only: the stage shapes of the quantized GEMV for the same token count.
 template <ql_scheme S>
 static cudaError_t launch_gemv_wo_t(const GemvParams& p, int grid, size_t smem, cudaStream_t st) {
-  if (p.seg_len > 32 * 64) return cudaErrorInvalidValue;
+  const bool long_units = p.seg_len > 32 * 64;
+  if (p.M > 2)
+    return long_units ? launch_gemv_r<S, 4, 8, 4, true>(p, grid, smem, st)
+                      : launch_gemv_r<S, 4, 4, 4, true>(p, grid, smem, st);
+  if (p.M == 2) {
+    if (p.rows_per_stage == 8)
+      return long_units ? launch_gemv_r<S, 4, 8, 2, true>(p, grid, smem, st)
+                        : launch_gemv_r<S, 4, 4, 2, true>(p, grid, smem, st);
+    return long_units ? launch_gemv_r<S, 2, 8, 2, true>(p, grid, smem, st)
+                      : launch_gemv_r<S, 2, 4, 2, true>(p, grid, smem, st);
+  }
+  if (long_units) return cudaErrorNotSupported;  // one token: K <= 16384 keeps units short
   switch (p.rows_per_stage / 2) {
     case 1: return launch_gemv_r<S, 1, 4, 1, true>(p, grid, smem, st);
     case 2: return launch_gemv_r<S, 2, 4, 1, true>(p, grid, smem, st);
@@ -823,12 +931,17 @@ int gemv_max_k_tokens(int64_t M) {
   return M == 1 ? (int)kGemvMaxK : M == 2 ? (int)kGemvMaxK2 : M <= 4 ? (int)kGemvMaxK4 : 0;
 }
 
-// Stage shape, ring depth and grid for M tokens (xelem: bytes per staged x
-// element).  Returns cudaErrorInvalidValue / InvalidConfiguration for shapes
-// the kernel does not take.
-static cudaError_t gemv_setup(GemvParams& p, int64_t M, int64_t N, int64_t K, int xelem,
-                              int num_sms, int* grid, size_t* smem) {
-  p.N = N;
+// Stage shape, ring depth and CTA split for `count` products of M tokens and
+// K inputs (xelem: bytes per staged x element).  The SMs are shared out so
+// that the largest number of weight rows any CTA streams is as small as it
+// can be (one CTA at a time to the product whose CTAs carry the most rows;
+// no product gets more CTAs than it has ring stages).  Returns
+// cudaErrorInvalidValue / InvalidConfiguration for shapes the kernel does not
+// take.
+static cudaError_t gemv_setup(GemvParams& p, int64_t M, const ql_gemv_problem* probs, int count,
+                              int64_t K, int xelem, int num_sms, int* grid, size_t* smem) {
+  if (count < 1 || count > kGemvMaxGroup) return cudaErrorInvalidValue;
+  p.nprob = count;
   p.K = K;
   p.M = (int)M;
   // kRs: the largest power of two <= 4 whose stage of 2 kRs rows fits the
@@ -849,54 +962,114 @@ static cudaError_t gemv_setup(GemvParams& p, int64_t M, int64_t N, int64_t K, in
   p.seg_len = ((K + q - 1) / q + 127) / 128 * 128;
   // the kernel keeps at most 64 windows of 64 bytes per unit
   if (p.seg_len > 64 * 64) return cudaErrorInvalidValue;
-  const int64_t stage_rows_total = (N + p.rows_per_stage - 1) / p.rows_per_stage;
-  *grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms, stage_rows_total));
+  int g[kGemvMaxGroup];
+  int64_t cap[kGemvMaxGroup];
+  int used = 0;
+  for (int j = 0; j < count; ++j) {
+    p.prob[j] = GemvProblem{probs[j].x ? probs[j].x : static_cast<const uint16_t*>(probs[j].qx),
+                            probs[j].x ? nullptr : probs[j].sx,
+                            static_cast<const uint8_t*>(probs[j].wq), probs[j].sw, probs[j].y,
+                            probs[j].N};
+    cap[j] = (probs[j].N + p.rows_per_stage - 1) / p.rows_per_stage;
+    g[j] = 1;
+    ++used;
+  }
+  for (; used < num_sms; ++used) {
+    int best = -1;
+    for (int j = 0; j < count; ++j)
+      if (g[j] < cap[j] && (best < 0 || probs[j].N * g[best] > probs[best].N * g[j])) best = j;
+    if (best < 0) break;  // every product has one CTA per ring stage
+    ++g[best];
+  }
+  p.cta0[0] = 0;
+  for (int j = 0; j < kGemvMaxGroup; ++j) p.cta0[j + 1] = p.cta0[j] + (j < count ? g[j] : 0);
+  for (int j = count; j < kGemvMaxGroup; ++j) p.prob[j] = p.prob[0];
+  *grid = p.cta0[count];
   *smem = gemv_layout(K, p.stage_bytes, p.stages, kGemvSwCache, km, xelem).total;
   return cudaSuccess;
 }
 
-cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
-                        int64_t M, int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg,
-                        int num_sms, DevStatus* status, cudaStream_t st) {
-  if (M < 1 || M > 4 || K > gemv_max_k_tokens(M)) return cudaErrorInvalidValue;
-  GemvParams p;
-  p.x = x;
-  p.wq = static_cast<const uint8_t*>(wq);
-  p.sw = sw;
-  p.y = y;
-  int grid = 0;
-  size_t smem = 0;
-  cudaError_t e = gemv_setup(p, M, N, K, 1, num_sms, &grid, &smem);
-  if (e != cudaSuccess) return e;
-  p.dbg = dbg ? *dbg : ql_debug{nullptr, nullptr, nullptr, nullptr};
-  p.status = status;
+template <bool kWO>
+static cudaError_t launch_gemv_scheme(ql_scheme scheme, const GemvParams& p, int grid, size_t smem,
+                                      cudaStream_t st) {
   switch (scheme) {
-    case QL_W8A8_INT8_ROW: return launch_gemv_t<QL_W8A8_INT8_ROW>(p, grid, smem, st);
-    case QL_FP8_E4M3_ROW: return launch_gemv_t<QL_FP8_E4M3_ROW>(p, grid, smem, st);
-    default: return launch_gemv_t<QL_FP8_E4M3_BLOCK128>(p, grid, smem, st);
+    case QL_W8A8_INT8_ROW:
+      return kWO ? launch_gemv_wo_t<QL_W8A8_INT8_ROW>(p, grid, smem, st)
+                 : launch_gemv_t<QL_W8A8_INT8_ROW>(p, grid, smem, st);
+    case QL_FP8_E4M3_ROW:
+      return kWO ? launch_gemv_wo_t<QL_FP8_E4M3_ROW>(p, grid, smem, st)
+                 : launch_gemv_t<QL_FP8_E4M3_ROW>(p, grid, smem, st);
+    default:
+      return kWO ? launch_gemv_wo_t<QL_FP8_E4M3_BLOCK128>(p, grid, smem, st)
+                 : launch_gemv_t<QL_FP8_E4M3_BLOCK128>(p, grid, smem, st);
   }
 }
 
-cudaError_t launch_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const void* wq,
-                                    const float* sw, int64_t N, int64_t K, uint16_t* y,
-                                    int num_sms, DevStatus* status, cudaStream_t st) {
-  if (K > kGemvMaxKWO) return cudaErrorInvalidValue;
+cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
+                        int64_t M, int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg,
+                        int num_sms, DevStatus* status, cudaStream_t st, bool stall) {
+  if (M < 1 || M > 4 || K > gemv_max_k_tokens(M)) return cudaErrorInvalidValue;
+  const ql_gemv_problem one{x, nullptr, nullptr, wq, sw, y, N};
   GemvParams p;
-  p.x = x;
-  p.wq = static_cast<const uint8_t*>(wq);
-  p.sw = sw;
-  p.y = y;
   int grid = 0;
   size_t smem = 0;
-  cudaError_t e = gemv_setup(p, 1, N, K, 2, num_sms, &grid, &smem);
+  cudaError_t e = gemv_setup(p, M, &one, 1, K, 1, num_sms, &grid, &smem);
+  if (e != cudaSuccess) return e;
+  p.dbg = dbg ? *dbg : ql_debug{nullptr, nullptr, nullptr, nullptr};
+  p.status = status;
+  p.stall = stall ? 1 : 0;
+  return launch_gemv_scheme<false>(scheme, p, grid, smem, st);
+}
+
+cudaError_t launch_gemv_grouped(ql_scheme scheme, const ql_gemv_problem* probs, int count,
+                                int64_t K, int num_sms, DevStatus* status, cudaStream_t st) {
+  if (K > gemv_max_k()) return cudaErrorInvalidValue;
+  GemvParams p;
+  int grid = 0;
+  size_t smem = 0;
+  cudaError_t e = gemv_setup(p, 1, probs, count, K, 1, num_sms, &grid, &smem);
   if (e != cudaSuccess) return e;
   p.dbg = ql_debug{nullptr, nullptr, nullptr, nullptr};
   p.status = status;
-  switch (scheme) {
-    case QL_W8A8_INT8_ROW: return launch_gemv_wo_t<QL_W8A8_INT8_ROW>(p, grid, smem, st);
-    case QL_FP8_E4M3_ROW: return launch_gemv_wo_t<QL_FP8_E4M3_ROW>(p, grid, smem, st);
-    default: return launch_gemv_wo_t<QL_FP8_E4M3_BLOCK128>(p, grid, smem, st);
+  p.stall = 0;
+  return launch_gemv_scheme<false>(scheme, p, grid, smem, st);
+}
+
+int gemv_weight_only_max_k_tokens(int64_t M) {
+  // the largest K (a multiple of 16) whose staged f16 tokens and two ring
+  // stages fit the shared memory, found once per token count
+  static int cache[5] = {-1, -1, -1, -1, -1};
+  if (M < 1 || M > 4) return 0;
+  if (cache[M] < 0) {
+    int best = 0;
+    for (int64_t K = 16; K <= kGemvMaxKWO; K += 16) {
+      GemvParams p;
+      int grid = 0;
+      size_t smem = 0;
+      const ql_gemv_problem one{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 128};
+      if (gemv_setup(p, M, &one, 1, K, 2, 148, &grid, &smem) == cudaSuccess &&
+          (M > 1 || p.seg_len <= 32 * 64))
+        best = (int)K;
+    }
+    cache[M] = best;
   }
+  return cache[M];
+}
+
+cudaError_t launch_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const void* wq,
+                                    const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                    int num_sms, DevStatus* status, cudaStream_t st) {
+  if (M < 1 || M > 4 || K > kGemvMaxKWO) return cudaErrorNotSupported;
+  const ql_gemv_problem one{x, nullptr, nullptr, wq, sw, y, N};
+  GemvParams p;
+  int grid = 0;
+  size_t smem = 0;
+  // the staged f16 tokens and two ring stages must fit the shared memory
+  if (gemv_setup(p, M, &one, 1, K, 2, num_sms, &grid, &smem) != cudaSuccess) return cudaErrorNotSupported;
+  p.dbg = ql_debug{nullptr, nullptr, nullptr, nullptr};
+  p.status = status;
+  p.stall = 0;
+  return launch_gemv_scheme<true>(scheme, p, grid, smem, st);
 }
 
 }  // namespace ql

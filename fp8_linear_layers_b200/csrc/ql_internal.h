@@ -45,32 +45,54 @@ cudaError_t launch_quantize_weight(ql_scheme scheme, const uint16_t* w, int64_t 
 int gemv_max_k();
 int gemv_max_k_tokens(int64_t M);  // largest K the GEMV takes for M tokens (0: none)
 // M = 1 to 4 tokens (extra tokens ride on the MMA's B columns at no extra weight traffic).
+// stall: test hook, the producer issues no copies (every consumer wait runs out).
 cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
                         int64_t M, int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg,
-                        int num_sms, DevStatus* status, cudaStream_t st);
-// M = 1 weight-only product: x stays bf16 (staged as exactly scaled f16), W codes
-// dequantized to f16 in registers, f32 sums; K <= gemv_weight_only_max_k().
+                        int num_sms, DevStatus* status, cudaStream_t st, bool stall = false);
+// Up to QL_GEMV_MAX_GROUP M = 1 products of the same K in one launch.
+cudaError_t launch_gemv_grouped(ql_scheme scheme, const ql_gemv_problem* probs, int count,
+                                int64_t K, int num_sms, DevStatus* status, cudaStream_t st);
+// 1 <= M <= 4 weight-only product: x stays bf16 (staged as exactly scaled f16),
+// W codes dequantized to f16 in registers, f32 sums; K <= gemv_weight_only_max_k().
+// Returns cudaErrorNotSupported for shapes whose staged tokens and two ring
+// stages do not fit the shared memory.
 int gemv_weight_only_max_k();
+// largest K the weight-only GEMV takes for M (1..4) tokens (0: none)
+int gemv_weight_only_max_k_tokens(int64_t M);
+// 1 <= M <= 32 weight-only product: the GEMV kernel up to four tokens (within
+// its K limits), else tcgen05 kind::f16 with the weights converted to bf16.
+size_t gemm_small_wo_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K);
+size_t gemm_small_wo_zeroed_bytes(int64_t M, int64_t N);
+cudaError_t launch_gemm_small_wo(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
+                                 int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
+                                 size_t ws_bytes, int num_sms, DevStatus* status, cudaStream_t st);
 cudaError_t launch_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const void* wq,
-                                    const float* sw, int64_t N, int64_t K, uint16_t* y,
+                                    const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
                                     int num_sms, DevStatus* status, cudaStream_t st);
 
 // Large-M tcgen05 GEMM on pre-quantized activations.
 size_t gemm_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);
+// qy / sy (block scheme only): also write y's E4M3 codes [M,N] and per-128
+// scales [M,N/128]; y may then be null.
 cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
                         const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
                         void* workspace, size_t ws_bytes, const ql_debug* dbg, int num_sms,
-                        DevStatus* status, cudaStream_t st);
+                        DevStatus* status, cudaStream_t st, uint8_t* qy = nullptr,
+                        float* sy = nullptr);
 
 // Small-M (1..32) tensor-core GEMM, K split across the SMs.
 size_t gemm_small_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);
-// Byte offset of the arrival counters inside that workspace (they run to its end).
-// Bytes at the start of the workspace that must be zero when a call starts
-// (split-tile arrival counters and sums); a completed call leaves them zero.
+// Bytes at the start of that workspace that must be zero when a call starts
+// (split-tile arrival counters, then the atomic-sum slot of every tile); a
+// completed call leaves them zero.  0 when the shape runs on the GEMV kernel,
+// which does not use the workspace.
 size_t gemm_small_zeroed_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);
+// pre_qx / pre_sx: the input already quantized (x unused; no quantization
+// launch and no GEMV route).
 cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq,
                               const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
                               void* workspace, size_t ws_bytes, const ql_debug* dbg, int num_sms,
-                              DevStatus* status, cudaStream_t st);
+                              DevStatus* status, cudaStream_t st, const uint8_t* pre_qx = nullptr,
+                              const float* pre_sx = nullptr);
 
 }  // namespace ql

@@ -26,6 +26,14 @@ __host__ __device__ constexpr uint32_t idesc(bool int8, int m, int n) {
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
+// ---- instruction descriptor (kind::f16: bf16 x bf16 -> f32, dense, K-major A and B)
+//  bits [4,6)   D format: 1 = f32
+//  bits [7,10)  A format: 1 = bf16;  bits [10,13) B format: 1 = bf16
+//  bits [17,23) N >> 3;  bits [24,29) M >> 4
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
 // ---- shared-memory matrix descriptor: K-major tile of 128-byte rows written
 // by TMA with the 128-byte swizzle; 8-row groups are 1024 bytes apart.
 //  bits [0,14)  start address >> 4
@@ -60,6 +68,15 @@ QL_DEVINL void commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T with bf16 operands (kind::f16), K = 16 elements.
+QL_DEVINL void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t id, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(id), "r"(accumulate)
+      : "memory");
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, one instruction covers K = 32 bytes.

@@ -135,6 +135,55 @@ ql_status qlinear_quantize_act(ql_scheme scheme, const uint16_t* x, int64_t M, i
 ql_status qlinear_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
                        int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg, void* stream);
 
+/* Several M = 1 products with the same K in one launch: each product keeps
+ * its own input, weights, scales and output (e.g. a layer's q, k and v
+ * projections of one normalised input, or gate and up), and the numerics of
+ * each are those of qlinear_gemv, bit for bit.  Pages: the same as
+ * qlinear_gemv (W8A8 and Qwen3 FP8 "Loading": one row in a kernel that reads
+ * each weight byte once); a decode step runs a layer's projections that read
+ * one input side by side (W8A8 "Against bf16": decoding under CUDA graphs).
+ * The SMs are shared out in proportion to the products' weight bytes, each
+ * CTA streaming one product.
+ *   problems  host array of `count` descriptors, 1 <= count <=
+ *             QL_GEMV_MAX_GROUP (read during the call only):
+ *               x   device, bf16 [1,K] (products may share one x); or NULL
+ *                   when the input comes already quantized:
+ *               qx, sx  device, the input's codes [1,K] and scales ([1] or
+ *                   [K/128]) as qlinear_quantize_act (or a producer kernel)
+ *                   writes them; ignored when x is set
+ *               wq  device, [N,K] codes;  sw  device, the matching scales
+ *               y   device, out: bf16 [1,N] (outputs must not overlap)
+ *               N   output rows (> 0; a multiple of 128 for the block scheme)
+ * Errors: argument checks as for qlinear_gemv on every product; count outside
+ * [1, QL_GEMV_MAX_GROUP] -> QL_ERR_INVALID_ARG. */
+#define QL_GEMV_MAX_GROUP 8
+typedef struct ql_gemv_problem {
+  const uint16_t* x;
+  const void* qx;
+  const float* sx;
+  const void* wq;
+  const float* sw;
+  uint16_t* y;
+  int64_t N;
+} ql_gemv_problem;
+
+ql_status qlinear_gemv_grouped(ql_scheme scheme, const ql_gemv_problem* problems, int count,
+                               int64_t K, void* stream);
+
+/* M = 1 product on an input that its producer has already quantized (the
+ * activation quantization moved out of the product's critical path: the
+ * pages blame the prompt's "two kernels a projection" for its lost time,
+ * "Llama 3.1 8B Instruct W8A8", "Against bf16", and the Red Hat W8A8 post
+ * the inter-token latency lost to dynamic activation quantization).  The
+ * kernel reads the codes and scales instead of quantizing x; everything else
+ * is qlinear_gemv, and its output equals qlinear_gemv's on the x those codes
+ * came from.
+ *   qx  device, [1,K] codes;  sx  device, f32 [1] (row schemes) or [K/128]
+ *   wq, sw, y, N, K as for qlinear_gemv
+ * Errors: as for qlinear_gemv. */
+ql_status qlinear_gemv_prequant(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
+                                const float* sw, int64_t N, int64_t K, uint16_t* y, void* stream);
+
 /* M = 1 weight-only product ("equivalent" numerics: W8A16 / FP8 weight-only):
  * the activations are not rounded, only the weights are quantized,
  *   y[n] = bf16_rne( sum_k x[k] * (q_w[n,k] * s_w) ),
@@ -157,6 +206,29 @@ ql_status qlinear_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, cons
 ql_status qlinear_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const void* wq,
                                    const float* sw, int64_t N, int64_t K, uint16_t* y,
                                    void* stream);
+
+/* Weight-only product for 1 <= M <= 32 tokens (the numerics of
+ * qlinear_gemv_weight_only, token by token: x not rounded, f32 sums, then the
+ * weight scale; tolerance |y - y_exact| <= 2^-7 |y_exact| + 1e-3).  Same
+ * pages as qlinear_gemv_weight_only; the W8A8 and Qwen3 FP8 pages run up to
+ * 32 tokens on the tensor cores ("Loading").  Up to four tokens ride on the
+ * weight-only GEMV kernel's spare MMA columns (K up to 16384 for one token,
+ * 15744 for two, 7584 for three or four: the staged f16 tokens and two
+ * weight stages must fit the shared memory); other shapes run on the tensor
+ * cores (tcgen05 kind::f16: the codes are converted exactly to bf16 in
+ * shared memory and multiplied with the bf16 x, K split across the SMs).
+ *   x          device, bf16 [M,K];  y  device, out: bf16 [M,N]
+ *   workspace  device, qlinear_weight_only_workspace_bytes(scheme, M, N, K)
+ *              bytes (0: none needed, NULL allowed), 256-byte aligned,
+ *              ZERO-FILLED before its first use; a completed call leaves it
+ *              ready for the next call of the same shape (as for
+ *              qlinear_gemm_small).  Calls in flight together must not share it.
+ * Errors: argument checks as above; M = 0 is a no-op; M > 32 ->
+ * QL_ERR_UNSUPPORTED_SHAPE; a missing or small workspace -> QL_ERR_WORKSPACE. */
+ql_status qlinear_forward_weight_only(ql_scheme scheme, const uint16_t* x, const void* wq,
+                                      const float* sw, int64_t M, int64_t N, int64_t K,
+                                      uint16_t* y, void* workspace, size_t ws_bytes, void* stream);
+size_t qlinear_weight_only_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K);
 
 /* 1 <= M <= 32 product on the tensor cores (tcgen05, tokens on the MMA N side,
  * weights on the 128-row side, K split across the SMs).  Up to four tokens
@@ -181,6 +253,22 @@ ql_status qlinear_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const vo
 ql_status qlinear_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
                              int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
                              size_t ws_bytes, const ql_debug* dbg, void* stream);
+
+/* qlinear_gemm_small on an input its producer has already quantized (no
+ * quantization launch in the call: one kernel per projection; pages as for
+ * qlinear_gemv_prequant).  The tensor-core path runs for every 1 <= M <= 32.
+ *   qx, sx     device, [M,K] codes and f32 scales ([M] or [M,K/128]) as
+ *              qlinear_quantize_act writes them
+ *   workspace  as for qlinear_gemm_small (the same size; its quantized-token
+ *              part is not used)
+ * The output equals qlinear_gemm_small's on the x those codes came from (for
+ * int8 bit for bit; E4M3 sums of split tiles may differ in the last bits with
+ * the order in which their parts are added, within the output tolerance).
+ * Errors: as for qlinear_gemm_small. */
+ql_status qlinear_gemm_small_prequant(ql_scheme scheme, const void* qx, const float* sx,
+                                      const void* wq, const float* sw, int64_t M, int64_t N,
+                                      int64_t K, uint16_t* y, void* workspace, size_t ws_bytes,
+                                      void* stream);
 
 /* Large-M product on pre-quantized activations (tcgen05 kind::i8 into int32
  * TMEM accumulators, or kind::f8f6f4 E4M3 into f32; TMA-fed shared-memory
@@ -208,6 +296,26 @@ ql_status qlinear_gemm(ql_scheme scheme, const void* qx, const float* sx, const 
                        const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
                        void* workspace, size_t ws_bytes, const ql_debug* dbg, void* stream);
 
+/* qlinear_gemm (block scheme) whose epilogue also quantizes its own output
+ * for the product that reads it next: the E4M3 codes of y and one f32 scale
+ * per token per 128 outputs, exactly what qlinear_quantize_act writes for
+ * the bf16 y (s = absmax / 448 over the 128 bf16 outputs, one IEEE division;
+ * code = E4M3(y / s)).  A 128-wide output group lies inside one output tile,
+ * so no cross-tile reduction is needed, and the next product runs without a
+ * quantization launch of its own ("Llama 3.1 8B Instruct W8A8", "Against
+ * bf16": "two kernels a projection"; "Qwen3 8B FP8", "Loading": activations
+ * in groups of 128).
+ *   y       device, out: bf16 [M,N], or NULL to write only the codes
+ *   qy      device, out: [M,N] E4M3 codes
+ *   sy      device, out: f32 [M, N/128]
+ *   other arguments as for qlinear_gemm
+ * Errors: as for qlinear_gemm; a row scheme -> QL_ERR_UNSUPPORTED_SHAPE (its
+ * per-token scale spans every output tile). */
+ql_status qlinear_gemm_quant_out(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
+                                 const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                 void* qy, float* sy, void* workspace, size_t ws_bytes,
+                                 void* stream);
+
 /* The projection as a model calls it: bf16 X in, bf16 Y out, dispatching on
  * the token count the way the pages' "Loading" sections describe: M = 1 ->
  * qlinear_gemv, 2..32 -> qlinear_gemm_small, > 32 -> qlinear_quantize_act
@@ -224,6 +332,15 @@ ql_status qlinear_forward(ql_scheme scheme, const uint16_t* x, const void* wq, c
  * activations qlinear_forward keeps there for M > 32. */
 size_t qlinear_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K);
 size_t qlinear_forward_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K);
+
+/* Test hook for the timeout path (no counterpart in the pages): qlinear_gemv
+ * with its weight-copy engine held back, so that every consumer's bounded wait
+ * runs out after about 2 s; the kernel records QL_ERR_TIMEOUT (detail: the
+ * GEMV's kernel id << 8 | wait site) and returns without writing y.  The
+ * context stays usable.  Arguments as for qlinear_gemv. */
+ql_status qlinear_debug_gemv_stalled(ql_scheme scheme, const uint16_t* x, const void* wq,
+                                     const float* sw, int64_t N, int64_t K, uint16_t* y,
+                                     void* stream);
 
 /* Synchronises `stream`, then reads and clears the device status word that
  * kernels set when a bounded wait gives up.  Returns QL_OK, QL_ERR_TIMEOUT

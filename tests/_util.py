@@ -35,3 +35,36 @@ def assert_y_close(y_gpu_bits: np.ndarray, y_ref_bits: np.ndarray, what=""):
     assert bad[0].size == 0, (f"{what}: {bad[0].size} outputs out of tolerance; first "
                               f"{[(tuple(int(i) for i in idx), g[idx], r[idx]) for idx in zip(*bad)][:5]}")
     return float(err.max()) if err.size else 0.0
+
+
+def oracle_forward_par(scheme: int, x: np.ndarray, wq: np.ndarray, sw: np.ndarray, chunks: int = 0):
+    """oracle.forward split over output-row ranges on threads (the oracle's C
+    calls release the GIL), for full-size layers.  Block-scheme ranges are
+    whole 128-row blocks.  The same values as oracle.forward."""
+    import concurrent.futures
+    import os
+    qx, sx = oracle.quantize_act(scheme, x)
+    N = wq.shape[0]
+    chunks = chunks or min(32, os.cpu_count() or 4)
+    step = -(-N // chunks)
+    if scheme == oracle.FP8_BLOCK:
+        step = -(-step // 128) * 128
+    bounds = [(n0, min(N, n0 + step)) for n0 in range(0, N, step)]
+    with concurrent.futures.ThreadPoolExecutor(max_workers=len(bounds)) as ex:
+        parts = list(ex.map(lambda b: oracle.linear_rows(scheme, qx, sx, wq, sw, b[0], b[1]), bounds))
+    return np.concatenate(parts, axis=1)
+
+
+def oracle_wo_par(scheme: int, x: np.ndarray, wq: np.ndarray, sw: np.ndarray, chunks: int = 0):
+    """oracle.linear_weight_only split over output-row ranges on threads."""
+    import concurrent.futures
+    import os
+    N = wq.shape[0]
+    chunks = chunks or min(32, os.cpu_count() or 4)
+    step = -(-N // chunks)
+    if scheme == oracle.FP8_BLOCK:
+        step = -(-step // 128) * 128
+    bounds = [(n0, min(N, n0 + step)) for n0 in range(0, N, step)]
+    with concurrent.futures.ThreadPoolExecutor(max_workers=len(bounds)) as ex:
+        parts = list(ex.map(lambda b: oracle.linear_weight_only(scheme, x, wq, sw, b[0], b[1]), bounds))
+    return np.concatenate(parts, axis=1)

@@ -69,6 +69,32 @@ def test_host_validation_rejects_before_launch(L):
     assert WO(0, ALIGNED, ALIGNED, ALIGNED, 64, 40, ALIGNED, None) == SHAPE
     assert WO(2, ALIGNED, ALIGNED, ALIGNED, 100, 256, ALIGNED, None) == SHAPE
     assert WO(0, ALIGNED, ALIGNED, ALIGNED, 16, 16400, ALIGNED, None) == SHAPE
+    # the grouped GEMV: 1 to QL_GEMV_MAX_GROUP products, each checked as qlinear_gemv
+    import ctypes
+    P = ql._GemvProblem
+    table = (P * 2)(P(ALIGNED, 0, 0, ALIGNED, ALIGNED, ALIGNED, 64), P(ALIGNED, 0, 0, ALIGNED, ALIGNED, ALIGNED, 64))
+    tp = ctypes.cast(table, ctypes.c_void_p)
+    GR = L.qlinear_gemv_grouped
+    assert GR(0, tp, 0, 64, None) == INV
+    assert GR(0, tp, ql.GEMV_MAX_GROUP + 1, 64, None) == INV
+    assert GR(0, None, 1, 64, None) == INV
+    assert GR(7, tp, 2, 64, None) == INV
+    assert GR(0, tp, 2, 40, None) == SHAPE
+    assert GR(2, tp, 2, 256, None) == SHAPE      # N = 64: not a multiple of 128
+    table[1].y = ALIGNED + 4
+    assert GR(0, tp, 2, 64, None) == MIS
+    table[1].y = 0
+    assert GR(0, tp, 2, 64, None) == INV
+    table[1].y, table[1].x = ALIGNED, 0   # no x and no pre-quantized input
+    assert GR(0, tp, 2, 64, None) == INV
+    table[1].qx = ALIGNED
+    assert GR(0, tp, 2, 64, None) == INV  # codes without scales
+    table[1].sx = ALIGNED + 4
+    assert GR(0, tp, 2, 64, None) == MIS
+    PQ = L.qlinear_gemv_prequant
+    assert PQ(0, None, ALIGNED, ALIGNED, ALIGNED, 64, 64, ALIGNED, None) == INV
+    assert PQ(0, ALIGNED, None, ALIGNED, ALIGNED, 64, 64, ALIGNED, None) == INV
+    assert PQ(0, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 64, 40, ALIGNED, None) == SHAPE
     # M = 0 is a no-op that succeeds without a device
     assert L.qlinear_quantize_act(0, None, 0, 64, None, None, None) == 0
     assert L.qlinear_forward(0, None, None, None, 0, 64, 64, None, None, 0, None) == 0

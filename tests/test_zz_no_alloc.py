@@ -57,16 +57,19 @@ def test_noalloc_matches_workspace_entry_point(cuda, scheme, M, N, K):
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(cuda):
-    # 32 tokens x 133120 inputs: the quantized tokens alone take 4.3 MB and the
-    # per-SM partial slots 4.8 MB, more than the fixed 8 MiB scratch
-    M, N, K = 32, 128, 133120
+    # 32 tokens x 65536 outputs (512 tiles of 128 rows): the two partial-sum
+    # slots of 32 x 128 int32 per tile alone take 16.8 MB, more than the fixed
+    # 8 MiB scratch, so the call must refuse before launching anything
+    M, N, K = 32, 65536, 128
+    need = ql.workspace_bytes(ql.W8A8_INT8_ROW, M, N, K)
+    assert need > (8 << 20), need
     x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
     wq = torch.zeros((N, K), dtype=torch.uint8, device="cuda")
     sw = torch.ones(N, dtype=torch.float32, device="cuda")
     y = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
-    if ql.workspace_bytes(ql.W8A8_INT8_ROW, M, N, K) <= (8 << 20):
-        pytest.skip("this device's SM count makes the shape fit")
     st = ql.lib().qlinear_gemm_small_noalloc(ql.W8A8_INT8_ROW, x.data_ptr(), wq.data_ptr(), sw.data_ptr(),
                                              M, N, K, y.data_ptr(), torch.cuda.current_stream().cuda_stream)
-    assert st == 7
+    assert st == 7  # QL_ERR_WORKSPACE
     assert b"static scratch holds" in ql.lib().qlinear_last_cuda_error()
+    assert f"needs {need} bytes".encode() in ql.lib().qlinear_last_cuda_error()
+    assert torch.count_nonzero(y).item() == 0  # nothing ran
