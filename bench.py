@@ -69,6 +69,7 @@ class Product:
     K: int
     outliers: int
     wo: bool = False  # weight-only product (activations not rounded)
+    group: str = ""   # products of one (scheme, group) read one input; M = 1 ones share a launch
 
 
 @dataclass
@@ -102,13 +103,32 @@ class Workload:
         return p.N * p.K + sw + 2 * p.M * p.K + 2 * p.M * p.N
 
 
+# The projections of a decoder layer that read one input: q, k, v (the
+# normalised hidden state) and gate, up (the normalised attention output).
+LAYER_INPUT = {"q_proj": "qkv", "k_proj": "qkv", "v_proj": "qkv", "gate_proj": "gate_up",
+               "up_proj": "gate_up"}
+
+
+def gemv_route(M: int, K: int) -> bool:
+    """True when the library runs an M-token product on the GEMV kernel (one
+    launch): M = 1 up to K = 32768, two tokens up to 16384, three or four up to 8192."""
+    return (M == 1 and K <= 32768) or (M == 2 and K <= 16384) or (M in (3, 4) and K <= 8192)
+
+
 def workloads():
     from fp8_linear_layers_b200 import synthetic as S
     oc = S.outlier_count
     w = {}
     w["decode"] = Workload(
         "decode", "decode GEMV M=1: one Llama-3.1-8B layer's 7 projections (q,k,v,o,gate,up,down) "
-        "in W8A8 int8 and in FP8 E4M3 per-row, per-token dynamic activation quantization fused", "GB/s",
+        "in W8A8 int8 and in FP8 E4M3 per-row, per-token dynamic activation quantization fused; "
+        "the projections that read one input (q|k|v, gate|up) run as one grouped launch each, "
+        "from their own weight buffers: 4 launches per scheme", "GB/s",
+        [Product(n, s, 1, N, K, oc(K), group=LAYER_INPUT.get(n, n))
+         for s in (INT8, FP8R) for n, N, K in S.LLAMA31_8B])
+    w["decode-separate"] = Workload(
+        "decode-separate", "decode GEMV M=1: one Llama-3.1-8B layer's 7 projections in W8A8 int8 and in "
+        "FP8 E4M3 per-row, each its own launch (14 launches per step)", "GB/s",
         [Product(n, s, 1, N, K, oc(K)) for n, N, K in S.LLAMA31_8B for s in (INT8, FP8R)])
     w["decode-fused"] = Workload(
         "decode-fused", "decode GEMV M=1: one Llama-3.1-8B layer with q|k|v and gate|up stored side by "
@@ -132,8 +152,9 @@ def workloads():
         "Llama-3.1-8B layer's 7 projections with int8 and with FP8 E4M3 per-row weights", "GB/s",
         [Product(n, s, 1, N, K, oc(K), wo=True) for n, N, K in S.LLAMA31_8B for s in (INT8, FP8R)])
     w["qwen-decode"] = Workload(
-        "qwen-decode", "Qwen3-8B FP8 128x128-block projections at M=1 (7 shapes)", "GB/s",
-        [Product(n, FP8B, 1, N, K, 0) for n, N, K in S.QWEN3_8B])
+        "qwen-decode", "Qwen3-8B FP8 128x128-block projections at M=1 (7 shapes; q|k|v and gate|up "
+        "one grouped launch each on their shared input)", "GB/s",
+        [Product(n, FP8B, 1, N, K, 0, group=LAYER_INPUT.get(n, n)) for n, N, K in S.QWEN3_8B])
     w["qwen-small"] = Workload(
         "qwen-small", "Qwen3-8B FP8 128x128-block projections at M=32 (7 shapes)", "GB/s",
         [Product(n, FP8B, 32, N, K, 0) for n, N, K in S.QWEN3_8B])
@@ -150,11 +171,13 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["qlinear", "reference"], default="qlinear")
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "decode-fused", "prefill", "small", "kproj", "qwen-decode",
-                             "qwen-small", "qwen-prefill", "decode-wo"])
+                    choices=["decode", "decode-separate", "decode-fused", "prefill", "small", "kproj",
+                             "qwen-decode", "qwen-small", "qwen-prefill", "decode-wo"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only --workload (the default run also times the tensor-bound configs)")
     ap.add_argument("--e2e-steps", type=int, default=None)
     return ap.parse_args()
 
@@ -288,39 +311,59 @@ def measured_traffic(wl):
 class Runner:
     """Device buffers and launch closures for one workload (public API calls only).
 
-    Steps cycle through `copies` independent sets of quantized weights,
-    activations and outputs, enough that the bytes touched by consecutive
-    steps exceed twice the L2: no step finds its inputs in L2 from an earlier
-    one, so no flush is needed between timed steps.
+    Products of one (scheme, group) read one input; M = 1 ones run as one
+    grouped GEMV launch.  Steps cycle through `copies` independent sets of
+    quantized weights, activations and outputs, enough that the bytes touched
+    by consecutive steps exceed twice the L2: no step finds its inputs in L2
+    from an earlier one, so no flush is needed between timed steps.
     """
 
     def __init__(self, torch, ql, synthetic, wl: Workload):
         self.torch, self.ql, self.wl = torch, ql, wl
         per_step = sum(wl.bytes_touched(p) for p in wl.products)
         self.copies = max(2, -(-int(2 * L2_BYTES) // int(per_step)))
-        self.items = []
+        self.groups = []  # [{"p0", "xs", "items"}] in launch order
+        by_key = {}
         weights = {}
-        for p in wl.products:
-            key = (p.name, p.N, p.K)
-            if key not in weights:
-                weights[key] = synthetic.make_w_device(p.N, p.K, seed=0, tag=f"bench.{p.name}")
+        for j, p in enumerate(wl.products):
+            key = (p.scheme, p.M, p.K, p.wo, p.group) if p.group else j
+            g = by_key.get(key)
+            if g is None:
+                xs = [synthetic.make_x_device(p.M, p.K, seed=t, tag=f"bench.{p.group or p.name}.x.M{p.M}",
+                                              outliers=p.outliers) for t in range(self.copies)]
+                g = by_key[key] = {"p0": p, "xs": xs, "items": []}
+                self.groups.append(g)
+            wkey = (p.name, p.N, p.K)
+            if wkey not in weights:
+                weights[wkey] = synthetic.make_w_device(p.N, p.K, seed=0, tag=f"bench.{p.name}")
             n_w = 1 if per_step >= 2 * L2_BYTES else self.copies
-            wqs = [ql.quantize_weight(p.scheme, weights[key]) for _ in range(n_w)]
-            xs = [synthetic.make_x_device(p.M, p.K, seed=t, tag=f"bench.{p.name}.x.M{p.M}",
-                                          outliers=p.outliers) for t in range(self.copies)]
+            wqs = [ql.quantize_weight(p.scheme, weights[wkey]) for _ in range(n_w)]
             ys = [torch.empty((p.M, p.N), dtype=torch.bfloat16, device="cuda") for _ in range(self.copies)]
             ws_bytes = ql.forward_workspace_bytes(p.scheme, p.M, p.N, p.K)
             ws = ql.new_workspace(ws_bytes) if ws_bytes else None
-            item = dict(p=p, wqs=wqs, xs=xs, ys=ys, ws=ws, amount=wl.amount(p))
+            item = dict(p=p, wqs=wqs, ys=ys, ws=ws, xs=g["xs"], amount=wl.amount(p))
             if p.M > 32:  # pre-quantized activations for the dominant-kernel timing
-                item["q"] = [ql.quantize_act(p.scheme, x) for x in xs]
+                item["q"] = [ql.quantize_act(p.scheme, x) for x in g["xs"]]
                 gws = ql.workspace_bytes(p.scheme, p.M, p.N, p.K)  # the K split's sums (block scheme)
                 item["ws_gemm"] = ql.new_workspace(gws) if gws else None
-            self.items.append(item)
+            g["items"].append(item)
         del weights
         torch.cuda.synchronize()
-        self.step_amount = sum(i["amount"] for i in self.items)
-        self.launches_per_step = sum(1 if i["p"].M == 1 else 2 for i in self.items)
+        self.items = [i for g in self.groups for i in g["items"]]
+        self.step_amount = step_amount(wl)  # a group reads its one input once
+        self.launches_per_step = sum(self._launches(g) for g in self.groups)
+        self.dominant_launches = sum(self._grouped(g) or len(g["items"]) for g in self.groups)
+
+    @staticmethod
+    def _grouped(g) -> int:
+        """1 when the group runs as one grouped GEMV launch, else 0."""
+        p = g["p0"]
+        return int(len(g["items"]) > 1 and p.M == 1 and not p.wo)
+
+    def _launches(self, g) -> int:
+        if self._grouped(g):
+            return 1
+        return sum(1 if (i["p"].wo or gemv_route(i["p"].M, i["p"].K)) else 2 for i in g["items"])
 
     def _w(self, i, t):
         return i["wqs"][t % len(i["wqs"])]
@@ -332,26 +375,39 @@ class Runner:
         else:
             self.ql.forward(p.scheme, x, wq, sw, workspace=i["ws"], y=y)
 
+    def _run_group(self, g, x, t, ys=None):
+        """The group's products on input x through the public API (grouped when M = 1)."""
+        items = g["items"]
+        ys = ys or [i["ys"][t] for i in items]
+        if self._grouped(g):
+            self.ql.gemv_grouped(g["p0"].scheme, [(x, *self._w(i, t), y) for i, y in zip(items, ys)])
+        else:
+            for i, y in zip(items, ys):
+                self._forward(i, x, *self._w(i, t), y)
+
     def step(self, t):
-        for i in self.items:
-            wq, sw = self._w(i, t)
-            self._forward(i, i["xs"][t], wq, sw, i["ys"][t])
+        for g in self.groups:
+            self._run_group(g, g["xs"][t], t)
 
     def dominant(self, t):
         """Launches of the dominant kernel alone (the product on quantized inputs)."""
         ql = self.ql
-        for i in self.items:
-            p = i["p"]
-            wq, sw = self._w(i, t)
-            if p.wo:
-                ql.gemv_weight_only(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
-            elif p.M == 1:
-                ql.gemv(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
-            elif p.M <= 32:
-                ql.gemm_small(p.scheme, i["xs"][t], wq, sw, i["ws"], y=i["ys"][t])
-            else:
-                qx, sx = i["q"][t]
-                ql.gemm(p.scheme, qx, sx, wq, sw, workspace=i["ws_gemm"], y=i["ys"][t])
+        for g in self.groups:
+            if self._grouped(g):
+                self._run_group(g, g["xs"][t], t)
+                continue
+            for i in g["items"]:
+                p = i["p"]
+                wq, sw = self._w(i, t)
+                if p.wo:
+                    ql.gemv_weight_only(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
+                elif p.M == 1:
+                    ql.gemv(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
+                elif p.M <= 32:
+                    ql.gemm_small(p.scheme, i["xs"][t], wq, sw, i["ws"], y=i["ys"][t])
+                else:
+                    qx, sx = i["q"][t]
+                    ql.gemm(p.scheme, qx, sx, wq, sw, workspace=i["ws_gemm"], y=i["ys"][t])
 
     def capture(self, fn, stream):
         torch = self.torch
@@ -367,27 +423,30 @@ class Runner:
         return graphs
 
     def e2e_graph(self, stream):
-        """H2D of every product's activations (pinned host -> device), the
-        public forward() calls, D2H of every output."""
-        torch, ql = self.torch, self.ql
-        xs_tot = sum(i["p"].M * i["p"].K for i in self.items)
+        """H2D of every group's activations (pinned host -> device), the
+        public API calls, D2H of every output."""
+        torch = self.torch
+        xs_tot = sum(g["p0"].M * g["p0"].K for g in self.groups)
         ys_tot = sum(i["p"].M * i["p"].N for i in self.items)
         h_x = torch.empty(xs_tot, dtype=torch.bfloat16, pin_memory=True)
         h_y = torch.empty(ys_tot, dtype=torch.bfloat16, pin_memory=True)
         d_x = torch.empty(xs_tot, dtype=torch.bfloat16, device="cuda")
         d_y = torch.empty(ys_tot, dtype=torch.bfloat16, device="cuda")
         views, ox, oy = [], 0, 0
-        for i in self.items:
-            p = i["p"]
-            h_x[ox:ox + p.M * p.K].copy_(i["xs"][0].reshape(-1).cpu())
-            views.append((i, d_x[ox:ox + p.M * p.K].view(p.M, p.K), d_y[oy:oy + p.M * p.N].view(p.M, p.N)))
+        for g in self.groups:
+            p = g["p0"]
+            h_x[ox:ox + p.M * p.K].copy_(g["xs"][0].reshape(-1).cpu())
+            yv = []
+            for i in g["items"]:
+                q = i["p"]
+                yv.append(d_y[oy:oy + q.M * q.N].view(q.M, q.N))
+                oy += q.M * q.N
+            views.append((g, d_x[ox:ox + p.M * p.K].view(p.M, p.K), yv))
             ox += p.M * p.K
-            oy += p.M * p.N
 
         def body(c):
-            for i, xv, yv in views:
-                wq, sw = self._w(i, c)
-                self._forward(i, xv, wq, sw, yv)
+            for g, xv, yv in views:
+                self._run_group(g, xv, c, ys=yv)
 
         with torch.cuda.stream(stream):
             body(0)
@@ -418,10 +477,29 @@ def whole_job_value(world: int, amount_per_step: float, steps: int, ms: float, s
     return world * amount_per_step * steps / (ms / 1e3) / scale
 
 
+def input_groups(wl):
+    """Products grouped by the input they read, in launch order."""
+    groups = {}
+    for j, p in enumerate(wl.products):
+        key = (p.scheme, p.M, p.K, p.wo, p.group) if p.group else j
+        groups.setdefault(key, []).append(p)
+    return list(groups.values())
+
+
+def step_amount(wl) -> float:
+    """Algorithmic amount of one step: a group's shared input counts once."""
+    total = sum(wl.amount(p) for p in wl.products)
+    if wl.unit == "GB/s":
+        total -= sum((len(g) - 1) * 2 * g[0].M * g[0].K for g in input_groups(wl))
+    return total
+
+
 def workload_config(wl):
     return {"workload": wl.description, "key": wl.key,
             "products": [f"{SCHEME_NAME[p.scheme]} M={p.M} {p.name} {p.N}x{p.K}" for p in wl.products],
-            "amount_per_step": sum(wl.amount(p) for p in wl.products)}
+            "input_groups": ["|".join(p.name for p in g) + f" ({SCHEME_NAME[g[0].scheme]})"
+                             for g in input_groups(wl) if len(g) > 1],
+            "amount_per_step": step_amount(wl)}
 
 
 def timed(torch, stream, graphs, steps):
@@ -491,9 +569,38 @@ def _oracle_items(wl: Workload, rows_cap: int):
     return items
 
 
-def _oracle_run(scheme, x, wq, sw, wo):
+_POOL = {}
+
+
+def host_threads() -> int:
+    """The host's cores (nproc: the CPU set this process may run on)."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except (AttributeError, OSError):
+        return max(1, os.cpu_count() or 1)
+
+
+def _oracle_run(scheme, x, wq, sw, wo, threads=1):
+    """One product through the oracle; with threads > 1 its output rows are
+    split over host threads (the oracle's C calls release the GIL; the block
+    scheme keeps whole 128-row blocks).  The arithmetic is the oracle's."""
     import oracle
-    return oracle.linear_weight_only(scheme, x, wq, sw) if wo else oracle.forward(scheme, x, wq, sw)
+    if threads <= 1:
+        return oracle.linear_weight_only(scheme, x, wq, sw) if wo else oracle.forward(scheme, x, wq, sw)
+    import concurrent.futures
+    if threads not in _POOL:
+        _POOL[threads] = concurrent.futures.ThreadPoolExecutor(max_workers=threads)
+    N = wq.shape[0]
+    step = -(-N // threads)
+    if scheme == FP8B:
+        step = -(-step // 128) * 128
+    bounds = [(n0, min(N, n0 + step)) for n0 in range(0, N, step)]
+    if wo:
+        fn = lambda b: oracle.linear_weight_only(scheme, x, wq, sw, b[0], b[1])  # noqa: E731
+    else:
+        qx, sx = oracle.quantize_act(scheme, x)
+        fn = lambda b: oracle.linear_rows(scheme, qx, sx, wq, sw, b[0], b[1])  # noqa: E731
+    return list(_POOL[threads].map(fn, bounds))
 
 
 def sample_rows_text(wl: Workload, rows_cap: int) -> str:
@@ -513,18 +620,18 @@ def sample_rows_text(wl: Workload, rows_cap: int) -> str:
             f"({sum(counts)} rows in all)")
 
 
-def oracle_sample(wl: Workload, budget_s: float, rows_cap: int):
+def oracle_sample(wl: Workload, budget_s: float, rows_cap: int, threads: int = 1):
     """The CPU oracle (whole method from bf16 X) on the first rows_cap output
-    rows of every product of the workload, repeated for about budget_s.
+    rows of every product of the workload, repeated for about budget_s, on
+    `threads` host threads.
     Returns (throughput in the workload's unit, seconds, passes, amount per pass)."""
-    import oracle
     items = _oracle_items(wl, rows_cap)
     per_pass = sum(i[4] for i in items)
     done, t_used, passes = 0.0, 0.0, 0
     while t_used < budget_s or passes == 0:
         t0 = time.perf_counter()
         for scheme, x, wq, sw, amt, wo in items:
-            _oracle_run(scheme, x, wq, sw, wo)
+            _oracle_run(scheme, x, wq, sw, wo, threads)
             done += amt
         t_used += time.perf_counter() - t0
         passes += 1
@@ -532,10 +639,28 @@ def oracle_sample(wl: Workload, budget_s: float, rows_cap: int):
     return done / t_used / scale, t_used, passes, per_pass
 
 
-def pick_rows(wl: Workload, seconds: float) -> int:
-    """Rows per product so that one oracle pass takes about `seconds`."""
-    _, t, _, _ = oracle_sample(wl, 0.0, 8)
-    return max(1, int(8 * seconds / max(t, 1e-6)))
+def pick_rows(wl: Workload, seconds: float, threads: int = 1) -> int:
+    """Rows per product so that one oracle pass on `threads` threads takes about `seconds`."""
+    probe = 8 * threads
+    _, t, _, _ = oracle_sample(wl, 0.0, probe, threads)
+    return max(1, int(probe * seconds / max(t, 1e-6)))
+
+
+def cpu_baseline(wl, seconds: float, step_amount: float) -> dict:
+    """The oracle on all host cores (threads over output rows) and on one
+    thread, each on a bounded row sample of the workload for about `seconds`."""
+    out = {}
+    for threads in (host_threads(), 1):
+        rows = pick_rows(wl, min(seconds, 4.0), threads)
+        v, secs, passes, per_pass = oracle_sample(wl, seconds, rows, threads)
+        out[threads] = {"value": round(v, 6), "unit": wl.unit, "cores": threads, "kind": "oracle",
+                        "sample": f"{sample_rows_text(wl, rows)} "
+                                  f"({100 * per_pass / step_amount:.3g}% of a step) x {passes} passes, "
+                                  f"{secs:.1f} s, {threads} host thread{'s' if threads > 1 else ''}"}
+    top = out[host_threads()]
+    if host_threads() > 1:
+        top["single_thread"] = {k: out[1][k] for k in ("value", "sample")}
+    return top
 
 
 def base_line(wl, args, world):
@@ -551,35 +676,152 @@ def run_reference(args):
         return 0
     import oracle
     wl = workloads()[args.workload]
+    threads = host_threads()
     per_step = max(0.002, 60.0 / max(1, args.steps + args.warmup))
-    rows = pick_rows(wl, per_step)
+    rows = pick_rows(wl, per_step, threads)
     items = _oracle_items(wl, rows)
     step_amount = sum(i[4] for i in items)
     for _ in range(args.warmup):
         for scheme, x, wq, sw, _, wo in items:
-            _oracle_run(scheme, x, wq, sw, wo)
+            _oracle_run(scheme, x, wq, sw, wo, threads)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         for scheme, x, wq, sw, _, wo in items:
-            _oracle_run(scheme, x, wq, sw, wo)
+            _oracle_run(scheme, x, wq, sw, wo, threads)
     dt = time.perf_counter() - t0
     scale = 1e9 if wl.unit == "GB/s" else 1e12
     value = step_amount * args.steps / dt / scale
     full = sum(wl.amount(p) for p in wl.products)
     sample = (f"{sample_rows_text(wl, rows)}, "
-              f"{100 * step_amount / full:.3g}% of a full step, per step; single thread")
+              f"{100 * step_amount / full:.3g}% of a full step, per step; {threads} host threads "
+              f"over output rows")
     line = base_line(wl, args, args.gpus)
     line.update({"value": value, "impl": "reference", "ms_per_step": dt / args.steps * 1e3,
                  "dtype": ("f64 sums of exact bf16 x dequantized-weight products" if wl.products[0].wo
                            else "s8*s8->s32 (int8), e4m3*e4m3 exact (int64 fixed point)"),
                  "config": {**workload_config(wl), "parallelism": f"replicas x{args.gpus}",
                             "note": "CPU oracle, the plain definition, on a row sample per step"},
-                 "cpu_baseline": {"value": value, "unit": wl.unit, "cores": 1, "kind": "oracle",
+                 "cpu_baseline": {"value": value, "unit": wl.unit, "cores": threads, "kind": "oracle",
                                   "sample": sample},
                  "e2e": {"value": value, "unit": wl.unit, "h2d_bytes_per_step": 0,
                          "d2h_bytes_per_step": 0}})
     print(json.dumps(line), flush=True)
     return 0
+
+
+# Configurations timed after the headline in the default run, each reported
+# under "extra" in the same line: the W8A8 k_proj case (M = 8), W8A8 prefill
+# (M = 512, 1024) and the Qwen3-8B block scheme at M = 512.
+EXTRA_WORKLOADS = ("kproj", "prefill", "qwen-prefill")
+
+
+def measure(torch, ql, synthetic, wl, args, steps, warmup, world, rank, barrier, max_over_ranks,
+            cpu_seconds):
+    """Every leg of one workload's line: the timed graph replays, the dominant
+    kernel's own launches (roofline), end to end from host buffers, the parity
+    report and the oracle baseline.  Returns the line's fields."""
+    scale = 1e9 if wl.unit == "GB/s" else 1e12
+    stream = torch.cuda.Stream()
+    run = Runner(torch, ql, synthetic, wl)
+    graphs = run.capture(run.step, stream)
+
+    # ---- timed region: K steps, one graph replay each
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            graphs[i % len(graphs)].replay()
+    stream.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ms_local = timed(torch, stream, graphs, steps)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(ms_local)
+    value = whole_job_value(world, run.step_amount, steps, ms, scale)
+    status, detail = ql.device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} detail {detail:#x} after the timed region")
+    del graphs
+
+    # ---- the dominant kernel's own launches (for the roofline), same kind of timing
+    dgraphs = run.capture(run.dominant, stream)
+    dsteps = max(3, min(steps, 500))
+    with torch.cuda.stream(stream):
+        for i in range(min(warmup, 10)):
+            dgraphs[i % len(dgraphs)].replay()
+    d_ms = timed(torch, stream, dgraphs, dsteps)
+    n_dom = run.dominant_launches
+    per_launch_amount = run.step_amount / n_dom
+    per_launch_s = (d_ms / 1e3) / (dsteps * n_dom)
+    achieved = per_launch_amount / per_launch_s / scale
+    peak, peak_src = roofline_peak(wl)
+    traffic, traffic_src = measured_traffic(wl)
+    roofline = {"bound": wl.bound, "achieved": round(achieved, 1), "peak": round(peak, 1),
+                "unit": wl.unit, "frac": round(achieved / peak, 4), "traffic": traffic,
+                "traffic_source": traffic_src,
+                "kernel": wl.kernel, "peak_source": peak_src,
+                "duration_source": "CUDA events over graph replays of this kernel's launches "
+                                   "(inputs already quantized where the step quantizes separately)"}
+    del dgraphs
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = args.e2e_steps or max(10, min(steps, 1000))
+    g_e2e, h2d, d2h = run.e2e_graph(stream)
+    with torch.cuda.stream(stream):
+        for i in range(min(warmup, 10)):
+            g_e2e[i % len(g_e2e)].replay()
+            stream.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e2e_steps):
+            g_e2e[i % len(g_e2e)].replay()
+            stream.synchronize()  # the host reads every step's outputs
+        e1.record(stream)
+    e1.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = whole_job_value(world, run.step_amount, e2e_steps, e2e_ms, scale)
+    del g_e2e
+
+    # ---- the outputs against the oracle on a row sample (rank 0; never fatal)
+    parity = None
+    if rank == 0:
+        try:
+            with torch.cuda.stream(stream):
+                run.step(0)
+            stream.synchronize()
+            parity = parity_sample(run, torch)
+        except Exception as exc:  # the report must not cost the bench line
+            parity = {"error": f"{type(exc).__name__}: {exc}"}
+
+    cpu = None
+    if rank == 0 and world == 1 and cpu_seconds > 0:
+        cpu = cpu_baseline(wl, cpu_seconds, run.step_amount)
+    weight_bytes = sum(p.N * p.K for p in wl.products)
+    out = {
+        "metric": METRIC, "unit": wl.unit, "value": round(value, 1), "ms_per_step": ms / steps,
+        "steps": steps, "warmup": warmup,
+        "config": {**workload_config(wl),
+                   "launches_per_step": run.launches_per_step,
+                   "parallelism": f"replicas x{world}",
+                   "l2": (f"inputs larger than L2 (126 MB): consecutive steps cycle through "
+                          f"{run.copies} sets of weights/activations/outputs, "
+                          f"{run.copies * sum(wl.bytes_touched(p) for p in wl.products) / 1e6:.0f} MB "
+                          f"touched per cycle ({weight_bytes / 1e6:.0f} MB of weights per step); no flush"),
+                   "timing": "one CUDA graph replay per step, CUDA events on the launch stream"},
+        "roofline": roofline,
+        "parity": parity,
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_value, 1), "unit": wl.unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "how": "graph of H2D activations + the public API per product (grouped where a "
+                       "layer's products read one input) + D2H outputs, host sync per step"},
+        "gpu_launches": run.launches_per_step * steps,
+    }
+    del run
+    torch.cuda.empty_cache()
+    return out
 
 
 def main():
@@ -611,115 +853,29 @@ def main():
     def max_over_ranks(v: float) -> float:
         return max_over_ranks_of(torch, dist if world > 1 else None, v, "cuda")
 
-    wl = workloads()[args.workload]
-    scale = 1e9 if wl.unit == "GB/s" else 1e12
-    stream = torch.cuda.Stream()
-    run = Runner(torch, ql, synthetic, wl)
-    graphs = run.capture(run.step, stream)
-
-    # ---- timed region: K steps, one graph replay each
+    cpu_s = 0.0 if args.no_cpu_baseline else args.cpu_seconds
+    # one clock record spans every leg of every workload of the line
     sampler = ClockSampler(nvsmi_index(torch, dev) if rank == 0 else None).start()
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            graphs[i % len(graphs)].replay()
-    stream.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    ms_local = timed(torch, stream, graphs, args.steps)
-    torch.cuda.synchronize()
-    barrier()
+    wl = workloads()[args.workload]
+    head = measure(torch, ql, synthetic, wl, args, args.steps, args.warmup, world, rank, barrier,
+                   max_over_ranks, cpu_s)
+    extra = {}
+    if args.workload == "decode" and not args.no_extra:
+        # the tensor-bound configurations, each timed the same way; fewer steps
+        # (each of their steps is 10-400 us) so the whole run stays within minutes
+        for key in EXTRA_WORKLOADS:
+            xs = max(3, min(args.steps, 200))
+            extra[key] = measure(torch, ql, synthetic, workloads()[key], args, xs, max(3, min(args.warmup, 20)),
+                                 world, rank, barrier, max_over_ranks, min(cpu_s, 6.0))
     clocks = sampler.stop()
-    ms = max_over_ranks(ms_local)
-    value = whole_job_value(world, run.step_amount, args.steps, ms, scale)
-    status, detail = ql.device_status(stream)
-    if status != 0:
-        raise RuntimeError(f"device status {status} detail {detail:#x} after the timed region")
-
-    # ---- the dominant kernel's own launches (for the roofline), same kind of timing
-    dgraphs = run.capture(run.dominant, stream)
-    dsteps = max(3, min(args.steps, 500))
-    with torch.cuda.stream(stream):
-        for i in range(min(args.warmup, 10)):
-            dgraphs[i % len(dgraphs)].replay()
-    d_ms = timed(torch, stream, dgraphs, dsteps)
-    n_dom = len(run.items)
-    per_launch_amount = run.step_amount / n_dom
-    per_launch_s = (d_ms / 1e3) / (dsteps * n_dom)
-    achieved = per_launch_amount / per_launch_s / scale
-    peak, peak_src = roofline_peak(wl)
-    traffic, traffic_src = measured_traffic(wl)
-    roofline = {"bound": wl.bound, "achieved": round(achieved, 1), "peak": round(peak, 1),
-                "unit": wl.unit, "frac": round(achieved / peak, 4), "traffic": traffic,
-                "traffic_source": traffic_src,
-                "kernel": wl.kernel, "peak_source": peak_src,
-                "duration_source": "CUDA events over graph replays of this kernel's launches "
-                                   "(inputs already quantized where the step quantizes separately)"}
-    del dgraphs
-
-    # ---- end to end through the public API with host buffers
-    e2e_steps = args.e2e_steps or max(10, min(args.steps, 1000))
-    g_e2e, h2d, d2h = run.e2e_graph(stream)
-    with torch.cuda.stream(stream):
-        for i in range(min(args.warmup, 10)):
-            g_e2e[i % len(g_e2e)].replay()
-            stream.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for i in range(e2e_steps):
-            g_e2e[i % len(g_e2e)].replay()
-            stream.synchronize()  # the host reads every step's outputs
-        e1.record(stream)
-    e1.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = whole_job_value(world, run.step_amount, e2e_steps, e2e_ms, scale)
-    del g_e2e
-
-    # ---- the outputs against the oracle on a row sample (rank 0; never fatal)
-    parity = None
-    if rank == 0:
-        try:
-            with torch.cuda.stream(stream):
-                run.step(0)
-            stream.synchronize()
-            parity = parity_sample(run, torch)
-        except Exception as exc:  # the report must not cost the bench line
-            parity = {"error": f"{type(exc).__name__}: {exc}"}
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows = pick_rows(wl, min(args.cpu_seconds, 4.0))
-        v, secs, passes, per_pass = oracle_sample(wl, args.cpu_seconds, rows)
-        cpu = {"value": round(v, 6), "unit": wl.unit, "cores": 1, "kind": "oracle",
-               "sample": f"{sample_rows_text(wl, rows)} "
-                         f"({100 * per_pass / run.step_amount:.3g}% of a step) x {passes} passes, "
-                         f"{secs:.1f} s, single thread"}
 
     if rank == 0:
         line = base_line(wl, args, world)
-        weight_bytes = sum(p.N * p.K for p in wl.products)
-        line.update({
-            "value": round(value, 1), "ms_per_step": ms / args.steps,
-            "config": {**workload_config(wl),
-                       "launches_per_step": run.launches_per_step,
-                       "parallelism": f"replicas x{world}",
-                       "l2": (f"inputs larger than L2 (126 MB): consecutive steps cycle through "
-                              f"{run.copies} sets of weights/activations/outputs, "
-                              f"{run.copies * sum(wl.bytes_touched(p) for p in wl.products) / 1e6:.0f} MB "
-                              f"touched per cycle ({weight_bytes / 1e6:.0f} MB of weights per step); no flush"),
-                       "timing": "one CUDA graph replay per step, CUDA events on the launch stream"},
-            "roofline": roofline,
-            "parity": parity,
-            "cpu_baseline": cpu,
-            "e2e": {"value": round(e2e_value, 1), "unit": wl.unit, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                    "how": "graph of H2D activations + forward() per product + D2H outputs, "
-                           "host sync per step"},
-            "gpu_launches": run.launches_per_step * args.steps,
-            "clocks": clocks,
-        })
+        line.update(head)
+        line["clocks"] = clocks
+        if extra:
+            line["extra"] = extra
+            line["gpu_launches"] = head["gpu_launches"] + sum(e["gpu_launches"] for e in extra.values())
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

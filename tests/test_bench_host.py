@@ -29,9 +29,20 @@ def test_decode_layer_bytes():
     # the weight-only layer moves the same bytes through the same 14 products
     wo = w["decode-wo"]
     assert all(p.wo for p in wo.products) and not any(p.wo for p in dec.products)
-    assert [(p.name, p.scheme, p.N, p.K) for p in wo.products] == \
-        [(p.name, p.scheme, p.N, p.K) for p in dec.products]
+    assert sorted((p.name, p.scheme, p.N, p.K) for p in wo.products) == \
+        sorted((p.name, p.scheme, p.N, p.K) for p in dec.products)
     assert sum(wo.amount(p) for p in wo.products) == 436_879_360
+    # the same 14 products, each its own launch
+    sep = w["decode-separate"]
+    assert sorted((p.name, p.scheme) for p in sep.products) == sorted((p.name, p.scheme) for p in dec.products)
+    assert bench.step_amount(sep) == 436_879_360
+    # grouped decode: per scheme q|k|v and gate|up read one input each, counted once:
+    # 2 schemes x (2 + 1) duplicate 4096-wide bf16 inputs fewer
+    groups = bench.input_groups(dec)
+    assert [[p.name for p in g] for g in groups][:4] == [["q_proj", "k_proj", "v_proj"], ["o_proj"],
+                                                         ["gate_proj", "up_proj"], ["down_proj"]]
+    assert len(groups) == 8
+    assert bench.step_amount(dec) == 436_879_360 - 2 * 3 * 2 * 4096
     # side by side along N: the same weight bytes in 8 products
     assert _weights(w["decode-fused"]) == 2 * LLAMA_WEIGHT_BYTES
     assert len(w["decode-fused"].products) == 8
