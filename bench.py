@@ -70,6 +70,8 @@ class Product:
     outliers: int
     wo: bool = False  # weight-only product (activations not rounded)
     group: str = ""   # products of one (scheme, group) read one input; M = 1 ones share a launch
+    pre: bool = False  # the input arrives quantized (codes + scales from its producer); with M > 32
+                       # the product also quantizes its own output for the next product
 
 
 @dataclass
@@ -85,22 +87,31 @@ class Workload:
 
     @property
     def kernel(self):
-        if self.products[0].wo:
+        p = self.products[0]
+        if p.wo:
             return "ql::gemv_kernel (weight-only)"
-        M = self.products[0].M
-        return "ql::gemv_kernel" if M == 1 else ("ql::gemm_small_kernel" if M <= 32 else "ql::gemm_kernel")
+        if p.M > 32 and p.pre:
+            return "ql::gemm_kernel (output quantization fused)"
+        return "ql::gemv_kernel" if p.M == 1 else ("ql::gemm_small_kernel" if p.M <= 32 else "ql::gemm_kernel")
+
+    @staticmethod
+    def input_bytes(p: Product) -> float:
+        """Bytes of one product's input: bf16 x, or codes + f32 scales when it arrives quantized."""
+        if not p.pre:
+            return 2 * p.M * p.K
+        return p.M * p.K + 4 * p.M * (p.K // 128 if p.scheme == FP8B else 1)
 
     def bytes_touched(self, p: Product) -> float:
         """Bytes one product reads and writes in HBM (weights, scales, x, y)."""
         sw = 4 * (p.N // 128) * (p.K // 128) if p.scheme == FP8B else 4 * p.N
-        return p.N * p.K + sw + 2 * p.M * p.K + 2 * p.M * p.N + p.M * p.K
+        return p.N * p.K + sw + self.input_bytes(p) + 2 * p.M * p.N + p.M * p.K
 
     def amount(self, p: Product) -> float:
         """Algorithmic bytes (HBM-bound regimes) or ops (tensor-bound) of one product."""
         if self.unit == "TOPS":
             return 2.0 * p.M * p.N * p.K
         sw = 4 * (p.N // 128) * (p.K // 128) if p.scheme == FP8B else 4 * p.N
-        return p.N * p.K + sw + 2 * p.M * p.K + 2 * p.M * p.N
+        return p.N * p.K + sw + self.input_bytes(p) + 2 * p.M * p.N
 
 
 # The projections of a decoder layer that read one input: q, k, v (the
@@ -158,6 +169,22 @@ def workloads():
     w["qwen-small"] = Workload(
         "qwen-small", "Qwen3-8B FP8 128x128-block projections at M=32 (7 shapes)", "GB/s",
         [Product(n, FP8B, 32, N, K, 0) for n, N, K in S.QWEN3_8B])
+    w["decode-f2"] = Workload(
+        "decode-f2", "decode GEMV M=1 as the decode workload, each input arriving already quantized "
+        "(codes + scales written by its producer): q|k|v and gate|up grouped, 4 launches per scheme",
+        "GB/s", [Product(n, s, 1, N, K, oc(K), group=LAYER_INPUT.get(n, n), pre=True)
+                 for s in (INT8, FP8R) for n, N, K in S.LLAMA31_8B])
+    w["small-f2"] = Workload(
+        "small-f2", "small-batch tensor-core path as the small workload (M in {2, 8, 16, 32} x the 7 "
+        "Llama-3.1-8B shapes x {W8A8, FP8 row}), each input arriving already quantized: one kernel "
+        "per product", "GB/s",
+        [Product(n, s, M, N, K, oc(K), pre=True) for M in (2, 8, 16, 32) for s in (INT8, FP8R)
+         for n, N, K in S.LLAMA31_8B])
+    w["qwen-prefill-f2"] = Workload(
+        "qwen-prefill-f2", "Qwen3-8B FP8 128x128-block projections at M=512 (7 shapes), each input "
+        "arriving already quantized and each product also writing its own output's E4M3 codes and "
+        "per-128 scales for the product that reads it next: one kernel per projection", "TOPS",
+        [Product(n, FP8B, 512, N, K, 0, pre=True) for n, N, K in S.QWEN3_8B])
     w["qwen-prefill"] = Workload(
         "qwen-prefill", "Qwen3-8B FP8 128x128-block projections at M=512 (7 shapes), per-K-block "
         "promotion", "TOPS", [Product(n, FP8B, 512, N, K, 0) for n, N, K in S.QWEN3_8B])
@@ -172,7 +199,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["qlinear", "reference"], default="qlinear")
     ap.add_argument("--workload", default="decode",
                     choices=["decode", "decode-separate", "decode-fused", "prefill", "small", "kproj",
-                             "qwen-decode", "qwen-small", "qwen-prefill", "decode-wo"])
+                             "qwen-decode", "qwen-small", "qwen-prefill", "decode-wo", "decode-f2",
+                             "small-f2", "qwen-prefill-f2"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -332,6 +360,8 @@ class Runner:
                 xs = [synthetic.make_x_device(p.M, p.K, seed=t, tag=f"bench.{p.group or p.name}.x.M{p.M}",
                                               outliers=p.outliers) for t in range(self.copies)]
                 g = by_key[key] = {"p0": p, "xs": xs, "items": []}
+                # the step's input: bf16 x, or its codes + scales as a producer would write them
+                g["x_in"] = [ql.quantize_act(p.scheme, x) for x in xs] if p.pre else xs
                 self.groups.append(g)
             wkey = (p.name, p.N, p.K)
             if wkey not in weights:
@@ -342,8 +372,12 @@ class Runner:
             ws_bytes = ql.forward_workspace_bytes(p.scheme, p.M, p.N, p.K)
             ws = ql.new_workspace(ws_bytes) if ws_bytes else None
             item = dict(p=p, wqs=wqs, ys=ys, ws=ws, xs=g["xs"], amount=wl.amount(p))
+            if p.pre and p.M > 32:  # the output's own codes and scales
+                item["qy"] = [(torch.empty((p.M, p.N), dtype=torch.uint8, device="cuda"),
+                               torch.empty((p.M, p.N // 128), dtype=torch.float32, device="cuda"))
+                              for _ in range(self.copies)]
             if p.M > 32:  # pre-quantized activations for the dominant-kernel timing
-                item["q"] = [ql.quantize_act(p.scheme, x) for x in g["xs"]]
+                item["q"] = g["x_in"] if p.pre else [ql.quantize_act(p.scheme, x) for x in g["xs"]]
                 gws = ql.workspace_bytes(p.scheme, p.M, p.N, p.K)  # the K split's sums (block scheme)
                 item["ws_gemm"] = ql.new_workspace(gws) if gws else None
             g["items"].append(item)
@@ -356,14 +390,16 @@ class Runner:
 
     @staticmethod
     def _grouped(g) -> int:
-        """1 when the group runs as one grouped GEMV launch, else 0."""
+        """1 when the group runs as one qlinear_gemv_grouped launch (every M = 1
+        quantized product: a group of one included), else 0."""
         p = g["p0"]
-        return int(len(g["items"]) > 1 and p.M == 1 and not p.wo)
+        return int(p.M == 1 and not p.wo)
 
     def _launches(self, g) -> int:
         if self._grouped(g):
             return 1
-        return sum(1 if (i["p"].wo or gemv_route(i["p"].M, i["p"].K)) else 2 for i in g["items"])
+        return sum(1 if (i["p"].wo or i["p"].pre or gemv_route(i["p"].M, i["p"].K)) else 2
+                   for i in g["items"])
 
     def _w(self, i, t):
         return i["wqs"][t % len(i["wqs"])]
@@ -376,25 +412,36 @@ class Runner:
             self.ql.forward(p.scheme, x, wq, sw, workspace=i["ws"], y=y)
 
     def _run_group(self, g, x, t, ys=None):
-        """The group's products on input x through the public API (grouped when M = 1)."""
+        """The group's products on input x (bf16, or a (codes, scales) pair when
+        it arrives quantized) through the public API (grouped when M = 1)."""
         items = g["items"]
         ys = ys or [i["ys"][t] for i in items]
         if self._grouped(g):
             self.ql.gemv_grouped(g["p0"].scheme, [(x, *self._w(i, t), y) for i, y in zip(items, ys)])
+        elif g["p0"].pre:
+            qx, sx = x
+            for i, y in zip(items, ys):
+                p = i["p"]
+                wq, sw = self._w(i, t)
+                if p.M <= 32:
+                    self.ql.gemm_small_prequant(p.scheme, qx, sx, wq, sw, i["ws"], y=y)
+                else:
+                    qy, sy = i["qy"][t]
+                    self.ql.gemm_quant_out(p.scheme, qx, sx, wq, sw, workspace=i["ws_gemm"], y=y, qy=qy, sy=sy)
         else:
             for i, y in zip(items, ys):
                 self._forward(i, x, *self._w(i, t), y)
 
     def step(self, t):
         for g in self.groups:
-            self._run_group(g, g["xs"][t], t)
+            self._run_group(g, g["x_in"][t], t)
 
     def dominant(self, t):
         """Launches of the dominant kernel alone (the product on quantized inputs)."""
         ql = self.ql
         for g in self.groups:
-            if self._grouped(g):
-                self._run_group(g, g["xs"][t], t)
+            if self._grouped(g) or g["p0"].pre:  # one kernel per launch already
+                self._run_group(g, g["x_in"][t], t)
                 continue
             for i in g["items"]:
                 p = i["p"]
@@ -423,26 +470,28 @@ class Runner:
         return graphs
 
     def e2e_graph(self, stream):
-        """H2D of every group's activations (pinned host -> device), the
-        public API calls, D2H of every output."""
+        """H2D of every group's input (pinned host -> device: bf16 x, or codes
+        and scales), the public API calls, D2H of every output."""
         torch = self.torch
-        xs_tot = sum(g["p0"].M * g["p0"].K for g in self.groups)
         ys_tot = sum(i["p"].M * i["p"].N for i in self.items)
-        h_x = torch.empty(xs_tot, dtype=torch.bfloat16, pin_memory=True)
         h_y = torch.empty(ys_tot, dtype=torch.bfloat16, pin_memory=True)
-        d_x = torch.empty(xs_tot, dtype=torch.bfloat16, device="cuda")
         d_y = torch.empty(ys_tot, dtype=torch.bfloat16, device="cuda")
-        views, ox, oy = [], 0, 0
+        views, copies, h2d, oy = [], [], 0, 0
         for g in self.groups:
-            p = g["p0"]
-            h_x[ox:ox + p.M * p.K].copy_(g["xs"][0].reshape(-1).cpu())
+            src = g["x_in"][0]
+            parts = list(src) if isinstance(src, tuple) else [src]
+            dev = [torch.empty_like(a) for a in parts]
+            for a, d in zip(parts, dev):
+                h = torch.empty(a.shape, dtype=a.dtype, pin_memory=True)
+                h.copy_(a.cpu())
+                copies.append((d, h))
+                h2d += a.numel() * a.element_size()
             yv = []
             for i in g["items"]:
                 q = i["p"]
                 yv.append(d_y[oy:oy + q.M * q.N].view(q.M, q.N))
                 oy += q.M * q.N
-            views.append((g, d_x[ox:ox + p.M * p.K].view(p.M, p.K), yv))
-            ox += p.M * p.K
+            views.append((g, tuple(dev) if isinstance(src, tuple) else dev[0], yv))
 
         def body(c):
             for g, xv, yv in views:
@@ -455,11 +504,12 @@ class Runner:
         for c in range(self.copies):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                d_x.copy_(h_x, non_blocking=True)
+                for d, h in copies:
+                    d.copy_(h, non_blocking=True)
                 body(c)
                 h_y.copy_(d_y, non_blocking=True)
             graphs.append(g)
-        return graphs, 2 * xs_tot, 2 * ys_tot
+        return graphs, h2d, 2 * ys_tot
 
 
 def max_over_ranks_of(torch, dist, v: float, device) -> float:
@@ -490,7 +540,7 @@ def step_amount(wl) -> float:
     """Algorithmic amount of one step: a group's shared input counts once."""
     total = sum(wl.amount(p) for p in wl.products)
     if wl.unit == "GB/s":
-        total -= sum((len(g) - 1) * 2 * g[0].M * g[0].K for g in input_groups(wl))
+        total -= sum((len(g) - 1) * Workload.input_bytes(g[0]) for g in input_groups(wl))
     return total
 
 
@@ -564,8 +614,13 @@ def _oracle_items(wl: Workload, rows_cap: int):
         w = synthetic.make_w(rows, p.K, seed=0, tag=f"oracle.{p.name}")
         x = synthetic.make_x(p.M, p.K, seed=0, tag=f"oracle.{p.name}.x", outliers=p.outliers)
         wq, sw = oracle.quantize_weight(p.scheme, w)
-        items.append((p.scheme, x, wq, sw, wl.amount(Product(p.name, p.scheme, p.M, rows, p.K, 0)),
-                      p.wo))
+        # kind: "wo" weight-only; "pre" input already quantized (the codes are
+        # the oracle's, made here, outside the timed work); "preq" also
+        # quantizes the product's output; None the whole method from bf16 x
+        kind = "wo" if p.wo else (("preq" if p.M > 32 else "pre") if p.pre else None)
+        xin = oracle.quantize_act(p.scheme, x) if p.pre else x
+        items.append((p.scheme, xin, wq, sw,
+                      wl.amount(Product(p.name, p.scheme, p.M, rows, p.K, 0, pre=p.pre)), kind))
     return items
 
 
@@ -580,26 +635,43 @@ def host_threads() -> int:
         return max(1, os.cpu_count() or 1)
 
 
-def _oracle_run(scheme, x, wq, sw, wo, threads=1):
-    """One product through the oracle; with threads > 1 its output rows are
-    split over host threads (the oracle's C calls release the GIL; the block
-    scheme keeps whole 128-row blocks).  The arithmetic is the oracle's."""
+def _oracle_run(scheme, x, wq, sw, kind, threads=1):
+    """One product through the oracle (kind as in _oracle_items); with threads
+    > 1 its output rows are split over host threads (the oracle's C calls
+    release the GIL; the block scheme keeps whole 128-row blocks).  The
+    arithmetic is the oracle's."""
     import oracle
+    wo = kind == "wo"
+    if kind in ("pre", "preq"):
+        qx, sx = x
+        if threads <= 1:
+            y = oracle.linear(scheme, qx, sx, wq, sw)
+        else:
+            y = _oracle_rows(lambda b: oracle.linear_rows(scheme, qx, sx, wq, sw, b[0], b[1]),
+                             scheme, wq.shape[0], threads)
+            y = __import__("numpy").concatenate(y, axis=1)
+        if kind == "preq":
+            oracle.quantize_act(scheme, y)
+        return y
     if threads <= 1:
         return oracle.linear_weight_only(scheme, x, wq, sw) if wo else oracle.forward(scheme, x, wq, sw)
-    import concurrent.futures
-    if threads not in _POOL:
-        _POOL[threads] = concurrent.futures.ThreadPoolExecutor(max_workers=threads)
-    N = wq.shape[0]
-    step = -(-N // threads)
-    if scheme == FP8B:
-        step = -(-step // 128) * 128
-    bounds = [(n0, min(N, n0 + step)) for n0 in range(0, N, step)]
     if wo:
         fn = lambda b: oracle.linear_weight_only(scheme, x, wq, sw, b[0], b[1])  # noqa: E731
     else:
         qx, sx = oracle.quantize_act(scheme, x)
         fn = lambda b: oracle.linear_rows(scheme, qx, sx, wq, sw, b[0], b[1])  # noqa: E731
+    return _oracle_rows(fn, scheme, wq.shape[0], threads)
+
+
+def _oracle_rows(fn, scheme, N, threads):
+    """fn over output-row ranges on a pool of host threads."""
+    import concurrent.futures
+    if threads not in _POOL:
+        _POOL[threads] = concurrent.futures.ThreadPoolExecutor(max_workers=threads)
+    step = -(-N // threads)
+    if scheme == FP8B:
+        step = -(-step // 128) * 128
+    bounds = [(n0, min(N, n0 + step)) for n0 in range(0, N, step)]
     return list(_POOL[threads].map(fn, bounds))
 
 
@@ -630,8 +702,8 @@ def oracle_sample(wl: Workload, budget_s: float, rows_cap: int, threads: int = 1
     done, t_used, passes = 0.0, 0.0, 0
     while t_used < budget_s or passes == 0:
         t0 = time.perf_counter()
-        for scheme, x, wq, sw, amt, wo in items:
-            _oracle_run(scheme, x, wq, sw, wo, threads)
+        for scheme, x, wq, sw, amt, kind in items:
+            _oracle_run(scheme, x, wq, sw, kind, threads)
             done += amt
         t_used += time.perf_counter() - t0
         passes += 1
@@ -682,12 +754,12 @@ def run_reference(args):
     items = _oracle_items(wl, rows)
     step_amount = sum(i[4] for i in items)
     for _ in range(args.warmup):
-        for scheme, x, wq, sw, _, wo in items:
-            _oracle_run(scheme, x, wq, sw, wo, threads)
+        for scheme, x, wq, sw, _, kind in items:
+            _oracle_run(scheme, x, wq, sw, kind, threads)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        for scheme, x, wq, sw, _, wo in items:
-            _oracle_run(scheme, x, wq, sw, wo, threads)
+        for scheme, x, wq, sw, _, kind in items:
+            _oracle_run(scheme, x, wq, sw, kind, threads)
     dt = time.perf_counter() - t0
     scale = 1e9 if wl.unit == "GB/s" else 1e12
     value = step_amount * args.steps / dt / scale

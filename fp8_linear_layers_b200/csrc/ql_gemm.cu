@@ -432,18 +432,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc::fence_after();
           // 64 columns: 32-column loads; 128 columns: 16-column loads (registers)
           constexpr int kW = Cfg::kHalf == 64 ? 32 : 16;
-#pragma unroll
-          for (int c = 0; c < Cfg::kHalf / kW; ++c) {
-            uint32_t r[kW];
+          constexpr int kChunks = Cfg::kHalf / kW;
+          const uint32_t tbase = tmem + lane_base + buf * Cfg::kBufCols + c0;
+          auto ldw = [&](int c, uint32_t (&r)[kW]) {
             if constexpr (kW == 32)
-              tc::ld32(tmem + lane_base + buf * Cfg::kBufCols + c0 + c * kW, r);
+              tc::ld32(tbase + c * kW, r);
             else
-              tc::ld16(tmem + lane_base + buf * Cfg::kBufCols + c0 + c * kW, r);
-            tc::ld_wait();
+              tc::ld16(tbase + c * kW, r);
+          };
+          // software pipeline: chunk c + 1 is loaded while chunk c is promoted
+          uint32_t rb[2][kW];
+          ldw(0, rb[0]);
+          tc::ld_wait();
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) {
+            if (c + 1 < kChunks) ldw(c + 1, rb[(c + 1) & 1]);
 #pragma unroll
             for (int j = 0; j < kW / 2; ++j)
-              acc[(c * kW) / 2 + j] = __ffma2_rn(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])),
+              acc[(c * kW) / 2 + j] = __ffma2_rn(make_float2(__uint_as_float(rb[c & 1][2 * j]), __uint_as_float(rb[c & 1][2 * j + 1])),
                                                  make_float2(scale, scale), acc[(c * kW) / 2 + j]);
+            if (c + 1 < kChunks) tc::ld_wait();
           }
           tc::fence_before();
           __syncwarp();
@@ -469,7 +477,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // adds the two (f32 addition commutes: the same bits in either order
           // of arrival) and writes y.  (Adding the halves with L2 reductions
           // measured slower than the work saved.)
-          const int half = hi == p.nkb ? 1 : 0;  // the second half ends at the last K block
+          // this item's part of the tile's K blocks: lo = floor(part nkb / split)
+          const int half = (int)(((int64_t)lo * p.split + p.nkb - 1) / p.nkb);
           constexpr int kV = Cfg::kHalf / 4;     // float4 per thread
           auto slot = [&](int hf) {
             return reinterpret_cast<float4*>(p.parts) +
@@ -490,7 +499,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           named_bar_sync(kGemmEpiBar, kGemmEpiWarps * 32);
           if (!*last_flag) return true;
           __threadfence();
-          {
+          if (p.split == 2) {
             const float4* other = slot(1 - half);
             // eight 16-byte loads in flight at a time (the 128 running sums
             // leave no registers for more)
@@ -507,8 +516,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
               asm volatile("" ::: "memory");
             }
+          } else if constexpr (BN == 128) {
+            // more parts (128-wide tiles only): summed in part order 0, 1, ..., split - 1 whichever
+            // arrives last (this CTA's own part from its registers), so the
+            // bits do not depend on the order of arrival
+#pragma unroll
+            for (int j0 = 0; j0 < kV; j0 += 4) {
+              float4 tot[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) tot[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+              for (int hf = 0; hf < p.split; ++hf) {
+                float4 v[4];
+                if (hf == half) {
+#pragma unroll
+                  for (int j = 0; j < 4; ++j)
+                    v[j] = make_float4(acc[2 * (j0 + j)].x, acc[2 * (j0 + j)].y, acc[2 * (j0 + j) + 1].x,
+                                       acc[2 * (j0 + j) + 1].y);
+                } else {
+                  const float4* o = slot(hf);
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) v[j] = __ldcg(o + (j0 + j) * 32);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  tot[j] = make_float4(tot[j].x + v[j].x, tot[j].y + v[j].y, tot[j].z + v[j].z, tot[j].w + v[j].w);
+              }
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                acc[2 * (j0 + j)] = make_float2(tot[j].x, tot[j].y);
+                acc[2 * (j0 + j) + 1] = make_float2(tot[j].z, tot[j].w);
+              }
+              asm volatile("" ::: "memory");
+            }
           }
-          if (ew == 0 && lane == 0) p.counters[t] = 0u;  // both halves have arrived
+          if (ew == 0 && lane == 0) p.counters[t] = 0u;  // every part has arrived
         }
         const int mrow = m0 + q * 32;
         if constexpr (kQ) {
@@ -624,22 +665,34 @@ struct GemmPlan {
 static GemmPlan plan_gemm(ql_scheme s, int64_t M, int64_t N, int64_t K, int sms) {
   GemmPlan pl{pick_bn(s, M, N, sms), 1};
   if (s != QL_FP8_E4M3_BLOCK128) return pl;
-  const int64_t tiles = ((M + kGemmBM - 1) / kGemmBM) * ((N + 255) / 256);
+  const int64_t mt = (M + kGemmBM - 1) / kGemmBM;
+  const int64_t tiles = mt * ((N + 255) / 256);
   const int64_t nkb = (K + kGemmBK - 1) / kGemmBK;
-  if (2 * tiles <= sms && nkb >= 64) pl = GemmPlan{256, 2};
+  if (2 * tiles <= sms && nkb >= 64) return GemmPlan{256, 2};
+  // Tiles of the chosen width that fill at most a quarter of the SMs (small
+  // N, e.g. k/v at M = 512: 32 tiles of 128): split each tile's K blocks over
+  // 2, 4 or 8 CTAs, as many as fit one wave, keeping >= 8 K blocks a part.
+  const int64_t t_bn = mt * ((N + pl.bn - 1) / pl.bn);
+  int split = 1;
+  while (pl.bn == 128 && split < 8 && 4 * t_bn * split <= 2 * sms && t_bn * split * 2 <= sms &&
+         nkb / (split * 2) >= 8)
+    split *= 2;
+  if (split > 1) pl.split = split;
   return pl;
 }
 
 static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
-// Two slabs of one 128 x 256 f32 tile per tile.
-static size_t split_parts_bytes(int64_t tiles) { return (size_t)2 * tiles * kGemmBM * 256 * 4; }
+// One slab of one 128 x 256 f32 tile per part per tile.
+static size_t split_parts_bytes(int64_t tiles, int split) {
+  return (size_t)split * tiles * kGemmBM * 256 * 4;
+}
 
 size_t gemm_workspace_bytes(ql_scheme s, int64_t M, int64_t N, int64_t K, int sms) {
   const GemmPlan pl = plan_gemm(s, M, N, K, sms);
   if (pl.split == 1) return 0;
   const int64_t tiles = ((M + kGemmBM - 1) / kGemmBM) * ((N + pl.bn - 1) / pl.bn);
-  return align256(split_parts_bytes(tiles)) + align256((size_t)tiles * 4);
+  return align256(split_parts_bytes(tiles, pl.split)) + align256((size_t)tiles * 4);
 }
 
 template <ql_scheme S, int BN, bool kQ = false>
@@ -686,7 +739,7 @@ cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const
   p.split = pl.split;
   p.parts = pl.split > 1 ? static_cast<float*>(workspace) : nullptr;
   p.counters = pl.split > 1 ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) +
-                                                          align256(split_parts_bytes((int64_t)p.mt * p.nt)))
+                                                          align256(split_parts_bytes((int64_t)p.mt * p.nt, pl.split)))
                             : nullptr;
   p.acc_i32 = dbg ? dbg->acc_i32 : nullptr;
   p.acc_f32 = dbg ? dbg->acc_f32 : nullptr;

@@ -57,7 +57,8 @@ constexpr int kGemvThreads = kGemvConsumers + 32;
 constexpr int kGemvMaxStages = 6;
 constexpr int kEarlyStages = 2;                 // stages copied before x is quantized
 constexpr int kGemvStageTarget = 32768;
-constexpr int kGemvSmemBudget = 200 * 1024;     // one CTA per SM
+constexpr int kGemvSmemBudget = 224 * 1024;     // one CTA per SM
+constexpr int64_t kGemvStashMaxK = 16384;       // one token's bf16 x parked in shared memory up to this K
 constexpr int kGemvMaxK = 32768;
 constexpr int64_t kGemvMaxK2 = 16384;           // two tokens: units of at most 64 windows
 constexpr int64_t kGemvMaxK4 = 8192;            // three or four tokens: stages of 8 rows
@@ -94,7 +95,7 @@ struct GemvParams {
 };
 
 struct GemvSmemLayout {
-  int ring, qx, sx, swc, part, bars, flags, total;
+  int ring, qx, stash, sx, swc, part, bars, flags, total;
 };
 
 // Shared-memory carve-up; `sw_floats` is the number of weight scales cached,
@@ -107,6 +108,8 @@ __host__ __device__ inline GemvSmemLayout gemv_layout(int64_t K, int stage_bytes
   off += stages * stage_bytes;
   L.qx = off;  // M rows of K codes (or f16 values), each padded to whole 128-element blocks
   off += M * (int)((K + 127) / 128) * 128 * xelem;
+  L.stash = off;  // one token's bf16 x, read once from global memory and quantized from here
+  off += (M == 1 && K <= kGemvStashMaxK) ? (int)((K * 2 + 127) / 128 * 128) : 0;
   L.sx = off;
   off += (int)((M * (K / 128 + 1) + 31) / 32) * 128;
   L.swc = off;
@@ -311,6 +314,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   for (int i = tid; i < sw_cached; i += kGemvConsumers) sw_s[i] = __ldg(psw + sw_first + i);
 
   tc::grid_dependency_wait();  // x may be produced by the previous kernel
+  bool xready_done = false;  // xready arrives once, as soon as x is loaded where the path allows
   // 1. Fused activation quantization of x [kM, K] into shared memory: one pass
   //    for the absmax (the first kXLoads chunks per thread loaded together),
   //    one for the codes (x is L2-resident by then).
@@ -324,9 +328,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     const int64_t nchunk8 = K / 8;  // 16-byte chunks of 8 bf16
     constexpr int kXLoads = 8;
     const uint4* xg = reinterpret_cast<const uint4*>(px);
-    uint4* stash = nst > kEarlyStages && (int64_t)p.stage_bytes >= nchunk8 * 16
-                       ? reinterpret_cast<uint4*>(ring + kEarlyStages * p.stage_bytes)
-                       : nullptr;
+    uint4* stash = K <= kGemvStashMaxK ? reinterpret_cast<uint4*>(smem + L.stash) : nullptr;
     float a_tok = 0.0f;
 #pragma unroll
     for (int i = 0; i < kXLoads; ++i) {
@@ -343,6 +345,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     a_tok = warp_max(a_tok);
     if (lane == 0) blockred[warp] = a_tok;
     named_bar_sync(kBarConsumers, kGemvConsumers);
+    if (tid == 0) mbar_arrive(xready);  // x is loaded: the producer may fill the ring
+    xready_done = true;
     float a = blockred[0];
 #pragma unroll
     for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, blockred[w]);
@@ -363,7 +367,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
                           f32x2_to_f16x2(bf16_lo(v.z) * up, bf16_hi(v.z) * up),
                           f32x2_to_f16x2(bf16_lo(v.w) * up, bf16_hi(v.w) * up));
     }
-    if (stash) fence_proxy_async_smem();
     // zero the padding of the last 64-element window so it adds nothing
     for (int64_t b = 2 * K + tid * 16; b < 2 * ((K + 63) / 64 * 64); b += kGemvConsumers * 16)
       *reinterpret_cast<uint4*>(qx_s + b) = make_uint4(0, 0, 0, 0);
@@ -450,13 +453,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         }
       }
     } else {
-      // Ring slot kEarlyStages is not written before x is quantized (the
-      // producer waits for xready there): when x fits, the absmax pass parks
-      // its chunks in that slot and the code pass reads them from shared
-      // memory instead of a second trip to L2.
-      uint4* stash = nst > kEarlyStages && (int64_t)p.stage_bytes >= nchunk8 * 16
-                         ? reinterpret_cast<uint4*>(ring + kEarlyStages * p.stage_bytes)
-                         : nullptr;
+      // When x fits, the absmax pass parks its chunks in shared memory and
+      // the code pass reads them there instead of a second trip to L2; the
+      // producer resumes the weight stream as soon as x is loaded (xready),
+      // while the codes are computed.
+      uint4* stash = K <= kGemvStashMaxK ? reinterpret_cast<uint4*>(smem + L.stash) : nullptr;
       float a_tok = 0.0f;
 #pragma unroll
       for (int i = 0; i < kXLoads; ++i) {
@@ -473,6 +474,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       a_tok = warp_max(a_tok);
       if (lane == 0) blockred[warp] = a_tok;
       named_bar_sync(kBarConsumers, kGemvConsumers);
+      if (tid == 0) mbar_arrive(xready);  // x is loaded: the producer may fill the ring
+      xready_done = true;
       float a = blockred[0];
 #pragma unroll
       for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, blockred[w]);
@@ -499,8 +502,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         emit_all(std::true_type{});
       else
         emit_all(std::false_type{});
-      // the slot's next writer is the producer's bulk copy (the async proxy)
-      if (stash) fence_proxy_async_smem();
     }
     // zero the padding of the last 64-byte window so it adds nothing
     for (int64_t b = K + tid * 16; b < (K + 63) / 64 * 64; b += kGemvConsumers * 16)
@@ -612,7 +613,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         *reinterpret_cast<uint4*>(qx_s + tok * xstride + b) = make_uint4(0, 0, 0, 0);
     named_bar_sync(kBarConsumers, kGemvConsumers);
   }
-  if (tid == 0) mbar_arrive(xready);  // the producer may fill the whole ring now
+  if (tid == 0 && !xready_done) mbar_arrive(xready);  // the producer may fill the whole ring now
   if (!kWO && blockIdx.x == 0 && (p.dbg.qx || p.dbg.sx)) {  // product 0's first CTA
     // [token, K] codes and [token, groups] scales; rows of K bytes (K % 16 == 0)
     const int ns = kBlock ? (int)KB : 1;

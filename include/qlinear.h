@@ -212,9 +212,9 @@ ql_status qlinear_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const vo
  * weight scale; tolerance |y - y_exact| <= 2^-7 |y_exact| + 1e-3).  Same
  * pages as qlinear_gemv_weight_only; the W8A8 and Qwen3 FP8 pages run up to
  * 32 tokens on the tensor cores ("Loading").  Up to four tokens ride on the
- * weight-only GEMV kernel's spare MMA columns (K up to 16384 for one token,
- * 15744 for two, 7584 for three or four: the staged f16 tokens and two
- * weight stages must fit the shared memory); other shapes run on the tensor
+ * weight-only GEMV kernel's spare MMA columns (K up to 16384 for one or two
+ * tokens, 8192 for three or four: the staged f16 tokens and two weight
+ * stages must fit the shared memory); other shapes run on the tensor
  * cores (tcgen05 kind::f16: the codes are converted exactly to bf16 in
  * shared memory and multiplied with the bf16 x, K split across the SMs).
  *   x          device, bf16 [M,K];  y  device, out: bf16 [M,N]
@@ -278,19 +278,21 @@ ql_status qlinear_gemm_small_prequant(ql_scheme scheme, const void* qx, const fl
  * accumulation); Qwen3 FP8 "Loading" (block scales).
  *   qx, sx     device, from qlinear_quantize_act
  *   workspace  optional (NULL / 0 bytes: whole tiles).  Block scheme only:
- *              when the 128x256 output tiles fill at most half the SMs (e.g.
- *              M = 512 with N = 4096, or N = 1024) and K >= 8192, a
- *              workspace of at least qlinear_workspace_bytes(...) bytes
- *              (256-byte aligned, ZERO-FILLED before its first use) lets the
- *              call split each tile's K blocks in two halves run by two CTAs
- *              that park their f32 partial sums in it (two 128x256 f32
- *              tiles per output tile, then one arrival counter per tile);
- *              the second to arrive adds the two (the same bits in either
- *              order).  A completed call leaves the
- *              counters zero again, for any next shape; zero the workspace
- *              again after a QL_ERR_TIMEOUT.  Two calls in flight at the same
- *              time must not share it.  Row schemes: qlinear_workspace_bytes
- *              returns 0.
+ *              when the output tiles are few -- 128x256 tiles filling at
+ *              most half the SMs with K >= 8192 (e.g. M = 512, N = 4096), or
+ *              128x128 tiles filling at most a quarter of them (e.g. M = 512,
+ *              N = 1024) -- a workspace of at least
+ *              qlinear_workspace_bytes(...) bytes (256-byte aligned,
+ *              ZERO-FILLED before its first use) lets the call split each
+ *              tile's K blocks over 2 (or, for 128-wide tiles, up to 4) CTAs
+ *              that park their f32 partial sums in it (one 128x256 f32 slab
+ *              per part per output tile, then one arrival counter per tile);
+ *              the last to arrive adds the parts in part order (the same
+ *              bits whatever the order of arrival).  A completed call leaves
+ *              the counters zero again, for any next shape; zero the
+ *              workspace again after a QL_ERR_TIMEOUT.  Two calls in flight
+ *              at the same time must not share it.  Row schemes:
+ *              qlinear_workspace_bytes returns 0.
  *   dbg        optional (NULL): acc_i32 (int8) / acc_f32 (E4M3 row) [M,N] */
 ql_status qlinear_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
                        const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,

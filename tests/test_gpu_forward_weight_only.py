@@ -1,8 +1,8 @@
 """GPU parity: the weight-only product for 1 <= M <= 32 tokens vs the oracle.
 
 Up to four tokens ride on the GEMV kernel's spare MMA columns (each token
-staged with its own power of two) within its K limits (16384 / 15744 / 7584
-for one / two / three or four tokens); every other shape runs on the tensor
+staged with its own power of two) within its K limits (16384 for one or two
+tokens, 8192 for three or four); every other shape runs on the tensor
 cores (tcgen05 kind::f16, the codes converted to bf16 in shared memory, K
 split over the SMs).  Llama-3.1-8B shapes, Qwen3-8B block shapes, ragged
 shapes, workspace reuse across calls, and the argument limits.
@@ -49,9 +49,10 @@ def test_forward_weight_only_qwen_block(cuda, M, name, N, K):
     _run(ql.FP8_E4M3_BLOCK128, M, N, K, outliers=0)
 
 
-@pytest.mark.parametrize("M,N,K", [(2, 37, 256), (3, 129, 4112), (4, 5, 6144), (2, 300, 15744),
-                                   (3, 150, 7584), (1, 1000, 1024), (5, 37, 272), (7, 1000, 4112),
-                                   (3, 150, 7600), (1, 130, 20000), (17, 300, 2064), (32, 128, 128)])
+@pytest.mark.parametrize("M,N,K", [(2, 37, 256), (3, 129, 4112), (4, 5, 6144), (2, 300, 16384),
+                                   (3, 150, 8192), (1, 1000, 1024), (5, 37, 272), (7, 1000, 4112),
+                                   (3, 150, 8208), (1, 130, 20000), (17, 300, 2064), (32, 128, 128),
+                                   (2, 64, 16400)])
 @pytest.mark.parametrize("scheme", [ql.W8A8_INT8_ROW, ql.FP8_E4M3_ROW])
 def test_forward_weight_only_odd_shapes(cuda, M, N, K, scheme):
     _run(scheme, M, N, K, outliers=min(3, K))
@@ -59,7 +60,7 @@ def test_forward_weight_only_odd_shapes(cuda, M, N, K, scheme):
 
 def test_forward_weight_only_limits(cuda):
     # the GEMV route's K limits, as the library reports them through the workspace size
-    for M, K in ((1, 16384), (2, 15744), (3, 7584), (4, 7584)):
+    for M, K in ((1, 16384), (2, 16384), (3, 8192), (4, 8192)):
         assert ql.weight_only_workspace_bytes(ql.FP8_E4M3_ROW, M, 256, K) == 0
         assert ql.weight_only_workspace_bytes(ql.FP8_E4M3_ROW, M, 256, K + 16) > 0
     assert ql.weight_only_workspace_bytes(ql.FP8_E4M3_ROW, 5, 256, 256) > 0

@@ -125,3 +125,4 @@ def test_grouped_argument_checks(cuda):
     assert L.qlinear_gemv_grouped(ql.FP8_E4M3_ROW, tp, 1, 100, stream) == 2  # K % 16 != 0
     torch.cuda.synchronize()
     assert torch.count_nonzero(y).item() == 0
+
