@@ -312,7 +312,7 @@ _GEMV_SOURCES = ["ql_gemv.cu", "ql_common.cuh", "ql_tc.cuh", "ql_internal.h"]
 KERNEL_SOURCES = {"ql::gemv_kernel": _GEMV_SOURCES, "ql::gemv_kernel (weight-only)": _GEMV_SOURCES}
 TRAFFIC = {
     # workload: (bytes per launch, kernel source hash, summary file)
-    "decode": (31236974, "233ea157dd920e9f", "profiles/gemv_decode_dram.md"),
+    "decode": (54668224, "f67eb144cf9e747e", "profiles/gemv_decode_dram.md"),
     "decode-wo": (31224887, "233ea157dd920e9f", "profiles/gemv_decode_weight_only_dram.md"),
 }
 
@@ -438,11 +438,14 @@ class Runner:
 
     def dominant(self, t):
         """Launches of the dominant kernel alone (the product on quantized inputs)."""
-        ql = self.ql
         for g in self.groups:
-            if self._grouped(g) or g["p0"].pre:  # one kernel per launch already
-                self._run_group(g, g["x_in"][t], t)
-                continue
+            self.dominant_group(g, t)
+
+    def dominant_group(self, g, t):
+        ql = self.ql
+        if self._grouped(g) or g["p0"].pre:  # one kernel per launch already
+            self._run_group(g, g["x_in"][t], t)
+        else:
             for i in g["items"]:
                 p = i["p"]
                 wq, sw = self._w(i, t)
@@ -787,6 +790,31 @@ def run_reference(args):
 EXTRA_WORKLOADS = ("kproj", "prefill", "qwen-prefill")
 
 
+def per_product_times(torch, run, stream, wl, peak, scale, reps=50):
+    """Each product's dominant-kernel launches (its group's, when grouped)
+    timed alone: graph replays cycling through the input copies, CUDA events;
+    the product's algorithmic amount over its time, and that against the
+    roofline peak."""
+    out = []
+    for g in run.groups:
+        def fn(t, g=g):
+            run.dominant_group(g, t)
+        graphs = run.capture(fn, stream)
+        with torch.cuda.stream(stream):
+            for i in range(5):
+                graphs[i % len(graphs)].replay()
+        ms = timed(torch, stream, graphs, reps) / reps
+        amount = sum(i["amount"] for i in g["items"])
+        if wl.unit == "GB/s":  # a grouped launch reads its shared input once
+            amount -= (len(g["items"]) - 1) * Workload.input_bytes(g["p0"])
+        v = amount / (ms / 1e3) / scale
+        p = g["p0"]
+        out.append({"products": "|".join(i["p"].name for i in g["items"]), "scheme": SCHEME_NAME[p.scheme],
+                    "M": p.M, "us": round(ms * 1e3, 2), "value": round(v, 1), "frac": round(v / peak, 4)})
+        del graphs
+    return out
+
+
 def measure(torch, ql, synthetic, wl, args, steps, warmup, world, rank, barrier, max_over_ranks,
             cpu_seconds):
     """Every leg of one workload's line: the timed graph replays, the dominant
@@ -834,6 +862,7 @@ def measure(torch, ql, synthetic, wl, args, steps, warmup, world, rank, barrier,
                 "duration_source": "CUDA events over graph replays of this kernel's launches "
                                    "(inputs already quantized where the step quantizes separately)"}
     del dgraphs
+    per_product = per_product_times(torch, run, stream, wl, peak, scale) if len(run.groups) > 1 else None
 
     # ---- end to end through the public API with host buffers
     e2e_steps = args.e2e_steps or max(10, min(steps, 1000))
@@ -883,6 +912,7 @@ def measure(torch, ql, synthetic, wl, args, steps, warmup, world, rank, barrier,
                           f"touched per cycle ({weight_bytes / 1e6:.0f} MB of weights per step); no flush"),
                    "timing": "one CUDA graph replay per step, CUDA events on the launch stream"},
         "roofline": roofline,
+        **({"per_product": per_product} if per_product else {}),
         "parity": parity,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 1), "unit": wl.unit, "h2d_bytes_per_step": h2d,
