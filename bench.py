@@ -309,11 +309,15 @@ L2_BYTES = 126e6
 # dram__bytes_write.sum), with the hash of the kernel sources it was taken on: when the
 # sources differ the figure no longer describes the kernel and the line reports null.
 _GEMV_SOURCES = ["ql_gemv.cu", "ql_common.cuh", "ql_tc.cuh", "ql_internal.h"]
-KERNEL_SOURCES = {"ql::gemv_kernel": _GEMV_SOURCES, "ql::gemv_kernel (weight-only)": _GEMV_SOURCES}
+_GEMM_SOURCES = ["ql_gemm.cu", "ql_common.cuh", "ql_tc.cuh", "ql_internal.h"]
+KERNEL_SOURCES = {"ql::gemv_kernel": _GEMV_SOURCES, "ql::gemv_kernel (weight-only)": _GEMV_SOURCES,
+                  "ql::gemm_kernel": _GEMM_SOURCES, "ql::gemm_kernel (output quantization fused)": _GEMM_SOURCES}
 TRAFFIC = {
     # workload: (bytes per launch, kernel source hash, summary file)
     "decode": (54668224, "f67eb144cf9e747e", "profiles/gemv_decode_dram.md"),
     "decode-wo": (31224887, "233ea157dd920e9f", "profiles/gemv_decode_weight_only_dram.md"),
+    "prefill": (56031552, "8efbefd47af5ee25", "profiles/gemm_prefill_int8_dram.md"),
+    "qwen-prefill": (30451895, "8efbefd47af5ee25", "profiles/gemm_qwen_prefill_block_dram.md"),
 }
 
 
