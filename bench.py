@@ -148,8 +148,10 @@ def workloads():
         [Product(n, s, 1, N, K, oc(K)) for n, N, K in S.LLAMA31_8B_FUSED for s in (INT8, FP8R)])
     w["prefill"] = Workload(
         "prefill", "prefill W8A8 int8 GEMM: M in {512, 1024} x Llama-3.1-8B gate/up 14336x4096, "
-        "down 4096x14336, fused qkv 6144x4096; per-token quantization + tcgen05 kind::i8", "TOPS",
-        [Product(n, INT8, M, N, K, oc(K)) for M in (512, 1024) for n, N, K in S.LLAMA31_8B_PREFILL])
+        "down 4096x14336, fused qkv 6144x4096; per-token quantization + tcgen05 kind::i8; gate|up one "
+        "grouped launch on their shared input", "TOPS",
+        [Product(n, INT8, M, N, K, oc(K), group=LAYER_INPUT.get(n, n)) for M in (512, 1024)
+         for n, N, K in S.LLAMA31_8B_PREFILL])
     w["small"] = Workload(
         "small", "small-batch tensor-core path: M in {2, 8, 16, 32} x the 7 Llama-3.1-8B shapes x "
         "{W8A8 int8, FP8 E4M3 per-row}, quantization fused", "GB/s",
@@ -183,11 +185,13 @@ def workloads():
     w["qwen-prefill-f2"] = Workload(
         "qwen-prefill-f2", "Qwen3-8B FP8 128x128-block projections at M=512 (7 shapes), each input "
         "arriving already quantized and each product also writing its own output's E4M3 codes and "
-        "per-128 scales for the product that reads it next: one kernel per projection", "TOPS",
-        [Product(n, FP8B, 512, N, K, 0, pre=True) for n, N, K in S.QWEN3_8B])
+        "per-128 scales for the product that reads it next: one kernel per projection (q|k|v and "
+        "gate|up read one input each)", "TOPS",
+        [Product(n, FP8B, 512, N, K, 0, group=LAYER_INPUT.get(n, n), pre=True) for n, N, K in S.QWEN3_8B])
     w["qwen-prefill"] = Workload(
         "qwen-prefill", "Qwen3-8B FP8 128x128-block projections at M=512 (7 shapes), per-K-block "
-        "promotion", "TOPS", [Product(n, FP8B, 512, N, K, 0) for n, N, K in S.QWEN3_8B])
+        "promotion; q|k|v and gate|up one grouped launch each on their shared input", "TOPS",
+        [Product(n, FP8B, 512, N, K, 0, group=LAYER_INPUT.get(n, n)) for n, N, K in S.QWEN3_8B])
     return w
 
 
@@ -316,8 +320,6 @@ TRAFFIC = {
     # workload: (bytes per launch, kernel source hash, summary file)
     "decode": (54668224, "f67eb144cf9e747e", "profiles/gemv_decode_dram.md"),
     "decode-wo": (31224887, "233ea157dd920e9f", "profiles/gemv_decode_weight_only_dram.md"),
-    "prefill": (56031552, "8efbefd47af5ee25", "profiles/gemm_prefill_int8_dram.md"),
-    "qwen-prefill": (30451895, "8efbefd47af5ee25", "profiles/gemm_qwen_prefill_block_dram.md"),
 }
 
 
@@ -344,7 +346,8 @@ class Runner:
     """Device buffers and launch closures for one workload (public API calls only).
 
     Products of one (scheme, group) read one input; M = 1 ones run as one
-    grouped GEMV launch.  Steps cycle through `copies` independent sets of
+    grouped GEMV launch, M > 32 ones as one quantization of the input and one
+    grouped GEMM launch.  Steps cycle through `copies` independent sets of
     quantized weights, activations and outputs, enough that the bytes touched
     by consecutive steps exceed twice the L2: no step finds its inputs in L2
     from an earlier one, so no flush is needed between timed steps.
@@ -380,17 +383,26 @@ class Runner:
                 item["qy"] = [(torch.empty((p.M, p.N), dtype=torch.uint8, device="cuda"),
                                torch.empty((p.M, p.N // 128), dtype=torch.float32, device="cuda"))
                               for _ in range(self.copies)]
-            if p.M > 32:  # pre-quantized activations for the dominant-kernel timing
-                item["q"] = g["x_in"] if p.pre else [ql.quantize_act(p.scheme, x) for x in g["xs"]]
+            if p.M > 32 and p.pre:  # quantized activations for the dominant-kernel timing
+                item["q"] = g["x_in"]
                 gws = ql.workspace_bytes(p.scheme, p.M, p.N, p.K)  # the K split's sums (block scheme)
                 item["ws_gemm"] = ql.new_workspace(gws) if gws else None
             g["items"].append(item)
         del weights
+        for g in self.groups:
+            p = g["p0"]
+            if gemm_grouped_route(p):
+                # the step's quantized input (written by the step), a quantized copy of each
+                # input for the dominant-kernel timing, and the group's K-split workspace
+                g["qbuf"] = ql.quantize_act(p.scheme, g["xs"][0])
+                g["q"] = [ql.quantize_act(p.scheme, x) for x in g["xs"]]
+                gws = ql.gemm_grouped_workspace_bytes(p.scheme, [i["p"].N for i in g["items"]], p.M, p.K)
+                g["ws_gemm"] = ql.new_workspace(gws) if gws else None
         torch.cuda.synchronize()
         self.items = [i for g in self.groups for i in g["items"]]
         self.step_amount = step_amount(wl)  # a group reads its one input once
         self.launches_per_step = sum(self._launches(g) for g in self.groups)
-        self.dominant_launches = sum(self._grouped(g) or len(g["items"]) for g in self.groups)
+        self.dominant_launches = dominant_launch_count(wl)
 
     @staticmethod
     def _grouped(g) -> int:
@@ -402,6 +414,8 @@ class Runner:
     def _launches(self, g) -> int:
         if self._grouped(g):
             return 1
+        if gemm_grouped_route(g["p0"]):
+            return 2
         return sum(1 if (i["p"].wo or i["p"].pre or gemv_route(i["p"].M, i["p"].K)) else 2
                    for i in g["items"])
 
@@ -422,6 +436,11 @@ class Runner:
         ys = ys or [i["ys"][t] for i in items]
         if self._grouped(g):
             self.ql.gemv_grouped(g["p0"].scheme, [(x, *self._w(i, t), y) for i, y in zip(items, ys)])
+        elif gemm_grouped_route(g["p0"]):
+            qx, sx = g["qbuf"]
+            self.ql.quantize_act(g["p0"].scheme, x, qx, sx)
+            self.ql.gemm_grouped(g["p0"].scheme, qx, sx, [(*self._w(i, t), y) for i, y in zip(items, ys)],
+                                 workspace=g["ws_gemm"])
         elif g["p0"].pre:
             qx, sx = x
             for i, y in zip(items, ys):
@@ -449,6 +468,10 @@ class Runner:
         ql = self.ql
         if self._grouped(g) or g["p0"].pre:  # one kernel per launch already
             self._run_group(g, g["x_in"][t], t)
+        elif gemm_grouped_route(g["p0"]):
+            qx, sx = g["q"][t]
+            ql.gemm_grouped(g["p0"].scheme, qx, sx, [(*self._w(i, t), i["ys"][t]) for i in g["items"]],
+                            workspace=g["ws_gemm"])
         else:
             for i in g["items"]:
                 p = i["p"]
@@ -532,6 +555,37 @@ def whole_job_value(world: int, amount_per_step: float, steps: int, ms: float, s
     """Replicas: every rank runs the same step, so the job moves world x the
     step's amount in the max-over-ranks time."""
     return world * amount_per_step * steps / (ms / 1e3) / scale
+
+
+def gemm_grouped_route(p: Product) -> bool:
+    """True when a group of M > 32 products runs as one quantization of its
+    input and one qlinear_gemm_grouped launch (a group of one included)."""
+    return p.M > 32 and not p.pre and not p.wo
+
+
+def dominant_launch_count(wl) -> int:
+    """Launches of the dominant kernel in one step: one per group that runs
+    grouped (M = 1 quantized GEMV, M > 32 GEMM), else one per product."""
+    n = 0
+    for g in input_groups(wl):
+        p = g[0]
+        n += 1 if ((p.M == 1 and not p.wo) or gemm_grouped_route(p)) else len(g)
+    return n
+
+
+def step_bytes(wl) -> float:
+    """Algorithmic HBM bytes of one step's dominant launches: weights, scales,
+    the kernel's input (q_x and s_x when M > 32; a group's input once) and y."""
+    total = 0.0
+    for g in input_groups(wl):
+        for j, p in enumerate(g):
+            sw = 4 * (p.N // 128) * (p.K // 128) if p.scheme == FP8B else 4 * p.N
+            if p.M > 32:
+                inp = p.M * p.K + 4 * p.M * (p.K // 128 if p.scheme == FP8B else 1)
+            else:
+                inp = Workload.input_bytes(p)
+            total += p.N * p.K + sw + 2 * p.M * p.N + (inp if j == 0 else 0)
+    return total
 
 
 def input_groups(wl):

@@ -42,7 +42,8 @@ EXPORTS = ("qlinear_quantize_weight", "qlinear_quantize_act", "qlinear_gemv", "q
            "qlinear_last_cuda_error", "qlinear_gemm_small_noalloc", "qlinear_gemv_weight_only",
            "qlinear_debug_gemv_stalled", "qlinear_forward_weight_only", "qlinear_gemv_grouped",
            "qlinear_gemv_prequant", "qlinear_gemm_small_prequant",
-           "qlinear_gemm_quant_out", "qlinear_weight_only_workspace_bytes")
+           "qlinear_gemm_quant_out", "qlinear_weight_only_workspace_bytes", "qlinear_gemm_grouped",
+           "qlinear_gemm_grouped_workspace_bytes")
 
 
 class QLinearError(RuntimeError):
@@ -98,6 +99,9 @@ def lib() -> ctypes.CDLL:
         L.qlinear_gemm_quant_out.argtypes = [i32, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp, sz, vp]
         L.qlinear_gemm_small.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp, vp]
         L.qlinear_gemm.argtypes = [i32, vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp, vp]
+        L.qlinear_gemm_grouped.argtypes = [i32, vp, vp, vp, i32, i64, i64, vp, sz, vp]
+        L.qlinear_gemm_grouped_workspace_bytes.argtypes = [i32, vp, i32, i64, i64]
+        L.qlinear_gemm_grouped_workspace_bytes.restype = sz
         L.qlinear_forward.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]
         L.qlinear_gemm_small_noalloc.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp]
         L.qlinear_workspace_bytes.argtypes = [i32, i64, i64, i64]
@@ -382,6 +386,44 @@ def gemm(scheme: int, qx: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: 
                               _dev(y, torch.bfloat16, "y"), wp, wn, debug._c() if debug else None,
                               _stream(stream)), "qlinear_gemm")
     return y
+
+
+GEMM_MAX_GROUP = 4  # QL_GEMM_MAX_GROUP
+
+
+class _GemmProblem(ctypes.Structure):
+    _fields_ = [("wq", ctypes.c_void_p), ("sw", ctypes.c_void_p), ("y", ctypes.c_void_p), ("N", ctypes.c_int64)]
+
+
+def gemm_grouped_workspace_bytes(scheme: int, Ns, M: int, K: int) -> int:
+    arr = (ctypes.c_int64 * len(Ns))(*Ns)
+    return int(lib().qlinear_gemm_grouped_workspace_bytes(scheme, ctypes.cast(arr, ctypes.c_void_p), len(Ns),
+                                                          M, K))
+
+
+def gemm_grouped(scheme: int, qx: torch.Tensor, sx: torch.Tensor, problems, workspace: torch.Tensor | None = None,
+                 stream=None) -> list:
+    """Several large-M products on one quantized input in one launch.
+    `problems` is a list of (wq [N,K], sw, y or None); returns the outputs [M,N]."""
+    if not 1 <= len(problems) <= GEMM_MAX_GROUP:
+        raise ValueError(f"1 to {GEMM_MAX_GROUP} products per grouped launch")
+    M, K = qx.shape
+    table = (_GemmProblem * len(problems))()
+    ys = []
+    for j, (wq, sw, y) in enumerate(problems):
+        if wq.shape[1] != K:
+            raise ValueError("every product of a grouped launch reads the same [M,K] input")
+        N = wq.shape[0]
+        if y is None:
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device)
+        table[j] = _GemmProblem(_dev(wq, torch.uint8, "wq"), _dev(sw, torch.float32, "sw"),
+                                _dev(y, torch.bfloat16, "y"), N)
+        ys.append(y)
+    wp, wn = _ws(workspace)
+    _check(lib().qlinear_gemm_grouped(scheme, _dev(qx, torch.uint8, "qx"), _dev(sx, torch.float32, "sx"),
+                                      ctypes.cast(table, ctypes.c_void_p), len(problems), M, K, wp, wn,
+                                      _stream(stream)), "qlinear_gemm_grouped")
+    return ys
 
 
 def gemm_quant_out(scheme: int, qx: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,

@@ -369,6 +369,48 @@ ql_status qlinear_gemm_quant_out(ql_scheme scheme, const void* qx, const float* 
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm_quant_out");
 }
 
+ql_status qlinear_gemm_grouped(ql_scheme scheme, const void* qx, const float* sx,
+                               const ql_gemm_problem* problems, int count, int64_t M, int64_t K,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  if (!problems || count < 1 || count > QL_GEMM_MAX_GROUP) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  int64_t Ns[QL_GEMM_MAX_GROUP];
+  for (int j = 0; j < count; ++j) {
+    QL_TRY(check_n(scheme, problems[j].N, K));
+    QL_TRY(check_m(M, problems[j].N, K));
+    Ns[j] = problems[j].N;
+  }
+  if (M == 0) return QL_OK;
+  QL_TRY(need(qx));
+  QL_TRY(need(sx));
+  for (int j = 0; j < count; ++j) {
+    QL_TRY(need(problems[j].wq));
+    QL_TRY(need(problems[j].sw));
+    QL_TRY(need(problems[j].y));
+  }
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  const size_t need_ws = ql::gemm_group_workspace_bytes(scheme, M, Ns, count, K, d.sms);
+  const bool use_ws = need_ws && workspace && ws_bytes >= need_ws;
+  if (use_ws && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return QL_ERR_MISALIGNED;
+  cudaError_t e = ql::launch_gemm_group(scheme, qx, sx, problems, count, M, K, use_ws ? workspace : nullptr,
+                                        use_ws ? ws_bytes : 0, nullptr, d.sms, d.status,
+                                        static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm_grouped");
+}
+
+size_t qlinear_gemm_grouped_workspace_bytes(ql_scheme scheme, const int64_t* Ns, int count, int64_t M,
+                                            int64_t K) {
+  DeviceInfo d;
+  if (!valid_scheme(scheme) || !Ns || count < 1 || count > QL_GEMM_MAX_GROUP || M <= 0 || K <= 0 ||
+      current_device(&d) != QL_OK)
+    return 0;
+  for (int j = 0; j < count; ++j)
+    if (Ns[j] <= 0) return 0;
+  return ql::gemm_group_workspace_bytes(scheme, M, Ns, count, K, d.sms);
+}
+
 size_t qlinear_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K) {
   DeviceInfo d;
   if (!valid_scheme(scheme) || M <= 0 || N <= 0 || K <= 0 || current_device(&d) != QL_OK) return 0;

@@ -24,6 +24,9 @@
 // the preceding kernel), q_x, s_x and y only after it.
 // Every mbarrier wait is bounded; on a timeout the kernel records it, drains
 // its own copies and MMAs, frees TMEM and returns.
+#include <climits>
+#include <cstring>
+
 #include "ql_tc.cuh"
 #include "ql_internal.h"
 
@@ -51,22 +54,57 @@ constexpr int kTmemCols = 512;
 constexpr int kGemmSmemBudget = 200 * 1024;
 constexpr int kGemmEarlyStages = 2;  // W tiles requested before the grid dependency wait
 
+// A launch runs 1 to kGemmMaxGroup products that read the same q_x (e.g. a
+// layer's q, k and v projections): product j owns tiles [t0[j], t0[j+1]).
+constexpr int kGemmMaxGroup = QL_GEMM_MAX_GROUP;
+
 struct GemmParams {
   const float* sx;
-  const float* sw;
-  uint16_t* y;
-  int M, N, K;
-  int mt, nt, nkb;  // tiles along M and N, K blocks of 128
+  const float* sw[kGemmMaxGroup];
+  uint16_t* y[kGemmMaxGroup];
+  int N[kGemmMaxGroup];
+  int t0[kGemmMaxGroup + 1];  // first tile of each product; INT_MAX past the last
+  int nprob;
+  int M, K;
+  int mt, ntiles, nkb;  // tiles along M, tiles in all, K blocks of 128
   int split;        // block scheme: K halves per tile (1 = whole tiles, or 2)
   float* parts;     // split = 2: f32 partial sums, [half][tile][warp][column / 4][lane][4]
   uint32_t* counters;  // split = 2: [mt * nt] arrivals per tile, zero between calls
   int32_t* acc_i32;
   float* acc_f32;
-  uint8_t* qy;      // block scheme: E4M3 codes of y [M,N] for the next product, or null
+  uint8_t* qy;      // block scheme, one product: E4M3 codes of y [M,N] for the next product, or null
   float* sy;        // and their scales [M, N/128]
   DevStatus* status;
 };
 
+// The W_q tensor maps of the products (kernel parameters: read by TMA from
+// the parameter space).
+struct GemmMapsB {
+  CUtensorMap m[kGemmMaxGroup];
+};
+
+// The product of tile t and t's index inside it, by constant-index selects
+// (a dynamic index would copy the parameter arrays to local memory).
+struct ProdView {
+  const float* sw;
+  uint16_t* y;
+  int N, tl, j;
+};
+QL_DEVINL ProdView prod_of(const GemmParams& p, int t) {
+  const int j = (t >= p.t0[1]) + (t >= p.t0[2]) + (t >= p.t0[3]);
+  ProdView v;
+  v.j = j;
+  v.sw = j == 0 ? p.sw[0] : j == 1 ? p.sw[1] : j == 2 ? p.sw[2] : p.sw[3];
+  v.y = j == 0 ? p.y[0] : j == 1 ? p.y[1] : j == 2 ? p.y[2] : p.y[3];
+  v.N = j == 0 ? p.N[0] : j == 1 ? p.N[1] : j == 2 ? p.N[2] : p.N[3];
+  v.tl = t - (j == 0 ? 0 : j == 1 ? p.t0[1] : j == 2 ? p.t0[2] : p.t0[3]);
+  return v;
+}
+QL_DEVINL const CUtensorMap* map_of(const GemmMapsB& b, int j) {
+  return j == 0 ? &b.m[0] : j == 1 ? &b.m[1] : j == 2 ? &b.m[2] : &b.m[3];
+}
+
+static_assert(kGemmMaxGroup == 4, "prod_of and map_of select among four products");
 constexpr uint32_t kGemmEpiBar = 1;  // named barrier of the epilogue warps
 
 // OR vote over the epilogue warps that doubles as their barrier.
@@ -159,7 +197,7 @@ QL_DEVINL void store_box32(uint8_t* box, int lane, const uint32_t (&w)[16], uint
 // kQ (block scheme only): the epilogue also writes y's E4M3 codes and scales.
 template <ql_scheme S, int BN, bool kQ = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ GemmMapsB tmB,
                 const GemmParams p) {
   constexpr bool kInt8 = S == QL_W8A8_INT8_ROW;
   constexpr bool kBlock = S == QL_FP8_E4M3_BLOCK128;
@@ -182,7 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* last_flag = abort_flag + 1;  // split tiles: this CTA adds the last part
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntiles = p.mt * p.nt;
+  const int ntiles = p.ntiles;
   // this CTA's work items b, b + G, ... as (tile, K blocks [lo, hi)): item i
   // is K range i % split of tile i / split; fn returns false to stop
   const int nitems = ntiles * p.split;
@@ -207,7 +245,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
     tc::prefetch_tmap(&tmA);
-    tc::prefetch_tmap(&tmB);
+    for (int j = 0; j < p.nprob; ++j) tc::prefetch_tmap(map_of(tmB, j));
   }
   if (warp == 1) {
     tc::tmem_alloc(tmem_holder, kTmemCols);
@@ -231,10 +269,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // kernel's own loads behind this kernel's weight reads.
       uint32_t pre = 0;
       for_each_item([&](int t, int lo, int hi) -> bool {
-        const int n0 = (t / p.mt) * BN;
+        const ProdView pv = prod_of(p, t);
+        const int n0 = (pv.tl / p.mt) * BN;
+        const CUtensorMap* mb = map_of(tmB, pv.j);
         for (int kb = lo; kb < hi && pre < (uint32_t)kGemmEarlyStages; ++kb, ++pre) {
           mbar_arrive_expect_tx(&full[pre], Cfg::kStage);
-          tc::tma_load_2d(ring + pre * Cfg::kStage + Cfg::kStageA, &tmB, kb * kGemmBK, n0, &full[pre], pol_b);
+          tc::tma_load_2d(ring + pre * Cfg::kStage + Cfg::kStageA, mb, kb * kGemmBK, n0, &full[pre], pol_b);
         }
         return pre < (uint32_t)kGemmEarlyStages;
       });
@@ -242,7 +282,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for_each_item([&](int t, int lo, int hi) -> bool {
-        const int m0 = (t % p.mt) * kGemmBM, n0 = (t / p.mt) * BN;
+        const ProdView pv = prod_of(p, t);
+        const int m0 = (pv.tl % p.mt) * kGemmBM, n0 = (pv.tl / p.mt) * BN;
+        const CUtensorMap* mb = map_of(tmB, pv.j);
         for (int kb = lo; kb < hi; ++kb, ++it) {
           const int s = it % kStages;
           if (it < pre) {  // its W tile is on the way: the q_x tile completes the stage
@@ -257,7 +299,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* st = ring + s * Cfg::kStage;
           mbar_arrive_expect_tx(&full[s], Cfg::kStage);
           tc::tma_load_2d(st, &tmA, kb * kGemmBK, m0, &full[s], pol_a);
-          tc::tma_load_2d(st + Cfg::kStageA, &tmB, kb * kGemmBK, n0, &full[s], pol_b);
+          tc::tma_load_2d(st + Cfg::kStageA, mb, kb * kGemmBK, n0, &full[s], pol_b);
         }
         return true;
       });
@@ -340,7 +382,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t jt = 0;
     bool ok = true;
     for_each_item([&](int t, int lo, int hi) -> bool {
-      const int m0 = (t % p.mt) * kGemmBM, n0 = (t / p.mt) * BN;
+      const ProdView pv = prod_of(p, t);
+      const int N = pv.N;
+      uint16_t* const Y = pv.y;
+      const float* const SW = pv.sw;
+      const int m0 = (pv.tl % p.mt) * kGemmBM, n0 = (pv.tl / p.mt) * BN;
       const int m = m0 + q * 32 + lane;
       const bool live_m = m < p.M;
       const int c0 = h * Cfg::kHalf;  // first column of this warp inside the tile
@@ -354,7 +400,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
           const int n = n0 + c0 + c * 32 + lane;
-          swl[c] = c * 32 + lane < Cfg::kHalf && n < p.N ? __ldg(p.sw + n) : 0.0f;
+          swl[c] = c * 32 + lane < Cfg::kHalf && n < N ? __ldg(SW + n) : 0.0f;
         }
         const uint32_t buf = jt % kBufs;
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kBufs) & 1, abort_flag));
@@ -376,26 +422,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const float a = kInt8 ? __int2float_rn((int)r[j]) : __uint_as_float(r[j]);
             v[j] = __fmul_rn(__fmul_rn(a, sxm), __shfl_sync(0xffffffffu, swc, j));
           }
-          if (live_m && n < p.N) {
+          if (live_m && n < N) {
             if (p.acc_i32 || p.acc_f32) {
 #pragma unroll
               for (int j = 0; j < W; ++j) {
-                if (n + j < p.N) {
-                  if (kInt8 && p.acc_i32) p.acc_i32[(int64_t)m * p.N + n + j] = (int)r[j];
-                  if (!kInt8 && p.acc_f32) p.acc_f32[(int64_t)m * p.N + n + j] = __uint_as_float(r[j]);
+                if (n + j < N) {
+                  if (kInt8 && p.acc_i32) p.acc_i32[(int64_t)m * N + n + j] = (int)r[j];
+                  if (!kInt8 && p.acc_f32) p.acc_f32[(int64_t)m * N + n + j] = __uint_as_float(r[j]);
                 }
               }
             }
           }
           // whole 32-column chunks inside N leave through the box (uniform per warp)
-          if (W == 32 && n + 32 <= p.N && (p.N & 7) == 0) {
+          if (W == 32 && n + 32 <= N && (N & 7) == 0) {
             uint32_t w[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j)
               w[j] = (uint32_t)f32_to_bf16_rn(v[2 * j]) | ((uint32_t)f32_to_bf16_rn(v[2 * j + 1]) << 16);
-            store_box32(staging + ew * Cfg::kBox, lane, w, p.y, m0 + q * 32, n, p.M, p.N);
-          } else if (live_m && n < p.N) {
-            store_row<W>(p.y, m, n, p.N, v);
+            store_box32(staging + ew * Cfg::kBox, lane, w, Y, m0 + q * 32, n, p.M, N);
+          } else if (live_m && n < N) {
+            store_row<W>(Y, m, n, N, v);
           }
         };
 #pragma unroll
@@ -410,7 +456,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // block scheme: promote each 128-deep partial into f32 registers
         static_assert(BN == 128 || BN == 256, "block tiles are 128 or 256 wide");
         const int ncol = n0 + c0;
-        const bool live_n = ncol < p.N;
+        const bool live_n = ncol < N;
         const int nbw = ncol >> 7;  // this warp's columns lie in one 128-row weight block
         // running sums as pairs: one packed f32x2 FMA (two IEEE fmas) per pair
         float2 acc[Cfg::kHalf / 2];
@@ -419,12 +465,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // scales of K block kb+1 are loaded while the MMAs of block kb run
         const bool live = live_m && live_n;
         float sx_next = live ? __ldg(p.sx + (int64_t)m * KB + lo) : 0.0f;
-        float sw_next = live ? __ldg(p.sw + (int64_t)nbw * KB + lo) : 0.0f;
+        float sw_next = live ? __ldg(SW + (int64_t)nbw * KB + lo) : 0.0f;
         for (int kb = lo; kb < hi; ++kb) {
           const float scale = sx_next * sw_next;
           if (live && kb + 1 < hi) {
             sx_next = __ldg(p.sx + (int64_t)m * KB + kb + 1);
-            sw_next = __ldg(p.sw + (int64_t)nbw * KB + kb + 1);
+            sw_next = __ldg(SW + (int64_t)nbw * KB + kb + 1);
           }
           const uint32_t buf = jt % kBufs;
           ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kBufs) & 1, abort_flag));
@@ -573,26 +619,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           auto pack = [&](int j) {
             return (uint32_t)f32_to_bf16_rn(acc[j].x) | ((uint32_t)f32_to_bf16_rn(acc[j].y) << 16);
           };
-          if (p.y && live_n && mrow < p.M) {
+          if (Y && live_n && mrow < p.M) {
 #pragma unroll
             for (int c = 0; c < Cfg::kHalf / 32; ++c) {
               uint32_t w[16];
 #pragma unroll
               for (int j = 0; j < 16; ++j) w[j] = pack(c * 16 + j);
-              store_box32(staging + ew * Cfg::kBox, lane, w, p.y, mrow, ncol + c * 32, p.M, p.N);
+              store_box32(staging + ew * Cfg::kBox, lane, w, Y, mrow, ncol + c * 32, p.M, N);
             }
           }
           const float sc = a / 448.0f;
           const Divisor dv = make_divisor(sc);
           if (live_n && live_m) {
-            uint8_t* qrow = p.qy + (int64_t)m * p.N + ncol;
+            uint8_t* qrow = p.qy + (int64_t)m * N + ncol;
 #pragma unroll
             for (int c = 0; c < Cfg::kHalf / 16; ++c) {
               const uint2 q0 = quant_chunk8<false>(make_uint4(pack(8 * c), pack(8 * c + 1), pack(8 * c + 2), pack(8 * c + 3)), dv);
               const uint2 q1 = quant_chunk8<false>(make_uint4(pack(8 * c + 4), pack(8 * c + 5), pack(8 * c + 6), pack(8 * c + 7)), dv);
               *reinterpret_cast<uint4*>(qrow + c * 16) = make_uint4(q0.x, q0.y, q1.x, q1.y);
             }
-            if ((ncol & 127) == 0) p.sy[(int64_t)m * (p.N / 128) + (ncol >> 7)] = sc;
+            if ((ncol & 127) == 0) p.sy[(int64_t)m * (N / 128) + (ncol >> 7)] = sc;
           }
         } else if (live_n && mrow < p.M) {
 #pragma unroll
@@ -601,7 +647,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j)
               w[j] = (uint32_t)f32_to_bf16_rn(acc[c * 16 + j].x) | ((uint32_t)f32_to_bf16_rn(acc[c * 16 + j].y) << 16);
-            store_box32(staging + ew * Cfg::kBox, lane, w, p.y, mrow, ncol + c * 32, p.M, p.N);
+            store_box32(staging + ew * Cfg::kBox, lane, w, Y, mrow, ncol + c * 32, p.M, N);
           }
         }
       }
@@ -623,20 +669,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ---------------------------------------------------------------- host side
 
-// Tile width for this shape: fill the SMs' waves best, 128-wide tiles taxed
-// for their lower MMA rate.
-static int pick_bn(ql_scheme s, int64_t M, int64_t N, int sms) {
+// Tile width for a launch: fill the SMs' waves best (the products of a group
+// share the width; their tiles add up).
+static int64_t group_tiles(int64_t mt, const int64_t* Ns, int count, int bn) {
+  int64_t t = 0;
+  for (int j = 0; j < count; ++j) t += mt * ((Ns[j] + bn - 1) / bn);
+  return t;
+}
+
+static int pick_bn(ql_scheme s, int64_t M, const int64_t* Ns, int count, int sms) {
   const int cands_row[5] = {256, 224, 192, 160, 128};
   const int cands_blk[2] = {256, 128};
   const int* c = s == QL_FP8_E4M3_BLOCK128 ? cands_blk : cands_row;
   const int nc = s == QL_FP8_E4M3_BLOCK128 ? 2 : 5;
   const int64_t mt = (M + kGemmBM - 1) / kGemmBM;
+  int64_t ncols = 0;
+  for (int j = 0; j < count; ++j) ncols += Ns[j];
   int best = c[0];
   double best_eff = -1.0;
   for (int i = 0; i < nc; ++i) {
-    const int64_t tiles = mt * ((N + c[i] - 1) / c[i]);
+    const int64_t tiles = group_tiles(mt, Ns, count, c[i]);
     const int64_t waves = (tiles + sms - 1) / sms;
-    double eff = (double)(mt * N) / (double)(waves * sms * (int64_t)kGemmBM * c[i] / kGemmBM);
+    double eff = (double)(mt * ncols) / (double)(waves * sms * (int64_t)c[i]);
     // measured: 128-wide tiles run the MMAs at ~85% of the wider tiles' rate
     // (row schemes) and ~60% for the block scheme, whose per-K-block
     // promotion costs the same per tile at either width
@@ -662,17 +716,17 @@ struct GemmPlan {
   int bn, split;
 };
 
-static GemmPlan plan_gemm(ql_scheme s, int64_t M, int64_t N, int64_t K, int sms) {
-  GemmPlan pl{pick_bn(s, M, N, sms), 1};
+static GemmPlan plan_gemm(ql_scheme s, int64_t M, const int64_t* Ns, int count, int64_t K, int sms) {
+  GemmPlan pl{pick_bn(s, M, Ns, count, sms), 1};
   if (s != QL_FP8_E4M3_BLOCK128) return pl;
   const int64_t mt = (M + kGemmBM - 1) / kGemmBM;
-  const int64_t tiles = mt * ((N + 255) / 256);
+  const int64_t tiles = group_tiles(mt, Ns, count, 256);
   const int64_t nkb = (K + kGemmBK - 1) / kGemmBK;
   if (2 * tiles <= sms && nkb >= 64) return GemmPlan{256, 2};
   // Tiles of the chosen width that fill at most a quarter of the SMs (small
   // N, e.g. k/v at M = 512: 32 tiles of 128): split each tile's K blocks over
   // 2, 4 or 8 CTAs, as many as fit one wave, keeping >= 8 K blocks a part.
-  const int64_t t_bn = mt * ((N + pl.bn - 1) / pl.bn);
+  const int64_t t_bn = group_tiles(mt, Ns, count, pl.bn);
   int split = 1;
   while (pl.bn == 128 && split < 8 && 4 * t_bn * split <= 2 * sms && t_bn * split * 2 <= sms &&
          nkb / (split * 2) >= 8)
@@ -688,20 +742,24 @@ static size_t split_parts_bytes(int64_t tiles, int split) {
   return (size_t)split * tiles * kGemmBM * 256 * 4;
 }
 
-size_t gemm_workspace_bytes(ql_scheme s, int64_t M, int64_t N, int64_t K, int sms) {
-  const GemmPlan pl = plan_gemm(s, M, N, K, sms);
+size_t gemm_group_workspace_bytes(ql_scheme s, int64_t M, const int64_t* Ns, int count, int64_t K, int sms) {
+  const GemmPlan pl = plan_gemm(s, M, Ns, count, K, sms);
   if (pl.split == 1) return 0;
-  const int64_t tiles = ((M + kGemmBM - 1) / kGemmBM) * ((N + pl.bn - 1) / pl.bn);
+  const int64_t tiles = group_tiles((M + kGemmBM - 1) / kGemmBM, Ns, count, pl.bn);
   return align256(split_parts_bytes(tiles, pl.split)) + align256((size_t)tiles * 4);
 }
 
+size_t gemm_workspace_bytes(ql_scheme s, int64_t M, int64_t N, int64_t K, int sms) {
+  return gemm_group_workspace_bytes(s, M, &N, 1, K, sms);
+}
+
 template <ql_scheme S, int BN, bool kQ = false>
-static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
+static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, const GemmMapsB& b,
                                  int sms, cudaStream_t st) {
   using Cfg = GemmCfg<BN, S == QL_FP8_E4M3_BLOCK128>;
   cudaError_t e = ensure_smem<gemm_kernel<S, BN, kQ>>(Cfg::kSmem);
   if (e != cudaSuccess) return e;
-  const int grid = (int)std::min<int64_t>((int64_t)p.mt * p.nt * p.split, sms);
+  const int grid = (int)std::min<int64_t>((int64_t)p.ntiles * p.split, sms);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemmThreads);
@@ -715,41 +773,63 @@ static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, cons
   return cudaLaunchKernelEx(&cfg, gemm_kernel<S, BN, kQ>, a, b, p);
 }
 
-cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
-                        const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
-                        size_t ws_bytes, const ql_debug* dbg, int num_sms, DevStatus* status,
-                        cudaStream_t st, uint8_t* qy, float* sy) {
-  if ((qy != nullptr) != (sy != nullptr) || (qy && scheme != QL_FP8_E4M3_BLOCK128))
+cudaError_t launch_gemm_group(ql_scheme scheme, const void* qx, const float* sx, const ql_gemm_problem* probs,
+                              int count, int64_t M, int64_t K, void* workspace, size_t ws_bytes,
+                              const ql_debug* dbg, int num_sms, DevStatus* status, cudaStream_t st, uint8_t* qy,
+                              float* sy) {
+  if (count < 1 || count > kGemmMaxGroup) return cudaErrorInvalidValue;
+  if ((qy != nullptr) != (sy != nullptr) || (qy && (scheme != QL_FP8_E4M3_BLOCK128 || count != 1)))
     return cudaErrorInvalidValue;
+  if (dbg && count != 1) return cudaErrorInvalidValue;
+  int64_t Ns[kGemmMaxGroup];
+  for (int j = 0; j < count; ++j) Ns[j] = probs[j].N;
   // the K split needs its workspace; without one, whole tiles
-  GemmPlan pl = plan_gemm(scheme, M, N, K, num_sms);
-  const size_t need = gemm_workspace_bytes(scheme, M, N, K, num_sms);
-  if (pl.split > 1 && (workspace == nullptr || ws_bytes < need)) pl = GemmPlan{pick_bn(scheme, M, N, num_sms), 1};
+  GemmPlan pl = plan_gemm(scheme, M, Ns, count, K, num_sms);
+  const size_t need = gemm_group_workspace_bytes(scheme, M, Ns, count, K, num_sms);
+  if (pl.split > 1 && (workspace == nullptr || ws_bytes < need))
+    pl = GemmPlan{pick_bn(scheme, M, Ns, count, num_sms), 1};
   const int BN = pl.bn;
   GemmParams p;
   p.sx = sx;
-  p.sw = sw;
-  p.y = y;
+  p.nprob = count;
   p.M = (int)M;
-  p.N = (int)N;
   p.K = (int)K;
   p.mt = (int)((M + kGemmBM - 1) / kGemmBM);
-  p.nt = (int)((N + BN - 1) / BN);
   p.nkb = (int)((K + kGemmBK - 1) / kGemmBK);
+  GemmMapsB tb;
+  memset(&tb, 0, sizeof(tb));
+  int t = 0;
+  for (int j = 0; j < kGemmMaxGroup; ++j) {
+    if (j < count) {
+      p.sw[j] = probs[j].sw;
+      p.y[j] = probs[j].y;
+      p.N[j] = (int)probs[j].N;
+      p.t0[j] = t;
+      t += p.mt * (int)((probs[j].N + BN - 1) / BN);
+      cudaError_t e = make_tmap_u8_sw128(&tb.m[j], probs[j].wq, (uint64_t)K, (uint64_t)probs[j].N, (uint64_t)K,
+                                         kGemmBK, (uint32_t)BN);
+      if (e != cudaSuccess) return e;
+    } else {
+      p.sw[j] = nullptr;
+      p.y[j] = nullptr;
+      p.N[j] = 0;
+      p.t0[j] = INT_MAX;
+    }
+  }
+  p.t0[kGemmMaxGroup] = INT_MAX;
+  p.ntiles = t;
   p.split = pl.split;
   p.parts = pl.split > 1 ? static_cast<float*>(workspace) : nullptr;
   p.counters = pl.split > 1 ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) +
-                                                          align256(split_parts_bytes((int64_t)p.mt * p.nt, pl.split)))
+                                                          align256(split_parts_bytes((int64_t)p.ntiles, pl.split)))
                             : nullptr;
   p.acc_i32 = dbg ? dbg->acc_i32 : nullptr;
   p.acc_f32 = dbg ? dbg->acc_f32 : nullptr;
   p.qy = qy;
   p.sy = sy;
   p.status = status;
-  CUtensorMap ta, tb;
+  CUtensorMap ta;
   cudaError_t e = make_tmap_u8_sw128(&ta, qx, (uint64_t)K, (uint64_t)M, (uint64_t)K, kGemmBK, kGemmBM);
-  if (e != cudaSuccess) return e;
-  e = make_tmap_u8_sw128(&tb, wq, (uint64_t)K, (uint64_t)N, (uint64_t)K, kGemmBK, (uint32_t)BN);
   if (e != cudaSuccess) return e;
   switch (scheme) {
     case QL_W8A8_INT8_ROW:
@@ -772,6 +852,14 @@ cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const
       if (BN == 256) return launch_gemm_t<QL_FP8_E4M3_BLOCK128, 256>(p, ta, tb, num_sms, st);
       return launch_gemm_t<QL_FP8_E4M3_BLOCK128, 128>(p, ta, tb, num_sms, st);
   }
+}
+
+cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
+                        const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
+                        size_t ws_bytes, const ql_debug* dbg, int num_sms, DevStatus* status,
+                        cudaStream_t st, uint8_t* qy, float* sy) {
+  const ql_gemm_problem one{wq, sw, y, N};
+  return launch_gemm_group(scheme, qx, sx, &one, 1, M, K, workspace, ws_bytes, dbg, num_sms, status, st, qy, sy);
 }
 
 }  // namespace ql

@@ -72,6 +72,13 @@ cudaError_t launch_gemv_weight_only(ql_scheme scheme, const uint16_t* x, const v
 
 // Large-M tcgen05 GEMM on pre-quantized activations.
 size_t gemm_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);
+// a group of 1..QL_GEMM_MAX_GROUP products on one q_x (their N in Ns)
+size_t gemm_group_workspace_bytes(ql_scheme scheme, int64_t M, const int64_t* Ns, int count, int64_t K,
+                                  int num_sms);
+cudaError_t launch_gemm_group(ql_scheme scheme, const void* qx, const float* sx, const ql_gemm_problem* probs,
+                              int count, int64_t M, int64_t K, void* workspace, size_t ws_bytes,
+                              const ql_debug* dbg, int num_sms, DevStatus* status, cudaStream_t st,
+                              uint8_t* qy = nullptr, float* sy = nullptr);
 // qy / sy (block scheme only): also write y's E4M3 codes [M,N] and per-128
 // scales [M,N/128]; y may then be null.
 cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,

@@ -318,6 +318,42 @@ ql_status qlinear_gemm_quant_out(ql_scheme scheme, const void* qx, const float* 
                                  void* qy, float* sy, void* workspace, size_t ws_bytes,
                                  void* stream);
 
+/* Several large-M products on one pre-quantized input in one launch: each
+ * product keeps its own weights, scales and output, and the output tiles of
+ * all of them are dealt to the same persistent CTAs, so that products too
+ * small to fill the SMs alone (a layer's k and v projections at M = 512) fill
+ * them together with their neighbours, and a layer's q, k, v (or gate, up)
+ * cost one launch and one quantization of their shared input.  Pages: as for
+ * qlinear_gemm (the projections of one decoder layer that read one input).
+ * Numerics of each product as qlinear_gemm: int8 bit for bit; E4M3 bit for
+ * bit whenever neither call splits K (the block scheme's K split is planned
+ * on the group's tile count).
+ *   qx, sx     device, the shared input from qlinear_quantize_act
+ *   problems   host array of `count` descriptors, 1 <= count <=
+ *              QL_GEMM_MAX_GROUP (read during the call only):
+ *                wq  device, [N,K] codes;  sw  device, the matching scales
+ *                y   device, out: bf16 [M,N] (outputs must not overlap)
+ *                N   output rows (> 0; a multiple of 128 for the block scheme)
+ *   workspace  optional, as for qlinear_gemm, of at least
+ *              qlinear_gemm_grouped_workspace_bytes(...) bytes
+ * Errors: argument checks as for qlinear_gemm on every product; count outside
+ * [1, QL_GEMM_MAX_GROUP] -> QL_ERR_INVALID_ARG. */
+#define QL_GEMM_MAX_GROUP 4
+typedef struct ql_gemm_problem {
+  const void* wq;
+  const float* sw;
+  uint16_t* y;
+  int64_t N;
+} ql_gemm_problem;
+
+ql_status qlinear_gemm_grouped(ql_scheme scheme, const void* qx, const float* sx,
+                               const ql_gemm_problem* problems, int count, int64_t M, int64_t K,
+                               void* workspace, size_t ws_bytes, void* stream);
+/* Workspace size (bytes) for qlinear_gemm_grouped; Ns: host array of the
+ * `count` products' N.  0 means none is needed. */
+size_t qlinear_gemm_grouped_workspace_bytes(ql_scheme scheme, const int64_t* Ns, int count, int64_t M,
+                                            int64_t K);
+
 /* The projection as a model calls it: bf16 X in, bf16 Y out, dispatching on
  * the token count the way the pages' "Loading" sections describe: M = 1 ->
  * qlinear_gemv, 2..32 -> qlinear_gemm_small, > 32 -> qlinear_quantize_act

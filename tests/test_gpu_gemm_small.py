@@ -78,14 +78,17 @@ def test_config_w8a8_k_proj_m8_seed0(cuda):
                                    # up to four tokens ride on the GEMV kernel's B columns; past
                                    # its K limits they take the split-K kernel
                                    (2, 1000, 4096), (2, 129, 16384), (2, 64, 16400), (3, 1001, 4096),
-                                   (4, 777, 2064), (4, 300, 8192), (3, 64, 8208), (4, 130, 16)])
+                                   (4, 777, 2064), (4, 300, 8192), (3, 64, 8208), (4, 130, 16),
+                                   # five to eight tokens of a small product: two GEMV passes
+                                   (5, 1000, 4096), (7, 129, 8192), (8, 4096, 4096), (6, 64, 8208),
+                                   (8, 4100, 4096)])
 def test_small_shapes_full_compare(cuda, scheme, M, N, K):
     _run(scheme, M, N, K)
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 128), (2, 256, 384), (16, 384, 4096), (32, 1280, 1024),
                                    (7, 128, 12288), (2, 384, 4096), (3, 256, 1024), (4, 512, 8192),
-                                   (4, 128, 8320)])
+                                   (4, 128, 8320), (6, 1024, 4096), (8, 4096, 4096)])
 def test_small_block_shapes(cuda, M, N, K):
     _run(ql.FP8_E4M3_BLOCK128, M, N, K, outliers=2)
 
