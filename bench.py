@@ -185,8 +185,8 @@ def workloads():
     w["qwen-prefill-f2"] = Workload(
         "qwen-prefill-f2", "Qwen3-8B FP8 128x128-block projections at M=512 (7 shapes), each input "
         "arriving already quantized and each product also writing its own output's E4M3 codes and "
-        "per-128 scales for the product that reads it next: one kernel per projection (q|k|v and "
-        "gate|up read one input each)", "TOPS",
+        "per-128 scales for the product that reads it next: no quantization launch, q|k|v and gate|up "
+        "one grouped launch each on their shared input", "TOPS",
         [Product(n, FP8B, 512, N, K, 0, group=LAYER_INPUT.get(n, n), pre=True) for n, N, K in S.QWEN3_8B])
     w["qwen-prefill"] = Workload(
         "qwen-prefill", "Qwen3-8B FP8 128x128-block projections at M=512 (7 shapes), per-K-block "
@@ -383,19 +383,16 @@ class Runner:
                 item["qy"] = [(torch.empty((p.M, p.N), dtype=torch.uint8, device="cuda"),
                                torch.empty((p.M, p.N // 128), dtype=torch.float32, device="cuda"))
                               for _ in range(self.copies)]
-            if p.M > 32 and p.pre:  # quantized activations for the dominant-kernel timing
-                item["q"] = g["x_in"]
-                gws = ql.workspace_bytes(p.scheme, p.M, p.N, p.K)  # the K split's sums (block scheme)
-                item["ws_gemm"] = ql.new_workspace(gws) if gws else None
             g["items"].append(item)
         del weights
         for g in self.groups:
             p = g["p0"]
-            if gemm_grouped_route(p):
+            if gemm_grouped_route(p) and not p.pre:
                 # the step's quantized input (written by the step), a quantized copy of each
                 # input for the dominant-kernel timing, and the group's K-split workspace
                 g["qbuf"] = ql.quantize_act(p.scheme, g["xs"][0])
                 g["q"] = [ql.quantize_act(p.scheme, x) for x in g["xs"]]
+            if gemm_grouped_route(p):
                 gws = ql.gemm_grouped_workspace_bytes(p.scheme, [i["p"].N for i in g["items"]], p.M, p.K)
                 g["ws_gemm"] = ql.new_workspace(gws) if gws else None
         torch.cuda.synchronize()
@@ -415,7 +412,7 @@ class Runner:
         if self._grouped(g):
             return 1
         if gemm_grouped_route(g["p0"]):
-            return 2
+            return 1 if g["p0"].pre else 2
         return sum(1 if (i["p"].wo or i["p"].pre or gemv_route(i["p"].M, i["p"].K)) else 2
                    for i in g["items"])
 
@@ -436,21 +433,20 @@ class Runner:
         ys = ys or [i["ys"][t] for i in items]
         if self._grouped(g):
             self.ql.gemv_grouped(g["p0"].scheme, [(x, *self._w(i, t), y) for i, y in zip(items, ys)])
+        elif gemm_grouped_route(g["p0"]) and g["p0"].pre:
+            qx, sx = x  # arrives quantized; each output also leaves quantized for its reader
+            self.ql.gemm_grouped(g["p0"].scheme, qx, sx,
+                                 [(*self._w(i, t), y, *i["qy"][t]) for i, y in zip(items, ys)],
+                                 workspace=g["ws_gemm"])
         elif gemm_grouped_route(g["p0"]):
             qx, sx = g["qbuf"]
             self.ql.quantize_act(g["p0"].scheme, x, qx, sx)
             self.ql.gemm_grouped(g["p0"].scheme, qx, sx, [(*self._w(i, t), y) for i, y in zip(items, ys)],
                                  workspace=g["ws_gemm"])
-        elif g["p0"].pre:
+        elif g["p0"].pre:  # 2 <= M <= 32 on quantized input
             qx, sx = x
             for i, y in zip(items, ys):
-                p = i["p"]
-                wq, sw = self._w(i, t)
-                if p.M <= 32:
-                    self.ql.gemm_small_prequant(p.scheme, qx, sx, wq, sw, i["ws"], y=y)
-                else:
-                    qy, sy = i["qy"][t]
-                    self.ql.gemm_quant_out(p.scheme, qx, sx, wq, sw, workspace=i["ws_gemm"], y=y, qy=qy, sy=sy)
+                self.ql.gemm_small_prequant(i["p"].scheme, qx, sx, *self._w(i, t), i["ws"], y=y)
         else:
             for i, y in zip(items, ys):
                 self._forward(i, x, *self._w(i, t), y)
@@ -468,7 +464,7 @@ class Runner:
         ql = self.ql
         if self._grouped(g) or g["p0"].pre:  # one kernel per launch already
             self._run_group(g, g["x_in"][t], t)
-        elif gemm_grouped_route(g["p0"]):
+        elif gemm_grouped_route(g["p0"]) and not g["p0"].pre:
             qx, sx = g["q"][t]
             ql.gemm_grouped(g["p0"].scheme, qx, sx, [(*self._w(i, t), i["ys"][t]) for i in g["items"]],
                             workspace=g["ws_gemm"])
@@ -480,11 +476,8 @@ class Runner:
                     ql.gemv_weight_only(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
                 elif p.M == 1:
                     ql.gemv(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
-                elif p.M <= 32:
+                else:  # 2 <= M <= 32 (M > 32 runs grouped)
                     ql.gemm_small(p.scheme, i["xs"][t], wq, sw, i["ws"], y=i["ys"][t])
-                else:
-                    qx, sx = i["q"][t]
-                    ql.gemm(p.scheme, qx, sx, wq, sw, workspace=i["ws_gemm"], y=i["ys"][t])
 
     def capture(self, fn, stream):
         torch = self.torch
@@ -558,9 +551,10 @@ def whole_job_value(world: int, amount_per_step: float, steps: int, ms: float, s
 
 
 def gemm_grouped_route(p: Product) -> bool:
-    """True when a group of M > 32 products runs as one quantization of its
-    input and one qlinear_gemm_grouped launch (a group of one included)."""
-    return p.M > 32 and not p.pre and not p.wo
+    """True when a group of M > 32 products runs as one qlinear_gemm_grouped
+    launch (a group of one included), after one quantization of its input
+    unless the input arrives quantized."""
+    return p.M > 32 and not p.wo
 
 
 def dominant_launch_count(wl) -> int:

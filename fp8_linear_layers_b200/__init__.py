@@ -392,7 +392,8 @@ GEMM_MAX_GROUP = 4  # QL_GEMM_MAX_GROUP
 
 
 class _GemmProblem(ctypes.Structure):
-    _fields_ = [("wq", ctypes.c_void_p), ("sw", ctypes.c_void_p), ("y", ctypes.c_void_p), ("N", ctypes.c_int64)]
+    _fields_ = [("wq", ctypes.c_void_p), ("sw", ctypes.c_void_p), ("y", ctypes.c_void_p), ("qy", ctypes.c_void_p),
+                ("sy", ctypes.c_void_p), ("N", ctypes.c_int64)]
 
 
 def gemm_grouped_workspace_bytes(scheme: int, Ns, M: int, K: int) -> int:
@@ -404,20 +405,29 @@ def gemm_grouped_workspace_bytes(scheme: int, Ns, M: int, K: int) -> int:
 def gemm_grouped(scheme: int, qx: torch.Tensor, sx: torch.Tensor, problems, workspace: torch.Tensor | None = None,
                  stream=None) -> list:
     """Several large-M products on one quantized input in one launch.
-    `problems` is a list of (wq [N,K], sw, y or None); returns the outputs [M,N]."""
+    `problems` is a list of (wq [N,K], sw, y or None) or, block scheme, of
+    (wq, sw, y or None, qy [M,N] uint8, sy [M,N/128] f32) to also write each
+    output's codes and scales (y may then be False: codes only); returns the
+    outputs [M,N] (None where not written)."""
     if not 1 <= len(problems) <= GEMM_MAX_GROUP:
         raise ValueError(f"1 to {GEMM_MAX_GROUP} products per grouped launch")
     M, K = qx.shape
     table = (_GemmProblem * len(problems))()
     ys = []
-    for j, (wq, sw, y) in enumerate(problems):
+    for j, prob in enumerate(problems):
+        wq, sw, y = prob[:3]
+        qy, sy = prob[3:5] if len(prob) > 3 else (None, None)
         if wq.shape[1] != K:
             raise ValueError("every product of a grouped launch reads the same [M,K] input")
         N = wq.shape[0]
         if y is None:
             y = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device)
+        elif y is False:
+            y = None
         table[j] = _GemmProblem(_dev(wq, torch.uint8, "wq"), _dev(sw, torch.float32, "sw"),
-                                _dev(y, torch.bfloat16, "y"), N)
+                                _dev(y, torch.bfloat16, "y") if y is not None else None,
+                                _dev(qy, torch.uint8, "qy") if qy is not None else None,
+                                _dev(sy, torch.float32, "sy") if sy is not None else None, N)
         ys.append(y)
     wp, wn = _ws(workspace)
     _check(lib().qlinear_gemm_grouped(scheme, _dev(qx, torch.uint8, "qx"), _dev(sx, torch.float32, "sx"),

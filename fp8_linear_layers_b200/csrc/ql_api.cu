@@ -384,11 +384,19 @@ ql_status qlinear_gemm_grouped(ql_scheme scheme, const void* qx, const float* sx
   if (M == 0) return QL_OK;
   QL_TRY(need(qx));
   QL_TRY(need(sx));
+  const bool quant_out = problems[0].qy != nullptr;
   for (int j = 0; j < count; ++j) {
     QL_TRY(need(problems[j].wq));
     QL_TRY(need(problems[j].sw));
-    QL_TRY(need(problems[j].y));
+    if ((problems[j].qy != nullptr) != quant_out || (problems[j].sy != nullptr) != quant_out)
+      return QL_ERR_INVALID_ARG;
+    if (!quant_out || problems[j].y) QL_TRY(need(problems[j].y));
+    if (quant_out) {
+      QL_TRY(need(problems[j].qy));
+      QL_TRY(need(problems[j].sy));
+    }
   }
+  if (quant_out && scheme != QL_FP8_E4M3_BLOCK128) return QL_ERR_UNSUPPORTED_SHAPE;
   DeviceInfo d;
   QL_TRY(current_device(&d));
   const size_t need_ws = ql::gemm_group_workspace_bytes(scheme, M, Ns, count, K, d.sms);

@@ -72,8 +72,8 @@ struct GemmParams {
   uint32_t* counters;  // split = 2: [mt * nt] arrivals per tile, zero between calls
   int32_t* acc_i32;
   float* acc_f32;
-  uint8_t* qy;      // block scheme, one product: E4M3 codes of y [M,N] for the next product, or null
-  float* sy;        // and their scales [M, N/128]
+  uint8_t* qy[kGemmMaxGroup];  // block scheme: E4M3 codes of each y [M,N] for the product that reads it next
+  float* sy[kGemmMaxGroup];    // and their scales [M, N/128] (kQ launches)
   DevStatus* status;
 };
 
@@ -90,6 +90,12 @@ struct ProdView {
   uint16_t* y;
   int N, tl, j;
 };
+QL_DEVINL uint8_t* qy_of(const GemmParams& p, int j) {
+  return j == 0 ? p.qy[0] : j == 1 ? p.qy[1] : j == 2 ? p.qy[2] : p.qy[3];
+}
+QL_DEVINL float* sy_of(const GemmParams& p, int j) {
+  return j == 0 ? p.sy[0] : j == 1 ? p.sy[1] : j == 2 ? p.sy[2] : p.sy[3];
+}
 QL_DEVINL ProdView prod_of(const GemmParams& p, int t) {
   const int j = (t >= p.t0[1]) + (t >= p.t0[2]) + (t >= p.t0[3]);
   ProdView v;
@@ -402,19 +408,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int n = n0 + c0 + c * 32 + lane;
           swl[c] = c * 32 + lane < Cfg::kHalf && n < N ? __ldg(SW + n) : 0.0f;
         }
+        const bool whole = p.split == 1;
         const uint32_t buf = jt % kBufs;
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[buf], (jt / kBufs) & 1, abort_flag));
-        if (!ok) return false;
+        // a split tile meets the other epilogue warps at barriers below: all vote first
+        if (!whole) {
+          if (gemm_epi_any(!ok)) return false;
+        } else if (!ok) {
+          return false;
+        }
         tc::fence_after();
-        // W = 32 columns at a time; a 16-column tail for 160- and 224-wide tiles
-        auto chunk = [&](int col, float swc, auto wtag) {
+        // scales, debug copies and bf16 stores of W raw accumulators r (s32 or
+        // f32 bits) of this thread's row from column col on (W = 32, or a
+        // 16-column tail for 160- and 224-wide tiles)
+        auto finish = [&](int col, float swc, const uint32_t* r, auto wtag) {
           constexpr int W = decltype(wtag)::value;
-          uint32_t r[W];
-          if constexpr (W == 32)
-            tc::ld32(tmem + lane_base + buf * Cfg::kBufCols + col, r);
-          else
-            tc::ld16(tmem + lane_base + buf * Cfg::kBufCols + col, r);
-          tc::ld_wait();
           const int n = n0 + col;
           float v[W];
 #pragma unroll
@@ -444,6 +452,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             store_row<W>(Y, m, n, N, v);
           }
         };
+        // K split: this item's part of the tile's K blocks (lo = floor(part nkb / split)),
+        // parked raw in its slab laid out the way the warps hold it (lane-minor:
+        // each warp store writes 512 contiguous bytes)
+        const int part = whole ? 0 : (int)(((int64_t)lo * p.split + p.nkb - 1) / p.nkb);
+        auto slab = [&](int hf) {
+          return reinterpret_cast<uint4*>(p.parts) +
+                 ((int64_t)(hf * ntiles + t) * kGemmEpiWarps + ew) * (Cfg::kHalf / 4) * 32 + lane;
+        };
+        auto chunk = [&](int col, float swc, auto wtag) {
+          constexpr int W = decltype(wtag)::value;
+          uint32_t r[W];
+          if constexpr (W == 32)
+            tc::ld32(tmem + lane_base + buf * Cfg::kBufCols + col, r);
+          else
+            tc::ld16(tmem + lane_base + buf * Cfg::kBufCols + col, r);
+          tc::ld_wait();
+          if (whole) {
+            finish(col, swc, r, wtag);
+          } else {
+            uint4* mine = slab(part);
+#pragma unroll
+            for (int i = 0; i < W / 4; ++i)
+              __stcg(mine + ((col - c0) / 4 + i) * 32, make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]));
+          }
+        };
 #pragma unroll
         for (int c = 0; c < Cfg::kHalf / 32; ++c) chunk(c0 + c * 32, swl[c], std::integral_constant<int, 32>{});
         if constexpr (Cfg::kHalf % 32 != 0)
@@ -452,6 +485,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);
         ++jt;
+        if (!whole) {
+          __threadfence();
+          named_bar_sync(kGemmEpiBar, kGemmEpiWarps * 32);
+          if (ew == 0 && lane == 0) {
+            const unsigned old = atomicAdd(p.counters + t, 1u);
+            *last_flag = old == (unsigned)(p.split - 1);
+          }
+          named_bar_sync(kGemmEpiBar, kGemmEpiWarps * 32);
+          if (!*last_flag) return true;
+          __threadfence();
+          // the last part to arrive adds every part's raw sums in part order
+          // (s32 adds are exact; f32 adds in a fixed order give the same bits
+          // whichever part arrived last) and finishes the tile
+          auto merged = [&](int col, float swc, auto wtag) {
+            constexpr int W = decltype(wtag)::value;
+            const int v0 = (col - c0) / 4;
+            uint32_t r[W];
+            {
+              const uint4* b0 = slab(0);
+#pragma unroll
+              for (int i = 0; i < W / 4; ++i) {
+                const uint4 x = __ldcg(b0 + (v0 + i) * 32);
+                r[4 * i] = x.x, r[4 * i + 1] = x.y, r[4 * i + 2] = x.z, r[4 * i + 3] = x.w;
+              }
+            }
+            for (int hf = 1; hf < p.split; ++hf) {
+              const uint4* o = slab(hf);
+#pragma unroll
+              for (int i = 0; i < W / 4; ++i) {
+                const uint4 x = __ldcg(o + (v0 + i) * 32);
+                const uint32_t xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  r[4 * i + k] = kInt8 ? r[4 * i + k] + xv[k]
+                                       : __float_as_uint(__fadd_rn(__uint_as_float(r[4 * i + k]), __uint_as_float(xv[k])));
+              }
+            }
+            finish(col, swc, r, wtag);
+          };
+#pragma unroll
+          for (int c = 0; c < Cfg::kHalf / 32; ++c) merged(c0 + c * 32, swl[c], std::integral_constant<int, 32>{});
+          if constexpr (Cfg::kHalf % 32 != 0)
+            merged(c0 + Cfg::kHalf / 32 * 32, swl[kChunks - 1], std::integral_constant<int, 16>{});
+          if (ew == 0 && lane == 0) p.counters[t] = 0u;  // every part has arrived
+        }
       } else {
         // block scheme: promote each 128-deep partial into f32 registers
         static_assert(BN == 128 || BN == 256, "block tiles are 128 or 256 wide");
@@ -631,14 +709,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const float sc = a / 448.0f;
           const Divisor dv = make_divisor(sc);
           if (live_n && live_m) {
-            uint8_t* qrow = p.qy + (int64_t)m * N + ncol;
+            uint8_t* qrow = qy_of(p, pv.j) + (int64_t)m * N + ncol;
 #pragma unroll
             for (int c = 0; c < Cfg::kHalf / 16; ++c) {
               const uint2 q0 = quant_chunk8<false>(make_uint4(pack(8 * c), pack(8 * c + 1), pack(8 * c + 2), pack(8 * c + 3)), dv);
               const uint2 q1 = quant_chunk8<false>(make_uint4(pack(8 * c + 4), pack(8 * c + 5), pack(8 * c + 6), pack(8 * c + 7)), dv);
               *reinterpret_cast<uint4*>(qrow + c * 16) = make_uint4(q0.x, q0.y, q1.x, q1.y);
             }
-            if ((ncol & 127) == 0) p.sy[(int64_t)m * (N / 128) + (ncol >> 7)] = sc;
+            if ((ncol & 127) == 0) sy_of(p, pv.j)[(int64_t)m * (N / 128) + (ncol >> 7)] = sc;
           }
         } else if (live_n && mrow < p.M) {
 #pragma unroll
@@ -704,25 +782,27 @@ static int pick_bn(ql_scheme s, int64_t M, const int64_t* Ns, int count, int sms
   return best;
 }
 
-// Block scheme with at most half a wave of 256-wide tiles and a long K
-// (M = 512 with N = 4096, K >= 8192: down_proj): each tile's K blocks are
-// split in two halves run by two CTAs, which meet in an f32 workspace.
-// Measured per K block, 256-wide tiles promote at ~1.6x the 128-wide rate, so
-// a split 256-wide tile beats a whole 128-wide one once K is long enough to
-// repay parking and re-reading the f32 halves (Qwen3-8B down_proj at M = 512:
-// 47 -> 36 us; at K = 4096 the split measured 2% slower than whole 128-wide
-// tiles).  Otherwise (and for the row schemes) whole tiles.
+// At most half a wave of 256-wide tiles and a long K (M = 512 with N = 4096,
+// K >= 8192: down_proj): each tile's K blocks are split in two halves run by
+// two CTAs, which meet in the workspace (the block scheme's f32 running sums;
+// the row schemes' raw s32 or f32 accumulators, added before the scales).
+// Measured per K block, 256-wide tiles run at ~1.5x the 128-wide rate (block
+// scheme: promote at ~1.6x), so a split 256-wide tile beats a whole 128-wide
+// one once K is long enough to repay parking and re-reading the halves
+// (Qwen3-8B down_proj at M = 512: 47 -> 36 us; at K = 4096 the split
+// measured 2% slower than whole 128-wide tiles).  Otherwise whole tiles,
+// except the block scheme's small-N rule below.
 struct GemmPlan {
   int bn, split;
 };
 
 static GemmPlan plan_gemm(ql_scheme s, int64_t M, const int64_t* Ns, int count, int64_t K, int sms) {
   GemmPlan pl{pick_bn(s, M, Ns, count, sms), 1};
-  if (s != QL_FP8_E4M3_BLOCK128) return pl;
   const int64_t mt = (M + kGemmBM - 1) / kGemmBM;
   const int64_t tiles = group_tiles(mt, Ns, count, 256);
   const int64_t nkb = (K + kGemmBK - 1) / kGemmBK;
   if (2 * tiles <= sms && nkb >= 64) return GemmPlan{256, 2};
+  if (s != QL_FP8_E4M3_BLOCK128) return pl;
   // Tiles of the chosen width that fill at most a quarter of the SMs (small
   // N, e.g. k/v at M = 512: 32 tiles of 128): split each tile's K blocks over
   // 2, 4 or 8 CTAs, as many as fit one wave, keeping >= 8 K blocks a part.
@@ -775,11 +855,15 @@ static cudaError_t launch_gemm_t(const GemmParams& p, const CUtensorMap& a, cons
 
 cudaError_t launch_gemm_group(ql_scheme scheme, const void* qx, const float* sx, const ql_gemm_problem* probs,
                               int count, int64_t M, int64_t K, void* workspace, size_t ws_bytes,
-                              const ql_debug* dbg, int num_sms, DevStatus* status, cudaStream_t st, uint8_t* qy,
-                              float* sy) {
+                              const ql_debug* dbg, int num_sms, DevStatus* status, cudaStream_t st) {
   if (count < 1 || count > kGemmMaxGroup) return cudaErrorInvalidValue;
-  if ((qy != nullptr) != (sy != nullptr) || (qy && (scheme != QL_FP8_E4M3_BLOCK128 || count != 1)))
-    return cudaErrorInvalidValue;
+  // output quantization: every product of the launch or none, block scheme only
+  const bool quant_out = probs[0].qy != nullptr;
+  for (int j = 0; j < count; ++j) {
+    if ((probs[j].qy != nullptr) != quant_out || (probs[j].sy != nullptr) != quant_out) return cudaErrorInvalidValue;
+    if (!quant_out && probs[j].y == nullptr) return cudaErrorInvalidValue;
+  }
+  if (quant_out && scheme != QL_FP8_E4M3_BLOCK128) return cudaErrorInvalidValue;
   if (dbg && count != 1) return cudaErrorInvalidValue;
   int64_t Ns[kGemmMaxGroup];
   for (int j = 0; j < count; ++j) Ns[j] = probs[j].N;
@@ -803,6 +887,8 @@ cudaError_t launch_gemm_group(ql_scheme scheme, const void* qx, const float* sx,
     if (j < count) {
       p.sw[j] = probs[j].sw;
       p.y[j] = probs[j].y;
+      p.qy[j] = static_cast<uint8_t*>(probs[j].qy);
+      p.sy[j] = probs[j].sy;
       p.N[j] = (int)probs[j].N;
       p.t0[j] = t;
       t += p.mt * (int)((probs[j].N + BN - 1) / BN);
@@ -812,6 +898,8 @@ cudaError_t launch_gemm_group(ql_scheme scheme, const void* qx, const float* sx,
     } else {
       p.sw[j] = nullptr;
       p.y[j] = nullptr;
+      p.qy[j] = nullptr;
+      p.sy[j] = nullptr;
       p.N[j] = 0;
       p.t0[j] = INT_MAX;
     }
@@ -825,8 +913,6 @@ cudaError_t launch_gemm_group(ql_scheme scheme, const void* qx, const float* sx,
                             : nullptr;
   p.acc_i32 = dbg ? dbg->acc_i32 : nullptr;
   p.acc_f32 = dbg ? dbg->acc_f32 : nullptr;
-  p.qy = qy;
-  p.sy = sy;
   p.status = status;
   CUtensorMap ta;
   cudaError_t e = make_tmap_u8_sw128(&ta, qx, (uint64_t)K, (uint64_t)M, (uint64_t)K, kGemmBK, kGemmBM);
@@ -845,7 +931,7 @@ cudaError_t launch_gemm_group(ql_scheme scheme, const void* qx, const float* sx,
       if (BN == 160) return launch_gemm_t<QL_FP8_E4M3_ROW, 160>(p, ta, tb, num_sms, st);
       return launch_gemm_t<QL_FP8_E4M3_ROW, 128>(p, ta, tb, num_sms, st);
     default:
-      if (qy) {
+      if (quant_out) {
         if (BN == 256) return launch_gemm_t<QL_FP8_E4M3_BLOCK128, 256, true>(p, ta, tb, num_sms, st);
         return launch_gemm_t<QL_FP8_E4M3_BLOCK128, 128, true>(p, ta, tb, num_sms, st);
       }
@@ -858,8 +944,9 @@ cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const
                         const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace,
                         size_t ws_bytes, const ql_debug* dbg, int num_sms, DevStatus* status,
                         cudaStream_t st, uint8_t* qy, float* sy) {
-  const ql_gemm_problem one{wq, sw, y, N};
-  return launch_gemm_group(scheme, qx, sx, &one, 1, M, K, workspace, ws_bytes, dbg, num_sms, status, st, qy, sy);
+  if ((qy != nullptr) != (sy != nullptr)) return cudaErrorInvalidValue;
+  const ql_gemm_problem one{wq, sw, y, qy, sy, N};
+  return launch_gemm_group(scheme, qx, sx, &one, 1, M, K, workspace, ws_bytes, dbg, num_sms, status, st);
 }
 
 }  // namespace ql

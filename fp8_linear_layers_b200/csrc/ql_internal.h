@@ -77,8 +77,7 @@ size_t gemm_group_workspace_bytes(ql_scheme scheme, int64_t M, const int64_t* Ns
                                   int num_sms);
 cudaError_t launch_gemm_group(ql_scheme scheme, const void* qx, const float* sx, const ql_gemm_problem* probs,
                               int count, int64_t M, int64_t K, void* workspace, size_t ws_bytes,
-                              const ql_debug* dbg, int num_sms, DevStatus* status, cudaStream_t st,
-                              uint8_t* qy = nullptr, float* sy = nullptr);
+                              const ql_debug* dbg, int num_sms, DevStatus* status, cudaStream_t st);
 // qy / sy (block scheme only): also write y's E4M3 codes [M,N] and per-128
 // scales [M,N/128]; y may then be null.
 cudaError_t launch_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,

@@ -333,16 +333,24 @@ ql_status qlinear_gemm_quant_out(ql_scheme scheme, const void* qx, const float* 
  *              QL_GEMM_MAX_GROUP (read during the call only):
  *                wq  device, [N,K] codes;  sw  device, the matching scales
  *                y   device, out: bf16 [M,N] (outputs must not overlap)
+ *                qy, sy  NULL, or (block scheme, set for every product of
+ *                    the call) device outputs as for qlinear_gemm_quant_out:
+ *                    y's E4M3 codes [M,N] and per-128 scales [M,N/128]; y may
+ *                    then be NULL
  *                N   output rows (> 0; a multiple of 128 for the block scheme)
  *   workspace  optional, as for qlinear_gemm, of at least
  *              qlinear_gemm_grouped_workspace_bytes(...) bytes
  * Errors: argument checks as for qlinear_gemm on every product; count outside
- * [1, QL_GEMM_MAX_GROUP] -> QL_ERR_INVALID_ARG. */
+ * [1, QL_GEMM_MAX_GROUP], qy without sy (or the reverse), codes asked of some
+ * products but not all, or no output at all -> QL_ERR_INVALID_ARG; codes
+ * with a row scheme -> QL_ERR_UNSUPPORTED_SHAPE. */
 #define QL_GEMM_MAX_GROUP 4
 typedef struct ql_gemm_problem {
   const void* wq;
   const float* sw;
   uint16_t* y;
+  void* qy;
+  float* sy;
   int64_t N;
 } ql_gemm_problem;
 

@@ -93,7 +93,7 @@ def test_host_validation_rejects_before_launch(L):
     assert GR(0, tp, 2, 64, None) == MIS
     # the grouped GEMM: 1 to QL_GEMM_MAX_GROUP products on one quantized input
     G = ql._GemmProblem
-    gt = (G * 2)(G(ALIGNED, ALIGNED, ALIGNED, 256), G(ALIGNED, ALIGNED, ALIGNED, 256))
+    gt = (G * 2)(G(ALIGNED, ALIGNED, ALIGNED, 0, 0, 256), G(ALIGNED, ALIGNED, ALIGNED, 0, 0, 256))
     gp = ctypes.cast(gt, ctypes.c_void_p)
     GG = L.qlinear_gemm_grouped
     assert GG(0, ALIGNED, ALIGNED, gp, 0, 64, 256, None, 0, None) == INV
@@ -107,6 +107,13 @@ def test_host_validation_rejects_before_launch(L):
     gt[1].N, gt[1].y = 256, 0
     assert GG(0, ALIGNED, ALIGNED, gp, 2, 64, 256, None, 0, None) == INV
     assert GG(0, None, None, gp, 2, 0, 256, None, 0, None) == 0  # M = 0: nothing to do
+    gt[1].y = ALIGNED
+    gt[0].qy, gt[0].sy = ALIGNED, ALIGNED  # output codes asked of one product but not the other
+    assert GG(2, ALIGNED, ALIGNED, gp, 2, 64, 256, None, 0, None) == INV
+    gt[1].qy, gt[1].sy = ALIGNED, ALIGNED
+    assert GG(0, ALIGNED, ALIGNED, gp, 2, 64, 256, None, 0, None) == SHAPE  # codes: block scheme only
+    gt[1].sy = ALIGNED + 4
+    assert GG(2, ALIGNED, ALIGNED, gp, 2, 64, 256, None, 0, None) == MIS
     PQ = L.qlinear_gemv_prequant
     assert PQ(0, None, ALIGNED, ALIGNED, ALIGNED, 64, 64, ALIGNED, None) == INV
     assert PQ(0, ALIGNED, None, ALIGNED, ALIGNED, 64, 64, ALIGNED, None) == INV

@@ -153,6 +153,44 @@ def test_gemm_block_split_k(cuda, M, N, K):
     assert_y_close(bits(yf)[pm, pn], ry, f"forward block {M}x{N}x{K}")
 
 
+@pytest.mark.parametrize("scheme", [ql.W8A8_INT8_ROW, ql.FP8_E4M3_ROW])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 8192), (200, 384, 8192), (300, 1000, 8320)])
+def test_gemm_row_split_k(cuda, scheme, M, N, K):
+    """Row schemes with few 256-wide tiles and K >= 8192: with a workspace each
+    tile's K blocks are split in two halves that park their raw accumulators
+    (s32 / f32) and the second to arrive adds them before the scales.  Every
+    output against the oracle (int8: accumulators and outputs bit-exact, and
+    equal to whole tiles without a workspace); two calls agree bit for bit and
+    leave the arrival counters zero."""
+    ws_n = ql.workspace_bytes(scheme, M, N, K)
+    assert ws_n > 256 * 1024
+    qx, sx, wq, sw = _inputs(scheme, M, N, K, outliers=3)
+    args = (u8_dev(qx), f32_dev(sx), u8_dev(wq), f32_dev(sw))
+    ws = ql.new_workspace(ws_n)
+    dbg = ql.Debug(acc_i32=torch.empty((M, N), dtype=torch.int32, device="cuda")
+                   if scheme == ql.W8A8_INT8_ROW else None,
+                   acc_f32=torch.empty((M, N), dtype=torch.float32, device="cuda")
+                   if scheme == ql.FP8_E4M3_ROW else None)
+    y1 = ql.gemm(scheme, *args, workspace=ws, debug=dbg)
+    y2 = torch.full((M, N), -7.0, dtype=torch.bfloat16, device="cuda")
+    ql.gemm(scheme, *args, workspace=ws, y=y2)
+    y0 = ql.gemm(scheme, *args)
+    st, detail = ql.device_status()
+    assert st == 0, f"device status {st} detail {detail:#x}"
+    assert torch.count_nonzero(ws[ws_n - 256:]) == 0, "the arrival counters must be left zero"
+    ry, racc_i, racc_d = oracle.linear(scheme, qx, sx, wq, sw, want_acc=True)
+    g1 = bits(y1)
+    assert np.array_equal(g1, bits(y2)), "two calls on one workspace differ"
+    if scheme == ql.W8A8_INT8_ROW:
+        assert np.array_equal(dbg.acc_i32.cpu().numpy(), racc_i), "int32 accumulators differ"
+        assert np.array_equal(g1, ry) and np.array_equal(bits(y0), ry)
+    else:
+        acc = dbg.acc_f32.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(acc - racc_d) <= 1e-5 * np.abs(racc_d).max() + 1e-6)
+        assert_y_close(g1, ry, f"gemm row split {M}x{N}x{K}")
+        assert_y_close(bits(y0), ry, f"gemm row whole tiles {M}x{N}x{K}")
+
+
 def test_forward_dispatches_large_m_through_quant_and_gemm(cuda):
     """qlinear_forward with M > 32: fused per-token quantization into the
     workspace, then the GEMM; compared with the oracle's whole method."""

@@ -154,6 +154,41 @@ def test_grouped_block_k_split(cuda):
         assert_y_close(got0[j], ry, f"grouped whole-tile product {j}")
 
 
+@pytest.mark.parametrize("M", [512, 300])
+def test_grouped_quant_out(cuda, M):
+    """Block scheme, q|k|v in one launch that also writes each output's E4M3
+    codes and per-128 scales for the product that reads it next: y equals the
+    grouped launch's y without them, bit for bit, and the codes and scales
+    equal the oracle's quantization of that bf16 y, bit for bit; a codes-only
+    call (no y) writes the same codes."""
+    scheme = ql.FP8_E4M3_BLOCK128
+    names = ("q_proj", "k_proj", "v_proj")
+    K = QWEN["q_proj"][1]
+    Ns = [QWEN[n][0] for n in names]
+    qx, sx, ws = _operands(scheme, M, Ns, K, seed=15)
+    dqx, dsx = u8_dev(qx), f32_dev(sx)
+    dws = [(u8_dev(wq), f32_dev(sw)) for wq, sw in ws]
+    n_ws = ql.gemm_grouped_workspace_bytes(scheme, Ns, M, K)
+    wsp = ql.new_workspace(n_ws) if n_ws else None
+    y_ref = ql.gemm_grouped(scheme, dqx, dsx, [(wq, sw, None) for wq, sw in dws], workspace=wsp)
+    q = [(torch.empty((M, N), dtype=torch.uint8, device="cuda"),
+          torch.empty((M, N // 128), dtype=torch.float32, device="cuda")) for N in Ns]
+    ys = ql.gemm_grouped(scheme, dqx, dsx, [(wq, sw, None, *q[j]) for j, (wq, sw) in enumerate(dws)],
+                         workspace=wsp)
+    q2 = [(torch.empty_like(a), torch.empty_like(b)) for a, b in q]
+    ql.gemm_grouped(scheme, dqx, dsx, [(wq, sw, False, *q2[j]) for j, (wq, sw) in enumerate(dws)], workspace=wsp)
+    torch.cuda.synchronize()
+    assert ql.device_status()[0] == 0
+    for j, n in enumerate(names):
+        yb = bits(ys[j])
+        assert np.array_equal(yb, bits(y_ref[j])), f"{n}: y differs from the grouped launch without codes"
+        rq, rs = oracle.quantize_act(scheme, yb)
+        assert np.array_equal(q[j][1].cpu().numpy().view(np.uint32), rs.view(np.uint32)), f"{n}: output scales"
+        assert np.array_equal(q[j][0].cpu().numpy(), rq), f"{n}: output codes"
+        assert np.array_equal(q2[j][0].cpu().numpy(), rq) and torch.equal(q2[j][1], q[j][1])
+        _sampled(scheme, qx, sx, *ws[j], yb, f"grouped quant-out {n}", seed=j, nsamp=500)
+
+
 def test_grouped_argument_checks(cuda):
     M, K, N = 64, 256, 256
     qx = torch.zeros((M, K), dtype=torch.uint8, device="cuda")
@@ -162,7 +197,7 @@ def test_grouped_argument_checks(cuda):
     sw = torch.ones(N, dtype=torch.float32, device="cuda")
     y = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
     L = ql.lib()
-    table = (ql._GemmProblem * 5)(*[ql._GemmProblem(wq.data_ptr(), sw.data_ptr(), y.data_ptr(), N)] * 5)
+    table = (ql._GemmProblem * 5)(*[ql._GemmProblem(wq.data_ptr(), sw.data_ptr(), y.data_ptr(), 0, 0, N)] * 5)
     tp = ctypes.cast(table, ctypes.c_void_p)
     stream = torch.cuda.current_stream().cuda_stream
     args = (qx.data_ptr(), sx.data_ptr())
@@ -175,7 +210,17 @@ def test_grouped_argument_checks(cuda):
     table[1].N = 200
     assert L.qlinear_gemm_grouped(ql.FP8_E4M3_BLOCK128, *args, tp, 2, M, K, None, 0, stream) == 2  # N % 128
     assert L.qlinear_gemm_grouped(ql.W8A8_INT8_ROW, *args, tp, 2, M, 100, None, 0, stream) == 2  # K % 16
+    # output codes: all products or none, block scheme only
+    qy = torch.zeros((M, N), dtype=torch.uint8, device="cuda")
+    sy = torch.zeros((M, N // 128), dtype=torch.float32, device="cuda")
+    table[1].N = N
+    table[0].qy, table[0].sy = qy.data_ptr(), sy.data_ptr()
+    assert L.qlinear_gemm_grouped(ql.FP8_E4M3_BLOCK128, *args, tp, 2, M, K, None, 0, stream) == 1
+    table[1].qy = qy.data_ptr()
+    assert L.qlinear_gemm_grouped(ql.FP8_E4M3_BLOCK128, *args, tp, 2, M, K, None, 0, stream) == 1  # no sy
+    table[1].sy = sy.data_ptr()
+    assert L.qlinear_gemm_grouped(ql.W8A8_INT8_ROW, *args, tp, 2, M, K, None, 0, stream) == 2
     torch.cuda.synchronize()
-    assert torch.count_nonzero(y).item() == 0
+    assert torch.count_nonzero(y).item() == 0 and torch.count_nonzero(qy).item() == 0
     assert ql.gemm_grouped_workspace_bytes(ql.W8A8_INT8_ROW, [N, N], M, K) == 0
     assert ql.gemm_grouped_workspace_bytes(ql.FP8_E4M3_BLOCK128, [], M, K) == 0
