@@ -320,6 +320,8 @@ TRAFFIC = {
     # workload: (bytes per launch, kernel source hash, summary file)
     "decode": (54668224, "f67eb144cf9e747e", "profiles/gemv_decode_dram.md"),
     "decode-wo": (31224887, "233ea157dd920e9f", "profiles/gemv_decode_weight_only_dram.md"),
+    "prefill": (75563605, "f5f95d3f977ccd3f", "profiles/gemm_prefill_int8_dram.md"),
+    "qwen-prefill": (52263872, "f5f95d3f977ccd3f", "profiles/gemm_qwen_prefill_block_dram.md"),
 }
 
 
