@@ -154,9 +154,10 @@ def workloads():
          for n, N, K in S.LLAMA31_8B_PREFILL])
     w["small"] = Workload(
         "small", "small-batch tensor-core path: M in {2, 8, 16, 32} x the 7 Llama-3.1-8B shapes x "
-        "{W8A8 int8, FP8 E4M3 per-row}, quantization fused", "GB/s",
-        [Product(n, s, M, N, K, oc(K)) for M in (2, 8, 16, 32) for s in (INT8, FP8R)
-         for n, N, K in S.LLAMA31_8B])
+        "{W8A8 int8, FP8 E4M3 per-row}, quantization fused; q|k|v and gate|up one grouped launch each "
+        "on their shared tokens", "GB/s",
+        [Product(n, s, M, N, K, oc(K), group=LAYER_INPUT.get(n, n)) for M in (2, 8, 16, 32)
+         for s in (INT8, FP8R) for n, N, K in S.LLAMA31_8B])
     w["kproj"] = Workload(
         "kproj", "W8A8 int8 k_proj shape: X [8, 4096] with 8 outlier channels, W [1024, 4096]",
         "GB/s", [Product("k_proj", INT8, 8, 1024, 4096, 8)])
@@ -169,8 +170,9 @@ def workloads():
         "one grouped launch each on their shared input)", "GB/s",
         [Product(n, FP8B, 1, N, K, 0, group=LAYER_INPUT.get(n, n)) for n, N, K in S.QWEN3_8B])
     w["qwen-small"] = Workload(
-        "qwen-small", "Qwen3-8B FP8 128x128-block projections at M=32 (7 shapes)", "GB/s",
-        [Product(n, FP8B, 32, N, K, 0) for n, N, K in S.QWEN3_8B])
+        "qwen-small", "Qwen3-8B FP8 128x128-block projections at M=32 (7 shapes; q|k|v and gate|up one "
+        "grouped launch each on their shared tokens)", "GB/s",
+        [Product(n, FP8B, 32, N, K, 0, group=LAYER_INPUT.get(n, n)) for n, N, K in S.QWEN3_8B])
     w["decode-f2"] = Workload(
         "decode-f2", "decode GEMV M=1 as the decode workload, each input arriving already quantized "
         "(codes + scales written by its producer): q|k|v and gate|up grouped, 4 launches per scheme",
@@ -179,9 +181,9 @@ def workloads():
     w["small-f2"] = Workload(
         "small-f2", "small-batch tensor-core path as the small workload (M in {2, 8, 16, 32} x the 7 "
         "Llama-3.1-8B shapes x {W8A8, FP8 row}), each input arriving already quantized: one kernel "
-        "per product", "GB/s",
-        [Product(n, s, M, N, K, oc(K), pre=True) for M in (2, 8, 16, 32) for s in (INT8, FP8R)
-         for n, N, K in S.LLAMA31_8B])
+        "per group (q|k|v and gate|up grouped on their shared tokens)", "GB/s",
+        [Product(n, s, M, N, K, oc(K), group=LAYER_INPUT.get(n, n), pre=True) for M in (2, 8, 16, 32)
+         for s in (INT8, FP8R) for n, N, K in S.LLAMA31_8B])
     w["qwen-prefill-f2"] = Workload(
         "qwen-prefill-f2", "Qwen3-8B FP8 128x128-block projections at M=512 (7 shapes), each input "
         "arriving already quantized and each product also writing its own output's E4M3 codes and "
@@ -397,6 +399,9 @@ class Runner:
             if gemm_grouped_route(p):
                 gws = ql.gemm_grouped_workspace_bytes(p.scheme, [i["p"].N for i in g["items"]], p.M, p.K)
                 g["ws_gemm"] = ql.new_workspace(gws) if gws else None
+            if small_grouped_route(p):
+                g["ws_small"] = ql.new_workspace(
+                    ql.gemm_small_grouped_workspace_bytes(p.scheme, [i["p"].N for i in g["items"]], p.M, p.K))
         torch.cuda.synchronize()
         self.items = [i for g in self.groups for i in g["items"]]
         self.step_amount = step_amount(wl)  # a group reads its one input once
@@ -415,6 +420,9 @@ class Runner:
             return 1
         if gemm_grouped_route(g["p0"]):
             return 1 if g["p0"].pre else 2
+        if small_grouped_route(g["p0"]):
+            p = g["p0"]
+            return 1 if (p.pre or gemv_route(p.M, p.K)) else 2
         return sum(1 if (i["p"].wo or i["p"].pre or gemv_route(i["p"].M, i["p"].K)) else 2
                    for i in g["items"])
 
@@ -445,10 +453,9 @@ class Runner:
             self.ql.quantize_act(g["p0"].scheme, x, qx, sx)
             self.ql.gemm_grouped(g["p0"].scheme, qx, sx, [(*self._w(i, t), y) for i, y in zip(items, ys)],
                                  workspace=g["ws_gemm"])
-        elif g["p0"].pre:  # 2 <= M <= 32 on quantized input
-            qx, sx = x
-            for i, y in zip(items, ys):
-                self.ql.gemm_small_prequant(i["p"].scheme, qx, sx, *self._w(i, t), i["ws"], y=y)
+        elif small_grouped_route(g["p0"]):
+            self.ql.gemm_small_grouped(g["p0"].scheme, x, [(*self._w(i, t), y) for i, y in zip(items, ys)],
+                                       g["ws_small"])
         else:
             for i, y in zip(items, ys):
                 self._forward(i, x, *self._w(i, t), y)
@@ -464,7 +471,7 @@ class Runner:
 
     def dominant_group(self, g, t):
         ql = self.ql
-        if self._grouped(g) or g["p0"].pre:  # one kernel per launch already
+        if self._grouped(g) or g["p0"].pre or small_grouped_route(g["p0"]):  # one launch (+ its quantization)
             self._run_group(g, g["x_in"][t], t)
         elif gemm_grouped_route(g["p0"]) and not g["p0"].pre:
             qx, sx = g["q"][t]
@@ -476,10 +483,8 @@ class Runner:
                 wq, sw = self._w(i, t)
                 if p.wo:
                     ql.gemv_weight_only(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
-                elif p.M == 1:
+                else:  # M = 1 (2 <= M <= 32 and M > 32 run grouped)
                     ql.gemv(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
-                else:  # 2 <= M <= 32 (M > 32 runs grouped)
-                    ql.gemm_small(p.scheme, i["xs"][t], wq, sw, i["ws"], y=i["ys"][t])
 
     def capture(self, fn, stream):
         torch = self.torch
@@ -559,13 +564,20 @@ def gemm_grouped_route(p: Product) -> bool:
     return p.M > 32 and not p.wo
 
 
+def small_grouped_route(p: Product) -> bool:
+    """True when a group of 2 <= M <= 32 products runs as one
+    qlinear_gemm_small_grouped call (a group of one included)."""
+    return 2 <= p.M <= 32 and not p.wo
+
+
 def dominant_launch_count(wl) -> int:
     """Launches of the dominant kernel in one step: one per group that runs
-    grouped (M = 1 quantized GEMV, M > 32 GEMM), else one per product."""
+    grouped (M = 1 quantized GEMV, 2 <= M <= 32 small-M, M > 32 GEMM), else one
+    per product."""
     n = 0
     for g in input_groups(wl):
         p = g[0]
-        n += 1 if ((p.M == 1 and not p.wo) or gemm_grouped_route(p)) else len(g)
+        n += 1 if ((p.M == 1 and not p.wo) or gemm_grouped_route(p) or small_grouped_route(p)) else len(g)
     return n
 
 

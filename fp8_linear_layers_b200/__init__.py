@@ -43,7 +43,8 @@ EXPORTS = ("qlinear_quantize_weight", "qlinear_quantize_act", "qlinear_gemv", "q
            "qlinear_debug_gemv_stalled", "qlinear_forward_weight_only", "qlinear_gemv_grouped",
            "qlinear_gemv_prequant", "qlinear_gemm_small_prequant",
            "qlinear_gemm_quant_out", "qlinear_weight_only_workspace_bytes", "qlinear_gemm_grouped",
-           "qlinear_gemm_grouped_workspace_bytes")
+           "qlinear_gemm_grouped_workspace_bytes", "qlinear_gemm_small_grouped",
+           "qlinear_gemm_small_grouped_workspace_bytes")
 
 
 class QLinearError(RuntimeError):
@@ -102,6 +103,9 @@ def lib() -> ctypes.CDLL:
         L.qlinear_gemm_grouped.argtypes = [i32, vp, vp, vp, i32, i64, i64, vp, sz, vp]
         L.qlinear_gemm_grouped_workspace_bytes.argtypes = [i32, vp, i32, i64, i64]
         L.qlinear_gemm_grouped_workspace_bytes.restype = sz
+        L.qlinear_gemm_small_grouped.argtypes = [i32, vp, vp, vp, vp, i32, i64, i64, vp, sz, vp]
+        L.qlinear_gemm_small_grouped_workspace_bytes.argtypes = [i32, vp, i32, i64, i64]
+        L.qlinear_gemm_small_grouped_workspace_bytes.restype = sz
         L.qlinear_forward.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]
         L.qlinear_gemm_small_noalloc.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp, vp]
         L.qlinear_workspace_bytes.argtypes = [i32, i64, i64, i64]
@@ -433,6 +437,42 @@ def gemm_grouped(scheme: int, qx: torch.Tensor, sx: torch.Tensor, problems, work
     _check(lib().qlinear_gemm_grouped(scheme, _dev(qx, torch.uint8, "qx"), _dev(sx, torch.float32, "sx"),
                                       ctypes.cast(table, ctypes.c_void_p), len(problems), M, K, wp, wn,
                                       _stream(stream)), "qlinear_gemm_grouped")
+    return ys
+
+
+def gemm_small_grouped_workspace_bytes(scheme: int, Ns, M: int, K: int) -> int:
+    arr = (ctypes.c_int64 * len(Ns))(*Ns)
+    return int(lib().qlinear_gemm_small_grouped_workspace_bytes(scheme, ctypes.cast(arr, ctypes.c_void_p),
+                                                                len(Ns), M, K))
+
+
+def gemm_small_grouped(scheme: int, x, problems, workspace: torch.Tensor, stream=None) -> list:
+    """Several 1 <= M <= 32 products on the same tokens in one launch.  x is a
+    bf16 [M,K] tensor or a pair (q_x [M,K] uint8, s_x f32) already quantized;
+    `problems` a list of (wq [N,K], sw, y or None); returns the outputs [M,N]."""
+    if not 1 <= len(problems) <= GEMM_MAX_GROUP:
+        raise ValueError(f"1 to {GEMM_MAX_GROUP} products per grouped launch")
+    qx, sx = x if isinstance(x, tuple) else (None, None)
+    xin = qx if qx is not None else x
+    M, K = xin.shape
+    table = (_GemmProblem * len(problems))()
+    ys = []
+    for j, (wq, sw, y) in enumerate(problems):
+        if wq.shape[1] != K:
+            raise ValueError("every product of a grouped launch reads the same [M,K] tokens")
+        N = wq.shape[0]
+        if y is None:
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=xin.device)
+        table[j] = _GemmProblem(_dev(wq, torch.uint8, "wq"), _dev(sw, torch.float32, "sw"),
+                                _dev(y, torch.bfloat16, "y"), None, None, N)
+        ys.append(y)
+    wp, wn = _ws(workspace)
+    if qx is None:
+        args = (_dev(x, torch.bfloat16, "x"), None, None)
+    else:
+        args = (None, _dev(qx, torch.uint8, "qx"), _dev(sx, torch.float32, "sx"))
+    _check(lib().qlinear_gemm_small_grouped(scheme, *args, ctypes.cast(table, ctypes.c_void_p), len(problems), M, K,
+                                            wp, wn, _stream(stream)), "qlinear_gemm_small_grouped")
     return ys
 
 

@@ -188,7 +188,7 @@ ql_status qlinear_gemv_grouped(ql_scheme scheme, const ql_gemv_problem* problems
   }
   DeviceInfo d;
   QL_TRY(current_device(&d));
-  cudaError_t e = ql::launch_gemv_grouped(scheme, problems, count, K, d.sms, d.status,
+  cudaError_t e = ql::launch_gemv_grouped(scheme, problems, count, 1, K, d.sms, d.status,
                                           static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemv_grouped");
 }
@@ -286,6 +286,52 @@ ql_status qlinear_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq
   cudaError_t e = ql::launch_gemm_small(scheme, x, wq, sw, M, N, K, y, workspace, ws_bytes, dbg,
                                         d.sms, d.status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm_small");
+}
+
+ql_status qlinear_gemm_small_grouped(ql_scheme scheme, const uint16_t* x, const void* qx, const float* sx,
+                                     const ql_gemm_problem* problems, int count, int64_t M, int64_t K,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  if (!valid_scheme(scheme)) return QL_ERR_INVALID_ARG;
+  if (!problems || count < 1 || count > QL_GEMM_MAX_GROUP) return QL_ERR_INVALID_ARG;
+  QL_TRY(check_k(scheme, K));
+  int64_t Ns[QL_GEMM_MAX_GROUP];
+  for (int j = 0; j < count; ++j) {
+    QL_TRY(check_n(scheme, problems[j].N, K));
+    QL_TRY(check_m(M, problems[j].N, K));
+    Ns[j] = problems[j].N;
+  }
+  if (M == 0) return QL_OK;
+  if (M > 32) return QL_ERR_UNSUPPORTED_SHAPE;
+  if (x) {
+    QL_TRY(need(x));
+  } else {
+    QL_TRY(need(qx));
+    QL_TRY(need(sx));
+  }
+  for (int j = 0; j < count; ++j) {
+    QL_TRY(need(problems[j].wq));
+    QL_TRY(need(problems[j].sw));
+    QL_TRY(need(problems[j].y));
+    if (problems[j].qy || problems[j].sy) return QL_ERR_INVALID_ARG;  // no output codes on this path
+  }
+  DeviceInfo d;
+  QL_TRY(current_device(&d));
+  const size_t need_ws = ql::gemm_small_group_workspace_bytes(scheme, M, Ns, count, K);
+  if (!workspace || ws_bytes < need_ws) return QL_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return QL_ERR_MISALIGNED;
+  cudaError_t e = ql::launch_gemm_small_group(scheme, x, problems, count, M, K, workspace, ws_bytes, nullptr, d.sms,
+                                              d.status, static_cast<cudaStream_t>(stream),
+                                              x ? nullptr : static_cast<const uint8_t*>(qx), x ? nullptr : sx);
+  return e == cudaSuccess ? QL_OK : cuda_fail(e, "qlinear_gemm_small_grouped");
+}
+
+size_t qlinear_gemm_small_grouped_workspace_bytes(ql_scheme scheme, const int64_t* Ns, int count, int64_t M,
+                                                  int64_t K) {
+  if (!valid_scheme(scheme) || !Ns || count < 1 || count > QL_GEMM_MAX_GROUP || M <= 0 || M > 32 || K <= 0)
+    return 0;
+  for (int j = 0; j < count; ++j)
+    if (Ns[j] <= 0) return 0;
+  return ql::gemm_small_group_workspace_bytes(scheme, M, Ns, count, K);
 }
 
 ql_status qlinear_gemm_small_prequant(ql_scheme scheme, const void* qx, const float* sx,

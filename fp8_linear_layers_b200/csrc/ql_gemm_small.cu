@@ -23,6 +23,9 @@
 // Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2..5
 // epilogue (one TMEM lane = one weight row per thread).  Every mbarrier wait is
 // bounded.
+#include <climits>
+#include <cstring>
+
 #include "ql_tc.cuh"
 #include "ql_internal.h"
 
@@ -48,12 +51,19 @@ struct SmallCfg {
   static_assert(kStage % 1024 == 0, "stage alignment");
 };
 
+// A launch runs 1 to kSmallMaxGroup products that read the same tokens (a
+// layer's q, k, v; gate, up): product j owns 128-row tiles [t0[j], t0[j+1]).
+constexpr int kSmallMaxGroup = QL_GEMM_MAX_GROUP;
+
 struct SmallParams {
   const float* sx;  // workspace: [M] or [M, K/128]
-  const float* sw;
-  uint16_t* y;
-  int M, N, K;
-  int ntn;          // 128-row tiles of W_q
+  const float* sw[kSmallMaxGroup];
+  uint16_t* y[kSmallMaxGroup];
+  int N[kSmallMaxGroup];
+  int t0[kSmallMaxGroup + 1];  // INT_MAX past the last product
+  int nprob;
+  int M, K;
+  int ntn;          // 128-row tiles of W_q, all products
   int nkb;          // 128-byte K blocks
   int units;        // ntn * nkb
   void* accum;         // [kSmallSlots][ntn][NTOK][128] int32 or f32: parked partials, or atomic
@@ -63,6 +73,33 @@ struct SmallParams {
   float* acc_f32;
   DevStatus* status;
 };
+
+// The products' W_q tensor maps (kernel parameters, read by TMA from the
+// parameter space).
+struct SmallMapsW {
+  CUtensorMap m[kSmallMaxGroup];
+};
+
+// Tile t's product and its tile index inside it, by constant-index selects.
+struct SmallProd {
+  const float* sw;
+  uint16_t* y;
+  int N, tl, j;
+};
+static_assert(kSmallMaxGroup == 4, "small_prod selects among four products");
+QL_DEVINL SmallProd small_prod(const SmallParams& p, int t) {
+  const int j = (t >= p.t0[1]) + (t >= p.t0[2]) + (t >= p.t0[3]);
+  SmallProd v;
+  v.j = j;
+  v.sw = j == 0 ? p.sw[0] : j == 1 ? p.sw[1] : j == 2 ? p.sw[2] : p.sw[3];
+  v.y = j == 0 ? p.y[0] : j == 1 ? p.y[1] : j == 2 ? p.y[2] : p.y[3];
+  v.N = j == 0 ? p.N[0] : j == 1 ? p.N[1] : j == 2 ? p.N[2] : p.N[3];
+  v.tl = t - (j == 0 ? 0 : j == 1 ? p.t0[1] : j == 2 ? p.t0[2] : p.t0[3]);
+  return v;
+}
+QL_DEVINL const CUtensorMap* small_map(const SmallMapsW& w, int j) {
+  return j == 0 ? &w.m[0] : j == 1 ? &w.m[1] : j == 2 ? &w.m[2] : &w.m[3];
+}
 
 // OR vote over the epilogue warps that doubles as their barrier.
 QL_DEVINL bool epi_any(bool pred) {
@@ -84,7 +121,7 @@ QL_DEVINL int unit_owner(int u, int U, int G) { return (int)((((int64_t)u + 1) *
 
 template <ql_scheme S, int NTOK>
 __global__ void __launch_bounds__(kSmallThreads, 1)
-    gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+    gemm_small_kernel(const __grid_constant__ SmallMapsW tmW, const __grid_constant__ CUtensorMap tmX,
                       const SmallParams p) {
   using Cfg = SmallCfg<NTOK>;
   constexpr bool kInt8 = S == QL_W8A8_INT8_ROW;
@@ -122,7 +159,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    tc::prefetch_tmap(&tmW);
+    for (int j = 0; j < p.nprob; ++j) tc::prefetch_tmap(small_map(tmW, j));
     tc::prefetch_tmap(&tmX);
   }
   if (warp == 1) {
@@ -147,8 +184,9 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       const int pre = n < kSmallEarlyStages ? n : kSmallEarlyStages;
       for (int j = 0; j < pre; ++j) {
         const int u = u0 + j;
+        const SmallProd pv = small_prod(p, u / nkb);
         mbar_arrive_expect_tx(&full[j], Cfg::kStage);
-        tc::tma_load_2d(ring + j * Cfg::kStage, &tmW, (u % nkb) * 128, (u / nkb) * 128, &full[j], pol_w);
+        tc::tma_load_2d(ring + j * Cfg::kStage, small_map(tmW, pv.j), (u % nkb) * 128, pv.tl * 128, &full[j], pol_w);
       }
       tc::grid_dependency_wait();  // q_x is written by the preceding kernel
       for (int j = 0; j < pre; ++j) {
@@ -166,7 +204,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         const int u = u0 + j;
         uint8_t* st = ring + s * Cfg::kStage;
         mbar_arrive_expect_tx(&full[s], Cfg::kStage);
-        tc::tma_load_2d(st, &tmW, (u % nkb) * 128, (u / nkb) * 128, &full[s], pol_w);
+        const SmallProd pv = small_prod(p, u / nkb);
+        tc::tma_load_2d(st, small_map(tmW, pv.j), (u % nkb) * 128, pv.tl * 128, &full[s], pol_w);
         tc::tma_load_2d(st + Cfg::kStageA, &tmX, (u % nkb) * 128, 0, &full[s], pol_x);
         issued = j + 1;
       }
@@ -241,7 +280,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       const int t = u / nkb;
       const int seg_end = min(u1, (t + 1) * nkb);
       const bool whole = (u == t * nkb) && (seg_end == (t + 1) * nkb);
-      const int n = t * 128 + q * 32 + lane;
+      const SmallProd pv = small_prod(p, t);
+      const int n = pv.tl * 128 + q * 32 + lane;  // this thread's output row in its product
       Acc acc[NTOK];
 #pragma unroll
       for (int m = 0; m < NTOK; ++m) acc[m] = 0;
@@ -262,7 +302,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         if (lane == 0) mbar_arrive(&tempty[buf]);
         ++jt;
       } else if (kBlock) {
-        const float* swt = p.sw + (int64_t)t * KB;
+        const float* swt = pv.sw + (int64_t)pv.tl * KB;
         // the next K block's scales are loaded while this block's MMAs run
         float sx_next[NTOK];
         float sw_next = __ldg(swt + (u - t * nkb));
@@ -357,22 +397,22 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
           if (et == 0) p.counters[t] = 0u;  // every contributor has arrived: reset for the next call
         }
       }
-      if (do_epilogue && n < p.N) {
-        const float swn = kBlock ? 1.0f : __ldg(p.sw + n);
+      if (do_epilogue && n < pv.N) {
+        const float swn = kBlock ? 1.0f : __ldg(pv.sw + n);
 #pragma unroll
         for (int m = 0; m < NTOK; ++m) {
           if (m < p.M) {
             float yv;
             if constexpr (kInt8) {
-              if (p.acc_i32) p.acc_i32[(int64_t)m * p.N + n] = acc[m];
+              if (p.acc_i32) p.acc_i32[(int64_t)m * pv.N + n] = acc[m];
               yv = __fmul_rn(__fmul_rn(__int2float_rn(acc[m]), __ldg(p.sx + m)), swn);
             } else if constexpr (kBlock) {
               yv = acc[m];
             } else {
-              if (p.acc_f32) p.acc_f32[(int64_t)m * p.N + n] = acc[m];
+              if (p.acc_f32) p.acc_f32[(int64_t)m * pv.N + n] = acc[m];
               yv = __fmul_rn(__fmul_rn(acc[m], __ldg(p.sx + m)), swn);
             }
-            p.y[(int64_t)m * p.N + n] = f32_to_bf16_rn(yv);
+            pv.y[(int64_t)m * pv.N + n] = f32_to_bf16_rn(yv);
           }
         }
       }
@@ -399,37 +439,49 @@ struct SmallLayout {
   size_t qx, sx, accum, counters, zeroed, total;
 };
 
-SmallLayout small_layout(ql_scheme s, int64_t M, int64_t N, int64_t K, int sms) {
+// ntiles: the 128-row W_q tiles of every product of the launch
+SmallLayout small_layout(ql_scheme s, int64_t M, int64_t ntiles, int64_t K) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
   const int ntok = M <= 16 ? 16 : 32;
-  (void)sms;
   // The region that must be zero when a call starts comes first: the arrival
   // counters, then partial-sum slot 0 of every tile (the atomic-sum slot);
   // slot 1 (parked partials, always written before they are read) follows.
-  const size_t slot_bytes = (size_t)((N + 127) / 128) * ntok * 128 * 4;
+  const size_t slot_bytes = (size_t)ntiles * ntok * 128 * 4;
   SmallLayout L;
   L.counters = 0;
-  L.accum = up((size_t)((N + 127) / 128) * 4);
+  L.accum = up((size_t)ntiles * 4);
   L.zeroed = L.accum + slot_bytes;
   L.qx = L.accum + up(kSmallSlots * slot_bytes);
   L.sx = L.qx + up((size_t)(M * K));
   L.total = L.sx + up((size_t)M * (s == QL_FP8_E4M3_BLOCK128 ? K / 128 : 1) * 4);
   return L;
 }
+
+int64_t small_tiles(const int64_t* Ns, int count) {
+  int64_t t = 0;
+  for (int j = 0; j < count; ++j) t += (Ns[j] + 127) / 128;
+  return t;
+}
 }  // namespace
 
+size_t gemm_small_group_workspace_bytes(ql_scheme scheme, int64_t M, const int64_t* Ns, int count, int64_t K) {
+  return small_layout(scheme, M, small_tiles(Ns, count), K).total;
+}
+
 size_t gemm_small_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms) {
-  return small_layout(scheme, M, N, K, num_sms).total;
+  (void)num_sms;
+  return gemm_small_group_workspace_bytes(scheme, M, &N, 1, K);
 }
 
 size_t gemm_small_zeroed_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms) {
+  (void)num_sms;
   // the GEMV route (up to four tokens) does not touch the workspace
   if (K <= gemv_max_k_tokens(M)) return 0;
-  return small_layout(scheme, M, N, K, num_sms).zeroed;
+  return small_layout(scheme, M, (N + 127) / 128, K).zeroed;
 }
 
 template <ql_scheme S, int NTOK>
-static cudaError_t launch_small_t(const SmallParams& p, const CUtensorMap& tw, const CUtensorMap& tx,
+static cudaError_t launch_small_t(const SmallParams& p, const SmallMapsW& tw, const CUtensorMap& tx,
                                   int grid, cudaStream_t st) {
   using Cfg = SmallCfg<NTOK>;
   cudaError_t e = ensure_smem<gemm_small_kernel<S, NTOK>>(Cfg::kSmem);
@@ -447,13 +499,15 @@ static cudaError_t launch_small_t(const SmallParams& p, const CUtensorMap& tw, c
   return cudaLaunchKernelEx(&cfg, gemm_small_kernel<S, NTOK>, tw, tx, p);
 }
 
-cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq,
-                              const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
-                              void* workspace, size_t ws_bytes, const ql_debug* dbg, int num_sms,
-                              DevStatus* status, cudaStream_t st, const uint8_t* pre_qx,
-                              const float* pre_sx) {
-  const SmallLayout L = small_layout(scheme, M, N, K, num_sms);
-  if (ws_bytes < L.total) return cudaErrorInvalidValue;
+cudaError_t launch_gemm_small_group(ql_scheme scheme, const uint16_t* x, const ql_gemm_problem* probs, int count,
+                                    int64_t M, int64_t K, void* workspace, size_t ws_bytes, const ql_debug* dbg,
+                                    int num_sms, DevStatus* status, cudaStream_t st, const uint8_t* pre_qx,
+                                    const float* pre_sx) {
+  if (count < 1 || count > kSmallMaxGroup || (dbg && count != 1)) return cudaErrorInvalidValue;
+  int64_t Ns[kSmallMaxGroup];
+  for (int j = 0; j < count; ++j) Ns[j] = probs[j].N;
+  const int64_t ntiles = small_tiles(Ns, count);
+  const SmallLayout L = small_layout(scheme, M, ntiles, K);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const uint8_t* qx = pre_qx;
   const float* sx = pre_sx;
@@ -462,23 +516,51 @@ cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* w
     // Up to four tokens: the GEMV kernel carries them on its MMA's B columns
     // with the activation quantization fused, at the weight traffic of one
     // token and without the split-K reduction (the workspace is not used).
-    if (K <= gemv_max_k_tokens(M))
-      return launch_gemv(scheme, x, wq, sw, M, N, K, y, dbg, num_sms, status, st);
+    if (K <= gemv_max_k_tokens(M)) {
+      if (count == 1) return launch_gemv(scheme, x, probs[0].wq, probs[0].sw, M, probs[0].N, K, probs[0].y, dbg,
+                                         num_sms, status, st);
+      ql_gemv_problem g[kSmallMaxGroup];
+      for (int j = 0; j < count; ++j) g[j] = ql_gemv_problem{x, nullptr, nullptr, probs[j].wq, probs[j].sw,
+                                                              probs[j].y, probs[j].N};
+      return launch_gemv_grouped(scheme, g, count, M, K, num_sms, status, st);
+    }
+    if (ws_bytes < L.total) return cudaErrorInvalidValue;
     uint8_t* wqx = ws + L.qx;
     float* wsx = reinterpret_cast<float*>(ws + L.sx);
     if ((e = launch_quantize_act(scheme, x, M, K, wqx, wsx, st)) != cudaSuccess) return e;
     qx = wqx;
     sx = wsx;
+  } else if (ws_bytes < L.total) {
+    return cudaErrorInvalidValue;
   }
 
   SmallParams p;
   p.sx = sx;
-  p.sw = sw;
-  p.y = y;
+  p.nprob = count;
   p.M = (int)M;
-  p.N = (int)N;
   p.K = (int)K;
-  p.ntn = (int)((N + 127) / 128);
+  SmallMapsW tw;
+  memset(&tw, 0, sizeof(tw));
+  int t = 0;
+  for (int j = 0; j < kSmallMaxGroup; ++j) {
+    if (j < count) {
+      p.sw[j] = probs[j].sw;
+      p.y[j] = probs[j].y;
+      p.N[j] = (int)probs[j].N;
+      p.t0[j] = t;
+      t += (int)((probs[j].N + 127) / 128);
+      if ((e = make_tmap_u8_sw128(&tw.m[j], probs[j].wq, (uint64_t)K, (uint64_t)probs[j].N, (uint64_t)K, 128,
+                                  128)) != cudaSuccess)
+        return e;
+    } else {
+      p.sw[j] = nullptr;
+      p.y[j] = nullptr;
+      p.N[j] = 0;
+      p.t0[j] = INT_MAX;
+    }
+  }
+  p.t0[kSmallMaxGroup] = INT_MAX;
+  p.ntn = t;
   p.nkb = (int)((K + 127) / 128);
   p.units = p.ntn * p.nkb;
   p.accum = ws + L.accum;
@@ -487,9 +569,7 @@ cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* w
   p.acc_f32 = dbg ? dbg->acc_f32 : nullptr;
   p.status = status;
   const int ntok = M <= 16 ? 16 : 32;
-  CUtensorMap tw, tx;
-  if ((e = make_tmap_u8_sw128(&tw, wq, (uint64_t)K, (uint64_t)N, (uint64_t)K, 128, 128)) != cudaSuccess)
-    return e;
+  CUtensorMap tx;
   if ((e = make_tmap_u8_sw128(&tx, qx, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)ntok)) !=
       cudaSuccess)
     return e;
@@ -517,6 +597,16 @@ cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* w
       return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq,
+                              const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                              void* workspace, size_t ws_bytes, const ql_debug* dbg, int num_sms,
+                              DevStatus* status, cudaStream_t st, const uint8_t* pre_qx,
+                              const float* pre_sx) {
+  const ql_gemm_problem one{wq, sw, y, nullptr, nullptr, N};
+  return launch_gemm_small_group(scheme, x, &one, 1, M, K, workspace, ws_bytes, dbg, num_sms, status, st, pre_qx,
+                                 pre_sx);
 }
 
 }  // namespace ql

@@ -1022,13 +1022,13 @@ cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, con
   return launch_gemv_scheme<false>(scheme, p, grid, smem, st);
 }
 
-cudaError_t launch_gemv_grouped(ql_scheme scheme, const ql_gemv_problem* probs, int count,
+cudaError_t launch_gemv_grouped(ql_scheme scheme, const ql_gemv_problem* probs, int count, int64_t M,
                                 int64_t K, int num_sms, DevStatus* status, cudaStream_t st) {
-  if (K > gemv_max_k()) return cudaErrorInvalidValue;
+  if (M < 1 || M > 4 || K > gemv_max_k_tokens(M)) return cudaErrorInvalidValue;
   GemvParams p;
   int grid = 0;
   size_t smem = 0;
-  cudaError_t e = gemv_setup(p, 1, probs, count, K, 1, num_sms, &grid, &smem);
+  cudaError_t e = gemv_setup(p, M, probs, count, K, 1, num_sms, &grid, &smem);
   if (e != cudaSuccess) return e;
   p.dbg = ql_debug{nullptr, nullptr, nullptr, nullptr};
   p.status = status;

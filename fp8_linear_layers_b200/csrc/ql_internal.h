@@ -49,8 +49,9 @@ int gemv_max_k_tokens(int64_t M);  // largest K the GEMV takes for M tokens (0: 
 cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, const float* sw,
                         int64_t M, int64_t N, int64_t K, uint16_t* y, const ql_debug* dbg,
                         int num_sms, DevStatus* status, cudaStream_t st, bool stall = false);
-// Up to QL_GEMV_MAX_GROUP M = 1 products of the same K in one launch.
-cudaError_t launch_gemv_grouped(ql_scheme scheme, const ql_gemv_problem* probs, int count,
+// Up to QL_GEMV_MAX_GROUP products of the same K and token count (1..4) in one
+// launch; K <= gemv_max_k_tokens(M).
+cudaError_t launch_gemv_grouped(ql_scheme scheme, const ql_gemv_problem* probs, int count, int64_t M,
                                 int64_t K, int num_sms, DevStatus* status, cudaStream_t st);
 // 1 <= M <= 4 weight-only product: x stays bf16 (staged as exactly scaled f16),
 // W codes dequantized to f16 in registers, f32 sums; K <= gemv_weight_only_max_k().
@@ -93,6 +94,14 @@ size_t gemm_small_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_
 // completed call leaves them zero.  0 when the shape runs on the GEMV kernel,
 // which does not use the workspace.
 size_t gemm_small_zeroed_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);
+// A group of 1..QL_GEMM_MAX_GROUP products on the same tokens (their N in
+// Ns): one quantization of the tokens and one launch (up to four tokens within
+// the GEMV's K limits: one grouped GEMV launch, no workspace used).
+size_t gemm_small_group_workspace_bytes(ql_scheme scheme, int64_t M, const int64_t* Ns, int count, int64_t K);
+cudaError_t launch_gemm_small_group(ql_scheme scheme, const uint16_t* x, const ql_gemm_problem* probs, int count,
+                                    int64_t M, int64_t K, void* workspace, size_t ws_bytes, const ql_debug* dbg,
+                                    int num_sms, DevStatus* status, cudaStream_t st,
+                                    const uint8_t* pre_qx = nullptr, const float* pre_sx = nullptr);
 // pre_qx / pre_sx: the input already quantized (x unused; no quantization
 // launch and no GEMV route).
 cudaError_t launch_gemm_small(ql_scheme scheme, const uint16_t* x, const void* wq,

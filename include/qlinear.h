@@ -362,6 +362,32 @@ ql_status qlinear_gemm_grouped(ql_scheme scheme, const void* qx, const float* sx
 size_t qlinear_gemm_grouped_workspace_bytes(ql_scheme scheme, const int64_t* Ns, int count, int64_t M,
                                             int64_t K);
 
+/* Several 1 <= M <= 32 products on the same tokens in one launch (a layer's
+ * q, k, v, or gate, up, in a small decode batch): the tokens are quantized
+ * once, and the 128-row weight tiles of every product share the SM-balanced
+ * K split, so that the small products (k and v: 4 MB of weights each) do not
+ * pay a launch and a reduction of their own.  Up to four tokens within the
+ * GEMV's K limits (as for qlinear_gemm_small) run as one grouped GEMV launch
+ * instead.  Numerics of each product as qlinear_gemm_small.  Pages: as for
+ * qlinear_gemm_small.
+ *   x          device, bf16 [M,K] tokens, quantized in the call; or NULL with
+ *   qx, sx     device, the tokens already quantized (codes [M,K], scales as
+ *              qlinear_quantize_act writes them): the tensor-core kernel runs
+ *              for every M, with no quantization launch
+ *   problems   host array of `count` descriptors, 1 <= count <=
+ *              QL_GEMM_MAX_GROUP (read during the call only): wq, sw, y, N as
+ *              for qlinear_gemm_grouped; qy and sy must be NULL
+ *   workspace  device, at least qlinear_gemm_small_grouped_workspace_bytes(...)
+ *              bytes, 256-byte aligned, zero-filled before its first use (as
+ *              for qlinear_gemm_small: a completed call leaves it ready)
+ * Errors: as for qlinear_gemm_small on every product; count outside
+ * [1, QL_GEMM_MAX_GROUP] or qy / sy set -> QL_ERR_INVALID_ARG. */
+ql_status qlinear_gemm_small_grouped(ql_scheme scheme, const uint16_t* x, const void* qx, const float* sx,
+                                     const ql_gemm_problem* problems, int count, int64_t M, int64_t K,
+                                     void* workspace, size_t ws_bytes, void* stream);
+size_t qlinear_gemm_small_grouped_workspace_bytes(ql_scheme scheme, const int64_t* Ns, int count, int64_t M,
+                                                  int64_t K);
+
 /* The projection as a model calls it: bf16 X in, bf16 Y out, dispatching on
  * the token count the way the pages' "Loading" sections describe: M = 1 ->
  * qlinear_gemv, 2..32 -> qlinear_gemm_small, > 32 -> qlinear_quantize_act

@@ -114,6 +114,21 @@ def test_host_validation_rejects_before_launch(L):
     assert GG(0, ALIGNED, ALIGNED, gp, 2, 64, 256, None, 0, None) == SHAPE  # codes: block scheme only
     gt[1].sy = ALIGNED + 4
     assert GG(2, ALIGNED, ALIGNED, gp, 2, 64, 256, None, 0, None) == MIS
+    # the grouped small-M path: 1 <= M <= 32, tokens bf16 or pre-quantized, no output codes
+    gt[0].qy = gt[0].sy = gt[1].qy = gt[1].sy = 0
+    gt[0].y = gt[1].y = ALIGNED
+    gt[1].N = 256
+    GS = L.qlinear_gemm_small_grouped
+    assert GS(0, ALIGNED, None, None, gp, 0, 8, 256, ALIGNED, 1 << 20, None) == INV
+    assert GS(0, ALIGNED, None, None, gp, ql.GEMM_MAX_GROUP + 1, 8, 256, ALIGNED, 1 << 20, None) == INV
+    assert GS(0, ALIGNED, None, None, gp, 2, 33, 256, ALIGNED, 1 << 20, None) == SHAPE
+    assert GS(0, None, None, None, gp, 2, 8, 256, ALIGNED, 1 << 20, None) == INV      # no tokens
+    assert GS(0, None, ALIGNED, None, gp, 2, 8, 256, ALIGNED, 1 << 20, None) == INV   # codes without scales
+    assert GS(0, ALIGNED + 8, None, None, gp, 2, 8, 256, ALIGNED, 1 << 20, None) == MIS
+    gt[1].qy = ALIGNED
+    assert GS(0, ALIGNED, None, None, gp, 2, 8, 256, ALIGNED, 1 << 20, None) == INV   # no output codes here
+    gt[1].qy = 0
+    assert GS(0, ALIGNED, None, None, gp, 2, 0, 256, None, 0, None) == 0             # M = 0
     PQ = L.qlinear_gemv_prequant
     assert PQ(0, None, ALIGNED, ALIGNED, ALIGNED, 64, 64, ALIGNED, None) == INV
     assert PQ(0, ALIGNED, None, ALIGNED, ALIGNED, 64, 64, ALIGNED, None) == INV

@@ -120,7 +120,9 @@ def test_grouped_launch_counts():
     assert bench.dominant_launch_count(w["qwen-prefill"]) == 4
     # inputs arriving quantized, outputs leaving quantized: the same 4 launches, no quantization launch
     assert bench.dominant_launch_count(w["qwen-prefill-f2"]) == 4
-    assert bench.dominant_launch_count(w["small"]) == len(w["small"].products)
+    # small-M: per M and scheme, q|k|v and gate|up grouped, o and down alone
+    assert bench.dominant_launch_count(w["small"]) == 4 * 2 * 4
+    assert bench.dominant_launch_count(w["kproj"]) == 1
     # the step's bytes: decode reads each group's input once
     dec = w["decode"]
     assert bench.step_bytes(dec) == bench.step_amount(dec)
