@@ -506,22 +506,31 @@ class Runner:
         ys_tot = sum(i["p"].M * i["p"].N for i in self.items)
         h_y = torch.empty(ys_tot, dtype=torch.bfloat16, pin_memory=True)
         d_y = torch.empty(ys_tot, dtype=torch.bfloat16, device="cuda")
-        views, copies, h2d, oy = [], [], 0, 0
+        # every group's input in one pinned buffer and one device buffer (256-byte
+        # aligned parts), so that a step's inputs cross in one copy
+        srcs = []
         for g in self.groups:
             src = g["x_in"][0]
-            parts = list(src) if isinstance(src, tuple) else [src]
-            dev = [torch.empty_like(a) for a in parts]
-            for a, d in zip(parts, dev):
-                h = torch.empty(a.shape, dtype=a.dtype, pin_memory=True)
-                h.copy_(a.cpu())
-                copies.append((d, h))
-                h2d += a.numel() * a.element_size()
+            srcs.append(list(src) if isinstance(src, tuple) else [src])
+        sizes = [[a.numel() * a.element_size() for a in parts] for parts in srcs]
+        total = sum((n + 255) // 256 * 256 for ns in sizes for n in ns)
+        h_x = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+        d_x = torch.empty(total, dtype=torch.uint8, device="cuda")
+        views, h2d, oy, ox = [], 0, 0, 0
+        for g, parts, ns in zip(self.groups, srcs, sizes):
+            dev = []
+            for a, n in zip(parts, ns):
+                h_x[ox:ox + n].copy_(a.contiguous().view(-1).view(torch.uint8).cpu())
+                dev.append(d_x[ox:ox + n].view(a.dtype).view(a.shape))
+                ox += (n + 255) // 256 * 256
+                h2d += n
             yv = []
             for i in g["items"]:
                 q = i["p"]
                 yv.append(d_y[oy:oy + q.M * q.N].view(q.M, q.N))
                 oy += q.M * q.N
-            views.append((g, tuple(dev) if isinstance(src, tuple) else dev[0], yv))
+            views.append((g, tuple(dev) if len(dev) > 1 else dev[0], yv))
+        copies = [(d_x, h_x)]
 
         def body(c):
             for g, xv, yv in views:
