@@ -312,18 +312,22 @@ def nvsmi_index(torch, dev: int):
 L2_BYTES = 126e6
 
 # DRAM bytes per launch of the dominant kernel from one ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum), with the hash of the kernel sources it was taken on: when the
-# sources differ the figure no longer describes the kernel and the line reports null.
-_GEMV_SOURCES = ["ql_gemv.cu", "ql_common.cuh", "ql_tc.cuh", "ql_internal.h"]
-_GEMM_SOURCES = ["ql_gemm.cu", "ql_common.cuh", "ql_tc.cuh", "ql_internal.h"]
+# dram__bytes_write.sum), with the hash of the kernel sources it was taken on (the kernel's
+# file and the device headers it includes; ql_internal.h declares host functions only): when
+# the sources differ the figure no longer describes the kernel and the line reports null.
+_GEMV_SOURCES = ["ql_gemv.cu", "ql_common.cuh", "ql_tc.cuh"]
+_GEMM_SOURCES = ["ql_gemm.cu", "ql_common.cuh", "ql_tc.cuh"]
+# the small-M workload's products run on the small-M kernel and (two tokens) on the GEMV
+_SMALL_SOURCES = ["ql_gemm_small.cu", "ql_gemv.cu", "ql_common.cuh", "ql_tc.cuh"]
 KERNEL_SOURCES = {"ql::gemv_kernel": _GEMV_SOURCES, "ql::gemv_kernel (weight-only)": _GEMV_SOURCES,
-                  "ql::gemm_kernel": _GEMM_SOURCES, "ql::gemm_kernel (output quantization fused)": _GEMM_SOURCES}
+                  "ql::gemm_kernel": _GEMM_SOURCES, "ql::gemm_kernel (output quantization fused)": _GEMM_SOURCES,
+                  "ql::gemm_small_kernel": _SMALL_SOURCES}
 TRAFFIC = {
     # workload: (bytes per launch, kernel source hash, summary file)
-    "decode": (54668224, "f67eb144cf9e747e", "profiles/gemv_decode_dram.md"),
-    "decode-wo": (31224887, "233ea157dd920e9f", "profiles/gemv_decode_weight_only_dram.md"),
-    "prefill": (75563605, "f5f95d3f977ccd3f", "profiles/gemm_prefill_int8_dram.md"),
-    "qwen-prefill": (52263872, "f5f95d3f977ccd3f", "profiles/gemm_qwen_prefill_block_dram.md"),
+    "decode": (54663840, "29a9fc85af754e2a", "profiles/gemv_decode_dram.md"),
+    "prefill": (75848448, "9e19ad71c9866eb3", "profiles/gemm_prefill_int8_dram.md"),
+    "qwen-prefill": (52170240, "9e19ad71c9866eb3", "profiles/gemm_qwen_prefill_block_dram.md"),
+    "small": (55246976, "5d259a5c0a98cba4", "profiles/gemm_small_dram.md"),
 }
 
 
