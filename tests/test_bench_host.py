@@ -94,7 +94,7 @@ def test_traffic_is_tied_to_kernel_sources(monkeypatch):
     monkeypatch.setitem(bench.TRAFFIC, "decode", (123, "0" * 16, "profiles/x.md"))
     assert bench.measured_traffic(wl) == (None, None)
     # a workload without a capture reports null
-    assert bench.measured_traffic(bench.workloads()["small"]) == (None, None)
+    assert bench.measured_traffic(bench.workloads()["qwen-small"]) == (None, None)
 
 
 def test_committed_traffic_summaries_exist():
