@@ -325,8 +325,8 @@ KERNEL_SOURCES = {"ql::gemv_kernel": _GEMV_SOURCES, "ql::gemv_kernel (weight-onl
 TRAFFIC = {
     # workload: (bytes per launch, kernel source hash, summary file)
     "decode": (54663840, "29a9fc85af754e2a", "profiles/gemv_decode_dram.md"),
-    "prefill": (75848448, "9e19ad71c9866eb3", "profiles/gemm_prefill_int8_dram.md"),
-    "qwen-prefill": (52170240, "9e19ad71c9866eb3", "profiles/gemm_qwen_prefill_block_dram.md"),
+    "prefill": (75848448, "87b077ff18efb3b1", "profiles/gemm_prefill_int8_dram.md"),
+    "qwen-prefill": (52170240, "87b077ff18efb3b1", "profiles/gemm_qwen_prefill_block_dram.md"),
     "small": (55246976, "5d259a5c0a98cba4", "profiles/gemm_small_dram.md"),
 }
 

@@ -67,9 +67,9 @@ struct GemmParams {
   int nprob;
   int M, K;
   int mt, ntiles, nkb;  // tiles along M, tiles in all, K blocks of 128
-  int split;        // block scheme: K halves per tile (1 = whole tiles, or 2)
-  float* parts;     // split = 2: f32 partial sums, [half][tile][warp][column / 4][lane][4]
-  uint32_t* counters;  // split = 2: [mt * nt] arrivals per tile, zero between calls
+  int split;        // K parts per tile (1 = whole tiles; 2, or up to 8 for 128-wide block tiles)
+  float* parts;     // split > 1: partial sums, [part][tile][warp][column / 4][lane][4]
+  uint32_t* counters;  // split > 1: [tiles] arrivals per tile, zero between calls
   int32_t* acc_i32;
   float* acc_f32;
   uint8_t* qy[kGemmMaxGroup];  // block scheme: E4M3 codes of each y [M,N] for the product that reads it next

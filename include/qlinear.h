@@ -277,22 +277,25 @@ ql_status qlinear_gemm_small_prequant(ql_scheme scheme, const void* qx, const fl
  * (larger batches: per-token int8 activations, int8 products, int32
  * accumulation); Qwen3 FP8 "Loading" (block scales).
  *   qx, sx     device, from qlinear_quantize_act
- *   workspace  optional (NULL / 0 bytes: whole tiles).  Block scheme only:
- *              when the output tiles are few -- 128x256 tiles filling at
- *              most half the SMs with K >= 8192 (e.g. M = 512, N = 4096), or
- *              128x128 tiles filling at most a quarter of them (e.g. M = 512,
- *              N = 1024) -- a workspace of at least
- *              qlinear_workspace_bytes(...) bytes (256-byte aligned,
+ *   workspace  optional (NULL / 0 bytes: whole tiles).  When the output
+ *              tiles are few -- 128x256 tiles filling at most half the SMs
+ *              with K >= 8192 (e.g. M = 512, N = 4096, K = 14336; every
+ *              scheme), or, block scheme, 128x128 tiles filling at most a
+ *              quarter of them (e.g. M = 512, N = 1024) -- a workspace of at
+ *              least qlinear_workspace_bytes(...) bytes (256-byte aligned,
  *              ZERO-FILLED before its first use) lets the call split each
- *              tile's K blocks over 2 (or, for 128-wide tiles, up to 4) CTAs
- *              that park their f32 partial sums in it (one 128x256 f32 slab
- *              per part per output tile, then one arrival counter per tile);
- *              the last to arrive adds the parts in part order (the same
- *              bits whatever the order of arrival).  A completed call leaves
- *              the counters zero again, for any next shape; zero the
- *              workspace again after a QL_ERR_TIMEOUT.  Two calls in flight
- *              at the same time must not share it.  Row schemes:
- *              qlinear_workspace_bytes returns 0.
+ *              tile's K blocks over 2 (or, for 128-wide block tiles, up to 4)
+ *              CTAs that park their partial sums in it (the block scheme's
+ *              f32 running sums; the row schemes' raw s32 / f32
+ *              accumulators, added before the scales: int8 outputs stay
+ *              bit-exact) -- one 128x256 slab per part per output tile, then
+ *              one arrival counter per tile; the last to arrive adds the
+ *              parts in part order (the same bits whatever the order of
+ *              arrival).  A completed call leaves the counters zero again,
+ *              for any next shape; zero the workspace again after a
+ *              QL_ERR_TIMEOUT.  Two calls in flight at the same time must not
+ *              share it.  qlinear_workspace_bytes returns 0 for shapes that
+ *              run whole tiles.
  *   dbg        optional (NULL): acc_i32 (int8) / acc_f32 (E4M3 row) [M,N] */
 ql_status qlinear_gemm(ql_scheme scheme, const void* qx, const float* sx, const void* wq,
                        const float* sw, int64_t M, int64_t N, int64_t K, uint16_t* y,
