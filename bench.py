@@ -92,7 +92,10 @@ class Workload:
             return "ql::gemv_kernel (weight-only)"
         if p.M > 32 and p.pre:
             return "ql::gemm_kernel (output quantization fused)"
-        return "ql::gemv_kernel" if p.M == 1 else ("ql::gemm_small_kernel" if p.M <= 32 else "ql::gemm_kernel")
+        if p.M == 1 or all(not g[0].pre and not g[0].wo and gemv_route(g[0].M, g[0].K, g)
+                           for g in input_groups(self)):
+            return "ql::gemv_kernel"
+        return "ql::gemm_small_kernel" if p.M <= 32 else "ql::gemm_kernel"
 
     @staticmethod
     def input_bytes(p: Product) -> float:
@@ -120,10 +123,15 @@ LAYER_INPUT = {"q_proj": "qkv", "k_proj": "qkv", "v_proj": "qkv", "gate_proj": "
                "up_proj": "gate_up"}
 
 
-def gemv_route(M: int, K: int) -> bool:
-    """True when the library runs an M-token product on the GEMV kernel (one
-    launch): M = 1 up to K = 32768, two tokens up to 16384, three or four up to 8192."""
-    return (M == 1 and K <= 32768) or (M == 2 and K <= 16384) or (M in (3, 4) and K <= 8192)
+def gemv_route(M: int, K: int, group=()) -> bool:
+    """True when the library runs M-token products on bf16 input (`group`: the
+    products of one launch) on the GEMV kernel: M = 1 up to K = 32768, two
+    tokens up to 16384, three or four up to 8192, and five to eight up to 8192
+    when the launch's weights take at most 8 MiB (two products of up to four
+    tokens each)."""
+    if (M == 1 and K <= 32768) or (M == 2 and K <= 16384) or (M in (3, 4) and K <= 8192):
+        return True
+    return 5 <= M <= 8 and K <= 8192 and sum(q.N * q.K for q in group) <= (8 << 20)
 
 
 def workloads():
@@ -324,10 +332,11 @@ KERNEL_SOURCES = {"ql::gemv_kernel": _GEMV_SOURCES, "ql::gemv_kernel (weight-onl
                   "ql::gemm_small_kernel": _SMALL_SOURCES}
 TRAFFIC = {
     # workload: (bytes per launch, kernel source hash, summary file)
-    "decode": (54663840, "29a9fc85af754e2a", "profiles/gemv_decode_dram.md"),
+    "decode": (54660384, "c19c7146a24ad7ed", "profiles/gemv_decode_dram.md"),
+    "kproj": (4325504, "c19c7146a24ad7ed", "profiles/gemv_kproj_dram.md"),
     "prefill": (75848448, "87b077ff18efb3b1", "profiles/gemm_prefill_int8_dram.md"),
     "qwen-prefill": (52170240, "87b077ff18efb3b1", "profiles/gemm_qwen_prefill_block_dram.md"),
-    "small": (55246976, "5d259a5c0a98cba4", "profiles/gemm_small_dram.md"),
+    "small": (55263000, "82bb5f3ca16b177a", "profiles/gemm_small_dram.md"),
 }
 
 
@@ -426,8 +435,8 @@ class Runner:
             return 1 if g["p0"].pre else 2
         if small_grouped_route(g["p0"]):
             p = g["p0"]
-            return 1 if (p.pre or gemv_route(p.M, p.K)) else 2
-        return sum(1 if (i["p"].wo or i["p"].pre or gemv_route(i["p"].M, i["p"].K)) else 2
+            return 1 if (p.pre or gemv_route(p.M, p.K, [i["p"] for i in g["items"]])) else 2
+        return sum(1 if (i["p"].wo or i["p"].pre or gemv_route(i["p"].M, i["p"].K, [i["p"]])) else 2
                    for i in g["items"])
 
     def _w(self, i, t):

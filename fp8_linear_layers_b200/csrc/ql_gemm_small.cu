@@ -524,6 +524,10 @@ cudaError_t launch_gemm_small_group(ql_scheme scheme, const uint16_t* x, const q
                                                               probs[j].y, probs[j].N};
       return launch_gemv_grouped(scheme, g, count, M, K, num_sms, status, st);
     }
+    // Five to eight tokens on small weights: the same kernel, each product
+    // as two of four tokens or fewer on the same weights.
+    if (!dbg && gemv_token_halves_pay(M, K, Ns, count))
+      return launch_gemv_token_halves(scheme, x, probs, count, M, K, num_sms, status, st);
     if (ws_bytes < L.total) return cudaErrorInvalidValue;
     uint8_t* wqx = ws + L.qx;
     float* wsx = reinterpret_cast<float*>(ws + L.sx);

@@ -62,7 +62,15 @@ constexpr int64_t kGemvStashMaxK = 16384;       // one token's bf16 x parked in 
 constexpr int kGemvMaxK = 32768;
 constexpr int64_t kGemvMaxK2 = 16384;           // two tokens: units of at most 64 windows
 constexpr int64_t kGemvMaxK4 = 8192;            // three or four tokens: stages of 8 rows
-constexpr int64_t kGemvMaxKWO = 16384;          // weight-only: 2K bytes of staged x beside the ring
+constexpr int64_t kGemvMaxKWO = 16384;
+// Five to eight tokens run on this kernel as two products of up to four
+// tokens over the same weights when the launch's weights take at most this
+// many bytes.  The halves' SMs each take the weight bytes in, so a launch
+// streams them twice over the SMs' ports (L2 hits arrive no faster than HBM
+// reads under a full stream).  Measured on B200, M = 8 int8, per launch: a
+// 4 MiB product 8.2 us against 10.3 us on the split-K kernel, 16 MiB equal
+// (12.3 us), 24 MiB 15.9 against 14.4 us, 112 MiB 45 against 28.7 us.
+constexpr int64_t kGemvHalvesMaxWeightBytes = 8ll << 20;          // weight-only: 2K bytes of staged x beside the ring
 constexpr int kGemvUnits = 16;                  // units per stage (the MMA's 16 A rows)
 constexpr int kGemvSwCache = 2048;              // row scales kept in shared memory
 constexpr uint32_t kBarConsumers = 1;           // named barrier of the consumer warps
@@ -77,6 +85,7 @@ struct GemvProblem {
   const float* sw;
   uint16_t* y;
   int64_t N;
+  int M;  // tokens of this product (at most the launch's M)
 };
 
 struct GemvParams {
@@ -84,7 +93,7 @@ struct GemvParams {
   int cta0[kGemvMaxGroup + 1];  // CTAs [cta0[j], cta0[j+1]) run product j
   int nprob;
   int64_t K;
-  int M;               // tokens: 1 to 4 (extra tokens ride on the MMA's B columns)
+  int M;               // tokens: 1 to 4 (extra tokens ride on the MMA's B columns); the largest product's
   int rows_per_stage;  // 2 kRs whole rows per ring stage (kRs = 1, 2 or 4: the kernel's template)
   int stage_bytes;     // R_s * K rounded up to 128
   int stages;          // ring depth
@@ -209,6 +218,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   const float* psw = p.prob[0].sw;
   uint16_t* py = p.prob[0].y;
   int64_t N = p.prob[0].N;
+  int Mt = p.prob[0].M;  // this product's tokens (padding tokens past them are zero)
   int cta_lo = p.cta0[0], cta_hi = p.cta0[1];
 #pragma unroll
   for (int j = 1; j < kGemvMaxGroup; ++j)
@@ -219,6 +229,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
       psw = p.prob[j].sw;
       py = p.prob[j].y;
       N = p.prob[j].N;
+      Mt = p.prob[j].M;
       cta_lo = p.cta0[j];
       cta_hi = p.cta0[j + 1];
     }
@@ -374,7 +385,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   } else if constexpr (kWO) {
     // Weight-only, kM tokens side by side: one absmax pass and one staging
     // pass for all of them, each token with its own power of two.  Padding
-    // tokens (past p.M) read nothing and stage zeros.
+    // tokens (past Mt) read nothing and stage zeros.
     const int nchunk8 = (int)(K / 8);
     const uint4* xg = reinterpret_cast<const uint4*>(px);  // token tok at tok * nchunk8
     const int64_t xs2 = 2 * xstride;                        // bytes between staged tokens
@@ -384,7 +395,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     for (int c = tid; c < nchunk8; c += kGemvConsumers) {
 #pragma unroll
       for (int tok = 0; tok < kM; ++tok) {
-        const uint4 v = tok < p.M ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
+        const uint4 v = tok < Mt ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
         amax[tok] = fmaxf(amax[tok], absmax_chunk8(v));
       }
     }
@@ -412,7 +423,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     for (int c = tid; c < nchunk8; c += kGemvConsumers) {
 #pragma unroll
       for (int tok = 0; tok < kM; ++tok) {
-        const uint4 v = tok < p.M ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
+        const uint4 v = tok < Mt ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
         const float u = up[tok];
         reinterpret_cast<uint4*>(qx_s + tok * xs2)[c] =
             make_uint4(f32x2_to_f16x2(bf16_lo(v.x) * u, bf16_hi(v.x) * u),
@@ -510,7 +521,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   } else {
     // kM tokens side by side: one absmax pass and one code pass for all of
     // them, every token's loads in flight together.  Padding tokens (past
-    // p.M) read nothing and get zero codes and scales.
+    // Mt) read nothing and get zero codes and scales.
     const int nchunk8 = (int)(K / 8);  // 16-byte chunks of 8 bf16 per token
     const uint4* xg = reinterpret_cast<const uint4*>(px);  // token tok at tok * nchunk8
     if constexpr (kBlock) {
@@ -523,7 +534,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 #pragma unroll
         for (int b = 0; b < kB; ++b) {
           const int f = base + b * kGemvConsumers + tid;
-          v[b] = f < total && f / nchunk8 < p.M ? __ldg(xg + f) : make_uint4(0, 0, 0, 0);
+          v[b] = f < total && f / nchunk8 < Mt ? __ldg(xg + f) : make_uint4(0, 0, 0, 0);
         }
         float sc[kB];
 #pragma unroll
@@ -562,8 +573,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         uint4 v[2 * kM];
 #pragma unroll
         for (int tok = 0; tok < kM; ++tok) {
-          v[2 * tok] = tok < p.M ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
-          v[2 * tok + 1] = tok < p.M && c2 < nchunk8 ? __ldg(xg + tok * nchunk8 + c2) : make_uint4(0, 0, 0, 0);
+          v[2 * tok] = tok < Mt ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
+          v[2 * tok + 1] = tok < Mt && c2 < nchunk8 ? __ldg(xg + tok * nchunk8 + c2) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int tok = 0; tok < kM; ++tok)
@@ -585,7 +596,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         const float sc = a / (kInt8 ? 127.0f : 448.0f);
         if (tid == 0) sx_s[tok] = sc;
         dv[tok] = make_divisor(sc);
-        if (tok < p.M) all_fast = all_fast && dv[tok].fast;
+        if (tok < Mt) all_fast = all_fast && dv[tok].fast;
       }
       // one uniform branch for all tokens: the IEEE path gives the same codes
       auto emit_all = [&](auto fast) {
@@ -595,11 +606,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
           uint4 v[kM];
 #pragma unroll
           for (int tok = 0; tok < kM; ++tok)
-            v[tok] = tok < p.M ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
+            v[tok] = tok < Mt ? __ldg(xg + tok * nchunk8 + c) : make_uint4(0, 0, 0, 0);
 #pragma unroll
           for (int tok = 0; tok < kM; ++tok)
             reinterpret_cast<uint2*>(qx_s + tok * xstride)[c] =
-                tok < p.M ? quant_chunk8<kInt8, kFast>(v[tok], dv[tok]) : make_uint2(0, 0);
+                tok < Mt ? quant_chunk8<kInt8, kFast>(v[tok], dv[tok]) : make_uint2(0, 0);
         }
       };
       if (all_fast)
@@ -617,12 +628,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   if (!kWO && blockIdx.x == 0 && (p.dbg.qx || p.dbg.sx)) {  // product 0's first CTA
     // [token, K] codes and [token, groups] scales; rows of K bytes (K % 16 == 0)
     const int ns = kBlock ? (int)KB : 1;
-    for (int64_t c = tid; c < (kM == 1 ? 1 : p.M) * (K / 16); c += kGemvConsumers) {
+    for (int64_t c = tid; c < (kM == 1 ? 1 : Mt) * (K / 16); c += kGemvConsumers) {
       const int64_t tok = kM == 1 ? 0 : c / (K / 16), cc = kM == 1 ? c : c % (K / 16);
       if (p.dbg.qx)
         reinterpret_cast<uint4*>(p.dbg.qx)[c] = reinterpret_cast<const uint4*>(qx_s + tok * xstride)[cc];
     }
-    for (int i = tid; i < (kM == 1 ? 1 : p.M) * ns; i += kGemvConsumers)
+    for (int i = tid; i < (kM == 1 ? 1 : Mt) * ns; i += kGemvConsumers)
       if (p.dbg.sx) p.dbg.sx[i] = sx_s[i];
   }
 
@@ -835,7 +846,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 #pragma unroll
           for (int o = 1; o < kQ; o <<= 1) vf += __shfl_xor_sync(0xffffffffu, vf, o);
         }
-        if ((kM == 1 ? wg == 0 : otok < p.M) && u % kQ == 0 && r < nr) {
+        if ((kM == 1 ? wg == 0 : otok < Mt) && u % kQ == 0 && r < nr) {
           const int64_t n = r0 + r;
           const int64_t o = otok * N + n;  // y and debug index [token, row]
           float yv;
@@ -866,6 +877,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 }
 
 int gemv_max_k() { return kGemvMaxK; }
+
+bool gemv_token_halves_pay(int64_t M, int64_t K, const int64_t* Ns, int count) {
+  if (M < 5 || M > 8 || K > kGemvMaxK4 || count < 1 || 2 * count > kGemvMaxGroup) return false;
+  int64_t bytes = 0;
+  for (int j = 0; j < count; ++j) bytes += Ns[j] * K;
+  return bytes <= kGemvHalvesMaxWeightBytes;
+}
 int gemv_weight_only_max_k() { return (int)kGemvMaxKWO; }
 
 template <ql_scheme S, int kRs, int kSteps, int kM, bool kWO = false>
@@ -940,7 +958,8 @@ int gemv_max_k_tokens(int64_t M) {
 // cudaErrorInvalidValue / InvalidConfiguration for shapes the kernel does not
 // take.
 static cudaError_t gemv_setup(GemvParams& p, int64_t M, const ql_gemv_problem* probs, int count,
-                              int64_t K, int xelem, int num_sms, int* grid, size_t* smem) {
+                              int64_t K, int xelem, int num_sms, int* grid, size_t* smem,
+                              const int* Ms = nullptr) {
   if (count < 1 || count > kGemvMaxGroup) return cudaErrorInvalidValue;
   p.nprob = count;
   p.K = K;
@@ -970,7 +989,7 @@ static cudaError_t gemv_setup(GemvParams& p, int64_t M, const ql_gemv_problem* p
     p.prob[j] = GemvProblem{probs[j].x ? probs[j].x : static_cast<const uint16_t*>(probs[j].qx),
                             probs[j].x ? nullptr : probs[j].sx,
                             static_cast<const uint8_t*>(probs[j].wq), probs[j].sw, probs[j].y,
-                            probs[j].N};
+                            probs[j].N, Ms ? Ms[j] : (int)M};
     cap[j] = (probs[j].N + p.rows_per_stage - 1) / p.rows_per_stage;
     g[j] = 1;
     ++used;
@@ -1029,6 +1048,35 @@ cudaError_t launch_gemv_grouped(ql_scheme scheme, const ql_gemv_problem* probs, 
   int grid = 0;
   size_t smem = 0;
   cudaError_t e = gemv_setup(p, M, probs, count, K, 1, num_sms, &grid, &smem);
+  if (e != cudaSuccess) return e;
+  p.dbg = ql_debug{nullptr, nullptr, nullptr, nullptr};
+  p.status = status;
+  p.stall = 0;
+  return launch_gemv_scheme<false>(scheme, p, grid, smem, st);
+}
+
+cudaError_t launch_gemv_token_halves(ql_scheme scheme, const uint16_t* x, const ql_gemm_problem* probs,
+                                     int count, int64_t M, int64_t K, int num_sms, DevStatus* status,
+                                     cudaStream_t st) {
+  if (M < 5 || M > 8 || K > kGemvMaxK4 || count < 1 || 2 * count > kGemvMaxGroup) return cudaErrorInvalidValue;
+  // Each product becomes two products of the same weights: tokens 0-3 and
+  // tokens 4 .. M-1.  The two get the same number of CTAs, so CTA b of each
+  // streams the same weight rows at about the same time and the second read
+  // of a row is mostly served by L2 (the SMs still take in the weight bytes
+  // twice: worth it only while the launch's fixed cost dominates).
+  ql_gemv_problem g[kGemvMaxGroup];
+  int Ms[kGemvMaxGroup];
+  for (int j = 0; j < count; ++j) {
+    const ql_gemm_problem& q = probs[j];
+    g[2 * j] = ql_gemv_problem{x, nullptr, nullptr, q.wq, q.sw, q.y, q.N};
+    g[2 * j + 1] = ql_gemv_problem{x + 4 * K, nullptr, nullptr, q.wq, q.sw, q.y + 4 * q.N, q.N};
+    Ms[2 * j] = 4;
+    Ms[2 * j + 1] = (int)M - 4;
+  }
+  GemvParams p;
+  int grid = 0;
+  size_t smem = 0;
+  cudaError_t e = gemv_setup(p, 4, g, 2 * count, K, 1, num_sms, &grid, &smem, Ms);
   if (e != cudaSuccess) return e;
   p.dbg = ql_debug{nullptr, nullptr, nullptr, nullptr};
   p.status = status;

@@ -53,6 +53,15 @@ cudaError_t launch_gemv(ql_scheme scheme, const uint16_t* x, const void* wq, con
 // launch; K <= gemv_max_k_tokens(M).
 cudaError_t launch_gemv_grouped(ql_scheme scheme, const ql_gemv_problem* probs, int count, int64_t M,
                                 int64_t K, int num_sms, DevStatus* status, cudaStream_t st);
+// 5 <= M <= 8 tokens, K <= gemv_max_k_tokens(4), up to QL_GEMV_MAX_GROUP / 2
+// products on the same bf16 tokens x [M, K]: one GEMV launch in which each
+// product runs as two (tokens 0-3 and 4 .. M-1) over the same weights.
+// gemv_token_halves_pay: the shapes where that beats the split-K kernel (the
+// products' weights small enough for the launch's fixed cost to dominate).
+bool gemv_token_halves_pay(int64_t M, int64_t K, const int64_t* Ns, int count);
+cudaError_t launch_gemv_token_halves(ql_scheme scheme, const uint16_t* x, const ql_gemm_problem* probs,
+                                     int count, int64_t M, int64_t K, int num_sms, DevStatus* status,
+                                     cudaStream_t st);
 // 1 <= M <= 4 weight-only product: x stays bf16 (staged as exactly scaled f16),
 // W codes dequantized to f16 in registers, f32 sums; K <= gemv_weight_only_max_k().
 // Returns cudaErrorNotSupported for shapes whose staged tokens and two ring

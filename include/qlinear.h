@@ -234,7 +234,11 @@ size_t qlinear_weight_only_workspace_bytes(ql_scheme scheme, int64_t M, int64_t 
  * weights on the 128-row side, K split across the SMs).  Up to four tokens
  * (K <= 16384 for two, K <= 8192 for three or four) run instead on the
  * qlinear_gemv kernel, which carries them on its MMA's spare columns at the
- * weight traffic of one token; the result is the same.  Pages: W8A8
+ * weight traffic of one token; the result is the same.  Five to eight tokens
+ * with K <= 8192 on at most 8 MiB of weights (a k_proj-sized product) run on
+ * that kernel too, as two products of tokens 0-3 and 4..M-1 over the same
+ * weights in one launch, unless `dbg` asks for captures (the tensor-core
+ * kernel then runs).  Pages: W8A8
  * "Loading" (batches of at most 32 tokens on the tensor cores); Qwen3 FP8
  * "Loading" (same).
  * Activation quantization runs in the same call (a short quantize pass
@@ -370,8 +374,8 @@ size_t qlinear_gemm_grouped_workspace_bytes(ql_scheme scheme, const int64_t* Ns,
  * once, and the 128-row weight tiles of every product share the SM-balanced
  * K split, so that the small products (k and v: 4 MB of weights each) do not
  * pay a launch and a reduction of their own.  Up to four tokens within the
- * GEMV's K limits (as for qlinear_gemm_small) run as one grouped GEMV launch
- * instead.  Numerics of each product as qlinear_gemm_small.  Pages: as for
+ * GEMV's K limits, and five to eight on at most 8 MiB of weights in all (as
+ * for qlinear_gemm_small), run as one grouped GEMV launch instead.  Numerics of each product as qlinear_gemm_small.  Pages: as for
  * qlinear_gemm_small.
  *   x          device, bf16 [M,K] tokens, quantized in the call; or NULL with
  *   qx, sx     device, the tokens already quantized (codes [M,K], scales as

@@ -103,8 +103,9 @@ def test_committed_traffic_summaries_exist():
         wl = bench.workloads()[key]
         per_launch = bench.step_bytes(wl) / bench.dominant_launch_count(wl)
         if wl.bound == "hbm":
-            # the recorded DRAM traffic is within 1% of the algorithmic bytes (no re-reads)
-            assert bytes_per_launch == pytest.approx(per_launch, rel=0.01)
+            # the recorded DRAM traffic is within 1% of the algorithmic bytes (no re-reads),
+            # or within the ~50 KB every cold-cache launch adds (a 4 MB launch's 1%)
+            assert abs(bytes_per_launch - per_launch) <= max(0.01 * per_launch, 64 * 1024)
         else:
             # GEMMs: no operand re-read from HBM; y may still sit in L2 when the kernel ends
             assert 0.6 * per_launch <= bytes_per_launch <= 1.02 * per_launch

@@ -6,6 +6,11 @@ split tiles summed by their last contributor); the oracle runs the same
 definition.  The quantized tokens, their scales and (int8) the int32
 accumulators come back through the debug hook and must be bit-exact; bf16
 outputs are bit-exact for int8 and within 2^-7 |y| + 1e-3 for E4M3.
+
+Without the debug hook, five to eight tokens within K <= 8192 on at most 8 MiB
+of weights run on the GEMV kernel, each product as two products of four tokens
+or fewer over the same weights in one launch: those calls are checked on their
+outputs (and, int8, bit-equal to the split-K kernel's).
 """
 import numpy as np
 import pytest
@@ -79,7 +84,7 @@ def test_config_w8a8_k_proj_m8_seed0(cuda):
                                    # its K limits they take the split-K kernel
                                    (2, 1000, 4096), (2, 129, 16384), (2, 64, 16400), (3, 1001, 4096),
                                    (4, 777, 2064), (4, 300, 8192), (3, 64, 8208), (4, 130, 16),
-                                   # five to eight tokens of a small product: two GEMV passes
+                                   # five to eight tokens (with the debug hook: the split-K kernel)
                                    (5, 1000, 4096), (7, 129, 8192), (8, 4096, 4096), (6, 64, 8208),
                                    (8, 4100, 4096)])
 def test_small_shapes_full_compare(cuda, scheme, M, N, K):
@@ -148,3 +153,87 @@ def test_forward_dispatch_small_m(cuda, scheme):
         assert np.array_equal(bits(y), ry)
     else:
         assert_y_close(bits(y), ry, "forward small M")
+
+
+def _run_plain(scheme, M, N, K, seed=0, outliers=None, tag="plain", sample=None):
+    """The call without the debug hook; y (and a canary past it) against the
+    oracle.  Returns the output bits."""
+    if outliers is None:
+        outliers = synthetic.outlier_count(K) if scheme != ql.FP8_E4M3_BLOCK128 else 0
+    x = synthetic.make_x(M, K, seed=seed, tag=f"{tag}-x", outliers=outliers)
+    w = synthetic.make_w(N, K, seed=seed, tag=f"{tag}-w")
+    wq, sw = oracle.quantize_weight(scheme, w)
+    ws = ql.new_workspace(ql.workspace_bytes(scheme, M, N, K))
+    ypad = torch.full((M * N + 64,), -3.0, dtype=torch.bfloat16, device="cuda")
+    y = ypad[:M * N].view(M, N)
+    ql.gemm_small(scheme, bf16_dev(x), u8_dev(wq), f32_dev(sw), ws, y=y)
+    st, detail = ql.device_status()
+    assert st == 0, f"device status {st} detail {detail:#x}"
+    assert np.all(bits(ypad[M * N:]) == bits(torch.tensor([-3.0], dtype=torch.bfloat16))[0]), "wrote past y"
+    gy = bits(y)
+    what = f"small {scheme} {M}x{N}x{K} (no debug hook)"
+    if sample is None:
+        ry = oracle.forward(scheme, x, wq, sw)
+        if scheme == ql.W8A8_INT8_ROW:
+            assert np.array_equal(gy, ry), what + ": int8 outputs must be bit-exact"
+        else:
+            assert_y_close(gy, ry, what)
+    else:
+        rqx, rsx = oracle.quantize_act(scheme, x)
+        rng = np.random.default_rng(seed + 11)
+        pm = np.concatenate([rng.integers(0, M, sample), np.full(N, M - 1), np.full(N, 4 % M)])
+        pn = np.concatenate([rng.integers(0, N, sample), np.arange(N), np.arange(N)])
+        ry = oracle.linear_sampled(scheme, rqx, rsx, wq, sw, pm, pn)
+        if scheme == ql.W8A8_INT8_ROW:
+            assert np.array_equal(gy[pm, pn], ry), what
+        else:
+            assert_y_close(gy[pm, pn], ry, what + " sampled")
+    return gy
+
+
+def test_config_w8a8_k_proj_m8_seed0_plain(cuda):
+    """The same product without the debug hook (the GEMV kernel, two 4-token
+    halves): every output bit-exact."""
+    _run_plain(ql.W8A8_INT8_ROW, 8, 1024, 4096, seed=0, outliers=8, tag="cfg0")
+
+
+@pytest.mark.parametrize("M", [5, 6, 7, 8])
+@pytest.mark.parametrize("scheme,N,K", [(ql.W8A8_INT8_ROW, 1000, 4096), (ql.W8A8_INT8_ROW, 8, 8192),
+                                        (ql.W8A8_INT8_ROW, 4100, 48), (ql.W8A8_INT8_ROW, 64, 8208),
+                                        (ql.W8A8_INT8_ROW, 2048, 4096), (ql.W8A8_INT8_ROW, 2056, 4096),
+                                        (ql.FP8_E4M3_ROW, 129, 4096), (ql.FP8_E4M3_ROW, 520, 8192),
+                                        (ql.FP8_E4M3_ROW, 16, 272),
+                                        (ql.FP8_E4M3_BLOCK128, 1024, 4096), (ql.FP8_E4M3_BLOCK128, 128, 8192),
+                                        (ql.FP8_E4M3_BLOCK128, 384, 8320)])
+def test_five_to_eight_tokens_full_compare(cuda, M, scheme, N, K):
+    """Ragged N (partial stages, a product smaller than one stage per CTA), K at
+    and past the GEMV's four-token limit (8208, 8320: the split-K kernel),
+    weights of exactly 8 MiB (2048 x 4096: the GEMV) and just past it (2056 x
+    4096: the split-K kernel); int8 outputs also bit-equal to the split-K
+    kernel's (the debug-hook call)."""
+    gy = _run_plain(scheme, M, N, K, seed=M, tag=f"t58.{N}.{K}", outliers=3)
+    if scheme == ql.W8A8_INT8_ROW:
+        x = synthetic.make_x(M, K, seed=M, tag=f"t58.{N}.{K}-x", outliers=3)
+        w = synthetic.make_w(N, K, seed=M, tag=f"t58.{N}.{K}-w")
+        wq, sw = oracle.quantize_weight(scheme, w)
+        dbg = ql.Debug(acc_i32=torch.empty((M, N), dtype=torch.int32, device="cuda"))
+        ws = ql.new_workspace(ql.workspace_bytes(scheme, M, N, K))
+        y = ql.gemm_small(scheme, bf16_dev(x), u8_dev(wq), f32_dev(sw), ws, debug=dbg)
+        torch.cuda.synchronize()
+        assert np.array_equal(bits(y), gy), "GEMV route and split-K kernel differ"
+
+
+@pytest.mark.parametrize("M", [5, 8])
+@pytest.mark.parametrize("scheme", [ql.W8A8_INT8_ROW, ql.FP8_E4M3_ROW])
+@pytest.mark.parametrize("name,N,K", synthetic.LLAMA31_8B)
+def test_five_to_eight_tokens_llama_full_size(cuda, M, scheme, name, N, K):
+    """The Llama-3.1-8B layer at M = 5 and 8 without the debug hook (down_proj,
+    K = 14336, takes the split-K kernel): int8 every output up to 4096 rows,
+    else sampled outputs plus the last token's and the fifth token's rows."""
+    full = scheme == ql.W8A8_INT8_ROW and N <= 4096
+    _run_plain(scheme, M, N, K, seed=M, tag=f"llama58.{name}", sample=None if full else 1500)
+
+
+@pytest.mark.parametrize("name,N,K", synthetic.QWEN3_8B)
+def test_five_to_eight_tokens_qwen_block(cuda, name, N, K):
+    _run_plain(ql.FP8_E4M3_BLOCK128, 8, N, K, seed=8, tag=f"qwen58.{name}", sample=1000)
