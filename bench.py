@@ -19,9 +19,10 @@ Other workloads (``--workload``), same JSON line:
                 and FP8 per-row weights): 14 weight-only GEMVs, GB/s
 
 Legs of the line:
-  value     device time of K steps, each one CUDA-graph replay of the step's
-            launches (the pages decode under CUDA graphs); inputs resident in
-            HBM; decode and small-M steps stream more than L2 every step.
+  value     device time of K steps replayed from CUDA graphs (the pages decode
+            under CUDA graphs), 16 or more consecutive steps per graph so that
+            steps chain like a model's layers; inputs resident in HBM; decode
+            and small-M steps stream more than L2 every step.
   e2e       the same metric through the public API (``forward``) with the
             step's activations copied host->device from pinned memory and the
             outputs read back device->host every step (captured in a graph,
@@ -500,6 +501,9 @@ class Runner:
                     ql.gemv(p.scheme, i["xs"][t], wq, sw, y=i["ys"][t])
 
     def capture(self, fn, stream):
+        """Graphs of fn(t) for every input copy t, and one graph of a chain of
+        consecutive steps (a whole number of copy cycles, at least 16 steps):
+        see Steps."""
         torch = self.torch
         with torch.cuda.stream(stream):
             fn(0)  # warms the launch path (device info, attributes) before capture
@@ -510,7 +514,12 @@ class Runner:
             with torch.cuda.graph(g, stream=stream):
                 fn(t)
             graphs.append(g)
-        return graphs
+        n = self.copies * max(1, -(-STEP_CHAIN // self.copies))
+        chain = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(chain, stream=stream):
+            for t in range(n):
+                fn(t % self.copies)
+        return Steps(graphs, chain, n)
 
     def e2e_graph(self, stream):
         """H2D of every group's input (pinned host -> device: bf16 x, or codes
@@ -643,12 +652,42 @@ def workload_config(wl):
             "amount_per_step": step_amount(wl)}
 
 
-def timed(torch, stream, graphs, steps):
+# Steps replayed as one graph: a decode forward runs its layers inside one graph,
+# where each kernel's start overlaps the previous one's end (programmatic
+# dependent launch); a graph boundary per step would add a full drain and a
+# graph launch that the model does not pay.
+STEP_CHAIN = 16
+
+
+class Steps:
+    """Step i runs input copy i % copies: `chain` consecutive steps from a
+    multiple of `chain` (a multiple of the copies) replay as one captured graph
+    of those steps, any other step as the graph of its copy alone.  Every
+    kernel reads and writes global memory only after its grid-dependency wait
+    (before it: weight loads and shared-memory set-up), so a step's first
+    kernels may overlap the previous step's last ones exactly as the kernels
+    inside a step overlap."""
+
+    def __init__(self, singles, chain_graph, chain):
+        self.singles, self.chain_graph, self.chain = singles, chain_graph, chain
+
+    def run(self, i0, n):
+        i, end = i0, i0 + n
+        while i < end:
+            if i % self.chain == 0 and i + self.chain <= end:
+                self.chain_graph.replay()
+                i += self.chain
+            else:
+                self.singles[i % len(self.singles)].replay()
+                i += 1
+
+
+def timed(torch, stream, steps_graphs, steps):
+    """Device time (ms) of `steps` steps from step 0, CUDA events on the stream."""
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for i in range(steps):
-            graphs[i % len(graphs)].replay()
+        steps_graphs.run(0, steps)
         e1.record(stream)
     e1.synchronize()
     return e0.elapsed_time(e1)
@@ -889,8 +928,7 @@ def per_product_times(torch, run, stream, wl, peak, scale, reps=50):
             run.dominant_group(g, t)
         graphs = run.capture(fn, stream)
         with torch.cuda.stream(stream):
-            for i in range(5):
-                graphs[i % len(graphs)].replay()
+            graphs.run(0, graphs.chain + 5)  # every graph warm
         ms = timed(torch, stream, graphs, reps) / reps
         amount = sum(i["amount"] for i in g["items"])
         if wl.unit == "GB/s":  # a grouped launch reads its shared input once
@@ -913,10 +951,11 @@ def measure(torch, ql, synthetic, wl, args, steps, warmup, world, rank, barrier,
     run = Runner(torch, ql, synthetic, wl)
     graphs = run.capture(run.step, stream)
 
-    # ---- timed region: K steps, one graph replay each
+    # ---- timed region: K steps (chains of steps captured as one graph)
     with torch.cuda.stream(stream):
-        for i in range(warmup):
-            graphs[i % len(graphs)].replay()
+        graphs.run(0, warmup)
+        if warmup < graphs.chain:
+            graphs.chain_graph.replay()  # the chain graph warm too (untimed)
     stream.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -934,8 +973,7 @@ def measure(torch, ql, synthetic, wl, args, steps, warmup, world, rank, barrier,
     dgraphs = run.capture(run.dominant, stream)
     dsteps = max(3, min(steps, 500))
     with torch.cuda.stream(stream):
-        for i in range(min(warmup, 10)):
-            dgraphs[i % len(dgraphs)].replay()
+        dgraphs.run(0, dgraphs.chain + min(warmup, 10))
     d_ms = timed(torch, stream, dgraphs, dsteps)
     n_dom = run.dominant_launches
     per_launch_amount = run.step_amount / n_dom
@@ -998,7 +1036,9 @@ def measure(torch, ql, synthetic, wl, args, steps, warmup, world, rank, barrier,
                           f"{run.copies} sets of weights/activations/outputs, "
                           f"{run.copies * sum(wl.bytes_touched(p) for p in wl.products) / 1e6:.0f} MB "
                           f"touched per cycle ({weight_bytes / 1e6:.0f} MB of weights per step); no flush"),
-                   "timing": "one CUDA graph replay per step, CUDA events on the launch stream"},
+                   "timing": (f"steps replayed {STEP_CHAIN}+ at a time as one captured CUDA graph "
+                              "(each step's kernels overlap the previous step's by programmatic dependent "
+                              "launch, as layers inside one model graph), CUDA events on the launch stream")},
         "roofline": roofline,
         **({"per_product": per_product} if per_product else {}),
         "parity": parity,
