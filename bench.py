@@ -337,7 +337,7 @@ TRAFFIC = {
     "kproj": (4325504, "c19c7146a24ad7ed", "profiles/gemv_kproj_dram.md"),
     "prefill": (75848448, "87b077ff18efb3b1", "profiles/gemm_prefill_int8_dram.md"),
     "qwen-prefill": (52170240, "87b077ff18efb3b1", "profiles/gemm_qwen_prefill_block_dram.md"),
-    "small": (55263000, "82bb5f3ca16b177a", "profiles/gemm_small_dram.md"),
+    "small": (55263000, "6a8d32a8ea860c98", "profiles/gemm_small_dram.md"),
 }
 
 

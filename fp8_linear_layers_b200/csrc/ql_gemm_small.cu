@@ -475,8 +475,9 @@ size_t gemm_small_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_
 
 size_t gemm_small_zeroed_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms) {
   (void)num_sms;
-  // the GEMV route (up to four tokens) does not touch the workspace
-  if (K <= gemv_max_k_tokens(M)) return 0;
+  // the GEMV routes (up to four tokens; five to eight on small weights) do
+  // not touch the workspace
+  if (K <= gemv_max_k_tokens(M) || gemv_token_halves_pay(M, K, &N, 1)) return 0;
   return small_layout(scheme, M, (N + 127) / 128, K).zeroed;
 }
 

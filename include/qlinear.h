@@ -456,7 +456,8 @@ const char* qlinear_last_cuda_error(void);
  *     any stream capture.
  *   - All calls share the one array and it keeps the previous call's
  *     contents: each call clears the sums and counters that must start at zero (an
- *     asynchronous memset on `stream`).  Calls whose GPU work overlaps --
+ *     asynchronous memset on `stream`; none when the shape runs on the GEMV
+ *     kernel, which uses no scratch).  Calls whose GPU work overlaps --
  *     on different streams, or from different threads -- race on the array
  *     and give wrong results; serialise them. */
 ql_status qlinear_gemm_small_noalloc(ql_scheme scheme, const uint16_t* x, const void* wq,
