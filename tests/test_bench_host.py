@@ -1,6 +1,8 @@
 """Host-side logic of bench.py (CPU only): the workloads' algorithmic amounts
-against the shape totals, the oracle sample's description, and the rule that a
-DRAM-traffic figure is reported only for the kernel sources it was taken on."""
+against the shape totals, the oracle sample's description, the rule that a
+DRAM-traffic figure is reported only for the kernel sources it was taken on,
+the routing that decides each step's launch count, and the replay of exactly
+K steps from chained step graphs."""
 import os
 import sys
 
@@ -164,3 +166,44 @@ def test_parity_sample_against_oracle_outputs():
     items[4]["ys"][0][0, 3] = items[4]["ys"][0][0, 3] * 1.5 + 1.0
     rep = bench.parity_sample(_FakeRun(items), torch, rows=8)
     assert not rep["within_tolerance"] and rep["max_abs_err"] > 0.5
+
+
+class _FakeGraph:
+    """Stands in for a captured CUDA graph: records which steps a replay runs."""
+
+    def __init__(self, log, steps):
+        self.log, self.steps = log, steps
+
+    def replay(self):
+        self.log.extend(self.steps)
+
+
+@pytest.mark.parametrize("copies,n", [(2, 300), (2, 7), (59, 200), (3, 16), (2, 0), (5, 1)])
+def test_chained_steps_replay_exactly_k_steps_in_copy_order(copies, n):
+    """Steps.run(0, n) replays n steps, step i on input copy i % copies, whether
+    a step comes from the chain graph or from its copy's own graph."""
+    chain = copies * max(1, -(-bench.STEP_CHAIN // copies))
+    log = []
+    singles = [_FakeGraph(log, [t]) for t in range(copies)]
+    chained = _FakeGraph(log, [t % copies for t in range(chain)])
+    bench.Steps(singles, chained, chain).run(0, n)
+    assert log == [i % copies for i in range(n)]
+
+
+def test_five_to_eight_tokens_route_follows_the_weight_bytes():
+    """The GEMV takes 5-8 tokens only when the launch's weights are at most
+    8 MiB (the library's rule); the launch count follows (one launch instead of
+    a quantization launch and the split-K kernel)."""
+    P = bench.Product
+    kproj = bench.workloads()["kproj"]
+    p = kproj.products[0]
+    assert bench.gemv_route(p.M, p.K, [p])
+    assert kproj.kernel == "ql::gemv_kernel"
+    assert bench.gemv_route(8, 4096, [P("x", bench.INT8, 8, 2048, 4096, 0)])
+    assert not bench.gemv_route(8, 4096, [P("x", bench.INT8, 8, 2056, 4096, 0)])
+    assert not bench.gemv_route(8, 8208, [P("x", bench.INT8, 8, 8, 8208, 0)])
+    assert not bench.gemv_route(9, 4096, [P("x", bench.INT8, 9, 8, 4096, 0)])
+    assert bench.gemv_route(4, 8192) and not bench.gemv_route(4, 8208)
+    # the small-M workload: at M = 8 every launch carries more than 8 MiB of weights
+    small = bench.workloads()["small"]
+    assert small.kernel == "ql::gemm_small_kernel"
