@@ -105,7 +105,8 @@ size_t gemm_small_workspace_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_
 size_t gemm_small_zeroed_bytes(ql_scheme scheme, int64_t M, int64_t N, int64_t K, int num_sms);
 // A group of 1..QL_GEMM_MAX_GROUP products on the same tokens (their N in
 // Ns): one quantization of the tokens and one launch (up to four tokens within
-// the GEMV's K limits: one grouped GEMV launch, no workspace used).
+// the GEMV's K limits, or five to eight on at most 8 MiB of weights with no
+// debug captures: one grouped GEMV launch, no workspace used).
 size_t gemm_small_group_workspace_bytes(ql_scheme scheme, int64_t M, const int64_t* Ns, int count, int64_t K);
 cudaError_t launch_gemm_small_group(ql_scheme scheme, const uint16_t* x, const ql_gemm_problem* probs, int count,
                                     int64_t M, int64_t K, void* workspace, size_t ws_bytes, const ql_debug* dbg,
