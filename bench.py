@@ -333,11 +333,11 @@ KERNEL_SOURCES = {"ql::gemv_kernel": _GEMV_SOURCES, "ql::gemv_kernel (weight-onl
                   "ql::gemm_small_kernel": _SMALL_SOURCES}
 TRAFFIC = {
     # workload: (bytes per launch, kernel source hash, summary file)
-    "decode": (54660384, "c19c7146a24ad7ed", "profiles/gemv_decode_dram.md"),
-    "kproj": (4325504, "c19c7146a24ad7ed", "profiles/gemv_kproj_dram.md"),
+    "decode": (54660384, "10803db7fb9f04b9", "profiles/gemv_decode_dram.md"),
+    "kproj": (4325504, "10803db7fb9f04b9", "profiles/gemv_kproj_dram.md"),
     "prefill": (75848448, "87b077ff18efb3b1", "profiles/gemm_prefill_int8_dram.md"),
     "qwen-prefill": (52170240, "87b077ff18efb3b1", "profiles/gemm_qwen_prefill_block_dram.md"),
-    "small": (55263000, "6a8d32a8ea860c98", "profiles/gemm_small_dram.md"),
+    "small": (55263000, "bb1a70d5446e5ea7", "profiles/gemm_small_dram.md"),
 }
 
 

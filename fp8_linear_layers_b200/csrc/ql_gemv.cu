@@ -62,7 +62,7 @@ constexpr int64_t kGemvStashMaxK = 16384;       // one token's bf16 x parked in 
 constexpr int kGemvMaxK = 32768;
 constexpr int64_t kGemvMaxK2 = 16384;           // two tokens: units of at most 64 windows
 constexpr int64_t kGemvMaxK4 = 8192;            // three or four tokens: stages of 8 rows
-constexpr int64_t kGemvMaxKWO = 16384;
+constexpr int64_t kGemvMaxKWO = 16384;          // weight-only: 2K bytes of staged x beside the ring
 // Five to eight tokens run on this kernel as two products of up to four
 // tokens over the same weights when the launch's weights take at most this
 // many bytes.  The halves' SMs each take the weight bytes in, so a launch
@@ -70,7 +70,7 @@ constexpr int64_t kGemvMaxKWO = 16384;
 // reads under a full stream).  Measured on B200, M = 8 int8, per launch: a
 // 4 MiB product 8.2 us against 10.3 us on the split-K kernel, 16 MiB equal
 // (12.3 us), 24 MiB 15.9 against 14.4 us, 112 MiB 45 against 28.7 us.
-constexpr int64_t kGemvHalvesMaxWeightBytes = 8ll << 20;          // weight-only: 2K bytes of staged x beside the ring
+constexpr int64_t kGemvHalvesMaxWeightBytes = 8ll << 20;
 constexpr int kGemvUnits = 16;                  // units per stage (the MMA's 16 A rows)
 constexpr int kGemvSwCache = 2048;              // row scales kept in shared memory
 constexpr uint32_t kBarConsumers = 1;           // named barrier of the consumer warps
