@@ -35,12 +35,12 @@ def _layer(scheme, shapes, M):
     return ws, ks
 
 
-@pytest.mark.parametrize("scheme,model", [(ql.W8A8_INT8_ROW, "llama"), (ql.FP8_E4M3_ROW, "llama"),
-                                          (ql.FP8_E4M3_BLOCK128, "qwen")])
-@pytest.mark.parametrize("M", [1, 8, 32])
+# the E4M3 row scheme at M = 1 and 8 (M = 32 runs the kernels W8A8 runs there)
+@pytest.mark.parametrize("scheme,model,M", [(ql.W8A8_INT8_ROW, "llama", 1), (ql.W8A8_INT8_ROW, "llama", 8),
+                                            (ql.W8A8_INT8_ROW, "llama", 32), (ql.FP8_E4M3_ROW, "llama", 1),
+                                            (ql.FP8_E4M3_ROW, "llama", 8), (ql.FP8_E4M3_BLOCK128, "qwen", 1),
+                                            (ql.FP8_E4M3_BLOCK128, "qwen", 8), (ql.FP8_E4M3_BLOCK128, "qwen", 32)])
 def test_layer_in_one_cuda_graph(cuda, scheme, model, M):
-    if scheme == ql.FP8_E4M3_ROW and M == 32:
-        pytest.skip("the E4M3 row scheme is covered at M = 1 and 8")
     shapes = synthetic.LLAMA31_8B if model == "llama" else synthetic.QWEN3_8B
     ws, ks = _layer(scheme, shapes, M)
     d_w = {n: (u8_dev(wq), f32_dev(sw)) for n, (wq, sw) in ws.items()}
